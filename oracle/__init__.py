@@ -1,0 +1,221 @@
+"""CPU oracle of the FP8 W8A8 linear path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library never calls it and
+shares no code with it.  The arithmetic lives in ``fp8q_oracle.c`` (plain C,
+fp64 unless the definition fixes fp32); this module compiles it with gcc and
+marshals numpy arrays through ctypes.  ``exact.py`` holds an exact-rational
+brute-force GEMM used to pin the C GEMM on tiny shapes.
+
+All bf16 tensors cross this interface as ``numpy.uint16`` bit patterns; codes
+as ``numpy.uint8`` e4m3fn bytes; scales as ``numpy.float32``; GEMM references
+as ``numpy.float64``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp8q_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``fp8q_oracle.c`` into ``liboracle.so`` (gcc, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+               "-fno-fast-math", _SRC, "-o", _LIB + ".tmp", "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_bf16_round.argtypes = [ctypes.c_double]
+        lib.oracle_bf16_round.restype = ctypes.c_float
+        lib.oracle_scale.argtypes = [ctypes.c_float, ctypes.c_int]
+        lib.oracle_scale.restype = ctypes.c_float
+        lib.oracle_group_quant.argtypes = [P, i64, i64, i64, i64, ctypes.c_int, P, P, P]
+        lib.oracle_rmsnorm_quant.argtypes = [P, P, ctypes.c_float, i64, i64, i64, i64,
+                                             ctypes.c_int, P, P, P]
+        lib.oracle_silu_mul_quant.argtypes = [P, i64, i64, i64, i64, ctypes.c_int, P, P, P]
+        lib.oracle_scaled_mm_rows.argtypes = [P, P, P, ctypes.c_int, P, ctypes.c_int, i64, i64,
+                                              i64, P, i64, P, P]
+        lib.oracle_scaled_mm_blockwise_rows.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, P]
+        lib.oracle_e4m3_encode_array.argtypes = [P, i64, P]
+        lib.oracle_e4m3_decode_array.argtypes = [P, i64, P]
+        lib.oracle_bf16_round_array.argtypes = [P, i64, P]
+        lib.oracle_scale_array.argtypes = [P, i64, ctypes.c_int, P]
+        for f in ("oracle_group_quant", "oracle_rmsnorm_quant", "oracle_silu_mul_quant",
+                  "oracle_scaled_mm_rows", "oracle_scaled_mm_blockwise_rows",
+                  "oracle_e4m3_encode_array", "oracle_e4m3_decode_array",
+                  "oracle_bf16_round_array", "oracle_scale_array"):
+            getattr(lib, f).restype = None
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# --------------------------------------------------------------------- formats
+def e4m3_encode(v) -> np.ndarray:
+    """Saturating round-to-nearest-even e4m3fn codes of fp32 values."""
+    v = _c(v, np.float32)
+    out = np.empty(v.shape, np.uint8)
+    _load().oracle_e4m3_encode_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def e4m3_decode(c) -> np.ndarray:
+    c = _c(c, np.uint8)
+    out = np.empty(c.shape, np.float64)
+    _load().oracle_e4m3_decode_array(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def bf16_round(v) -> np.ndarray:
+    """Nearest-even bfloat16 of fp64 values, returned as float32."""
+    v = _c(v, np.float64)
+    out = np.empty(v.shape, np.float32)
+    _load().oracle_bf16_round_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def scale(amax, ue8m0: bool = False) -> np.ndarray:
+    a = _c(amax, np.float32)
+    out = np.empty(a.shape, np.float32)
+    _load().oracle_scale_array(_ptr(a), a.size, int(ue8m0), _ptr(out))
+    return out
+
+
+# ---------------------------------------------------------------- quant ops
+def _quant_out(M, L, g, want_y):
+    q = np.empty((M, L), np.uint8)
+    s = np.empty((M, L // g), np.float32)
+    y = np.empty((M, L), np.float32) if want_y else None
+    return q, s, y
+
+
+def _check_group(L, g):
+    if g <= 0 or L % g != 0:
+        raise ValueError(f"group size {g} does not divide row length {L}")
+
+
+def group_quant(x_bits: np.ndarray, group_size: int, ue8m0: bool = False, want_y: bool = False):
+    """per_token_group_fp8_quant (group_size=128) / per-token quant (group_size=K).
+
+    x_bits: uint16 bf16 bits [M, K].  Returns (q [M,K] uint8, s [M,K/g] f32[, y]).
+    """
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    _check_group(K, group_size)
+    q, s, y = _quant_out(M, K, group_size, want_y)
+    _load().oracle_group_quant(_ptr(x), M, K, K, group_size, int(ue8m0), _ptr(q), _ptr(s), _ptr(y))
+    return (q, s, y) if want_y else (q, s)
+
+
+def rmsnorm_quant(x_bits, w_bits, eps: float, group_size: int, ue8m0: bool = False,
+                  want_y: bool = False):
+    """rms_norm_dynamic_per_token_quant (g=H) / rms_norm_per_block_quant (g=128)."""
+    x = _c(x_bits, np.uint16)
+    w = _c(w_bits, np.uint16)
+    M, H = x.shape
+    assert w.shape == (H,)
+    _check_group(H, group_size)
+    q, s, y = _quant_out(M, H, group_size, want_y)
+    _load().oracle_rmsnorm_quant(_ptr(x), _ptr(w), ctypes.c_float(eps), M, H, H, group_size,
+                                 int(ue8m0), _ptr(q), _ptr(s), _ptr(y))
+    return (q, s, y) if want_y else (q, s)
+
+
+def silu_mul_quant(x_bits, group_size: int, ue8m0: bool = False, want_y: bool = False):
+    """silu_and_mul_dynamic_per_token_quant (g=I) / silu_and_mul_per_block_quant (g=128).
+
+    x_bits: [M, 2I] = [gate | up].
+    """
+    x = _c(x_bits, np.uint16)
+    M, I2 = x.shape
+    assert I2 % 2 == 0
+    I = I2 // 2
+    _check_group(I, group_size)
+    q, s, y = _quant_out(M, I, group_size, want_y)
+    _load().oracle_silu_mul_quant(_ptr(x), M, I, I2, group_size, int(ue8m0), _ptr(q), _ptr(s),
+                                  _ptr(y))
+    return (q, s, y) if want_y else (q, s)
+
+
+# ---------------------------------------------------------------------- GEMMs
+def _rows(M, rows):
+    if rows is None:
+        rows = np.arange(M, dtype=np.int64)
+    rows = _c(rows, np.int64)
+    assert rows.ndim == 1 and (rows.size == 0 or (rows.min() >= 0 and rows.max() < M))
+    return rows
+
+
+def scaled_mm(a_q, b_q, sa, sb, rows=None):
+    """fp64 reference of scaled_mm for the listed rows of A.
+
+    a_q [M,K] uint8, b_q [N,K] uint8, sa: [M] (per token) or [1] (per tensor),
+    sb: [N] (per channel) or [1] (per tensor).  Returns (y_ref, absdot), both
+    [len(rows), N] float64.
+    """
+    a = _c(a_q, np.uint8)
+    b = _c(b_q, np.uint8)
+    M, K = a.shape
+    N, K2 = b.shape
+    assert K == K2
+    sa = _c(sa, np.float32).reshape(-1)
+    sb = _c(sb, np.float32).reshape(-1)
+    assert sa.size in (1, M) and sb.size in (1, N)
+    rows = _rows(M, rows)
+    y = np.empty((rows.size, N), np.float64)
+    ad = np.empty((rows.size, N), np.float64)
+    _load().oracle_scaled_mm_rows(_ptr(a), _ptr(b), _ptr(sa), int(sa.size == M), _ptr(sb), int(sb.size == N), M, N, K,
+                                  _ptr(rows), rows.size, _ptr(y), _ptr(ad))
+    return y, ad
+
+
+def scaled_mm_blockwise(a_q, b_q, sa, sb, rows=None):
+    """fp64 reference of scaled_mm_blockwise for the listed rows of A.
+
+    sa [M, K/128] (row-major, one scale per 1x128 group of A), sb [N/128, K/128].
+    """
+    a = _c(a_q, np.uint8)
+    b = _c(b_q, np.uint8)
+    M, K = a.shape
+    N, K2 = b.shape
+    assert K == K2 and K % 128 == 0 and N % 128 == 0
+    sa = _c(sa, np.float32)
+    sb = _c(sb, np.float32)
+    assert sa.shape == (M, K // 128) and sb.shape == (N // 128, K // 128)
+    rows = _rows(M, rows)
+    y = np.empty((rows.size, N), np.float64)
+    ad = np.empty((rows.size, N), np.float64)
+    _load().oracle_scaled_mm_blockwise_rows(_ptr(a), _ptr(b), _ptr(sa), _ptr(sb), M, N, K,
+                                            _ptr(rows), rows.size, _ptr(y), _ptr(ad))
+    return y, ad
