@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 W8A8 linear path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--m M] [--impl reference]
+
+Workload: one Qwen3-8B-shaped MLP block (hidden 4096, intermediate 12288) on a
+batch of M tokens (default 2048), through both FP8 schemes.  One step runs every
+op of the path once:
+  per-token quant and 1x128-group quant of the block input x,
+  per-token chain:  rmsnorm_quant(g=H) -> scaled_mm gate_up [4096->24576]
+                    -> silu_mul_quant(g=I) -> scaled_mm down [12288->4096],
+  blockwise chain:  rmsnorm_quant(g=128) -> scaled_mm_blockwise gate_up
+                    -> silu_mul_quant(g=128) -> scaled_mm_blockwise down.
+x is heavy-tailed Student-t(3) with 1% outlier channels x20 (seeded); weights
+W ~ N(0, 0.02), quantized once per output channel / per 128x128 block.
+
+`value` is whole-job TFLOP/s (GEMM FLOPs of all ranks / max-over-ranks device
+time), inputs resident in HBM; each timed step is bracketed by CUDA events and
+followed by an untimed L2 flush.  `e2e` is the same metric through the public
+API with the activations copied from pinned host memory and both outputs copied
+back inside the timed region.  `--impl reference` times the CPU oracle on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+H, I = 4096, 12288
+EPS = 1e-6
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--m", type=int, default=2048)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    return ap.parse_args()
+
+
+def gemm_flops(M):
+    return 2 * (2 * M * H * 2 * I + 2 * M * I * H)     # two chains x (gate_up + down)
+
+
+def quant_bytes(M):
+    """Algorithmic HBM bytes of the six quant launches of one step: the bf16 input
+    read once, e4m3 codes and fp32 scales written once, the RMSNorm weight once."""
+    gq_tok = 2 * M * H + M * H + 4 * M
+    gq_grp = 2 * M * H + M * H + 4 * M * (H // 128)
+    rms_tok = 2 * M * H + M * H + 4 * M + 2 * H
+    rms_grp = 2 * M * H + M * H + 4 * M * (H // 128) + 2 * H
+    silu_tok = 4 * M * I + M * I + 4 * M
+    silu_grp = 4 * M * I + M * I + 4 * M * (I // 128)
+    return gq_tok + gq_grp + rms_tok + rms_grp + silu_tok + silu_grp
+
+
+def workload_config(M, n):
+    return {"workload": f"qwen3-8b-mlp-block-m{M}-per-token+blockwise",
+            "model": "Qwen3-8B-shaped MLP (hidden 4096, intermediate 12288)",
+            "global_batch": M * n, "tokens_per_gpu": M, "seq_len": None,
+            "parallelism": f"replicas{n}" if n > 1 else "single-gpu",
+            "l2": "flushed between timed steps (256 MiB write)"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out"))
+                                 else "", f".clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}",
+                 "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 7:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[3:7]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.remove(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ native arm
+def run_native(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import fp8_quantized_linear_rms_b200 as fq
+    import fp8q_inputs as inp
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    M = args.m
+    torch.manual_seed(1234 + rank)
+
+    # ---- inputs (seeded, synthetic) and weights, resident in HBM
+    x_host = torch.from_numpy(inp.heavy_tailed_bf16(2000 + rank, M, H).view("int16")).view(torch.bfloat16)
+    x_pinned = x_host.pin_memory()
+    x = x_host.to(dev)
+    w_norm = torch.from_numpy(inp.rms_weight_bf16(2001, H).view("int16")).view(torch.bfloat16).to(dev)
+
+    def make_weight(N, K, seed):
+        g = torch.Generator(device=dev).manual_seed(seed)
+        return (torch.randn(N, K, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+
+    def per_channel(W):
+        q, s = fq.fp8q_group_quant(W, W.shape[1])
+        return q, s.reshape(-1).contiguous()
+
+    def per_block(W):
+        N, K = W.shape
+        wb = W.float().view(N // 128, 128, K // 128, 128)
+        amax = wb.abs().amax(dim=(1, 3)).clamp_min(1e-10)
+        s = (amax / 448.0).float()
+        q = (wb / s[:, None, :, None]).clamp(-448, 448).to(torch.float8_e4m3fn).view(N, K)
+        return q.contiguous(), s.contiguous()
+
+    Wgu = make_weight(2 * I, H, 11)
+    Wd = make_weight(H, I, 12)
+    gu_pt, sgu_pt = per_channel(Wgu)
+    d_pt, sd_pt = per_channel(Wd)
+    gu_bw, sgu_bw = per_block(Wgu)
+    d_bw, sd_bw = per_block(Wd)
+    del Wgu, Wd
+
+    # ---- activation buffers
+    f8 = torch.float8_e4m3fn
+    q_tok = torch.empty((M, H), dtype=f8, device=dev)
+    s_tok = torch.empty((M, 1), dtype=torch.float32, device=dev)
+    q_grp = torch.empty((M, H), dtype=f8, device=dev)
+    s_grp = torch.empty((M, H // 128), dtype=torch.float32, device=dev)
+    qa = torch.empty((M, H), dtype=f8, device=dev)
+    sa = torch.empty((M, 1), dtype=torch.float32, device=dev)
+    h = torch.empty((M, 2 * I), dtype=torch.bfloat16, device=dev)
+    qh = torch.empty((M, I), dtype=f8, device=dev)
+    sh = torch.empty((M, 1), dtype=torch.float32, device=dev)
+    out_pt = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+    qa_b = torch.empty((M, H), dtype=f8, device=dev)
+    sa_b = torch.empty((H // 128, M), dtype=torch.float32, device=dev)
+    h_b = torch.empty((M, 2 * I), dtype=torch.bfloat16, device=dev)
+    qh_b = torch.empty((M, I), dtype=f8, device=dev)
+    sh_b = torch.empty((I // 128, M), dtype=torch.float32, device=dev)
+    out_b = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+    ws = {k: fq.make_workspace(M, N, K, bw, dev) for k, (N, K, bw) in
+          {"gu": (2 * I, H, False), "d": (H, I, False), "gub": (2 * I, H, True),
+           "db": (H, I, True)}.items()}
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev_gu = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def step(xin, gu_events=None):
+        fq.fp8q_group_quant(xin, H, q=q_tok, scales=s_tok)
+        fq.fp8q_group_quant(xin, 128, q=q_grp, scales=s_grp)
+        fq.fp8q_rmsnorm_quant(xin, w_norm, EPS, H, q=qa, scales=sa)
+        if gu_events:
+            gu_events[0].record(stream)
+        fq.fp8q_scaled_mm(qa, gu_pt, sa.view(-1), sgu_pt, y=h, workspace=ws["gu"])
+        if gu_events:
+            gu_events[1].record(stream)
+        fq.fp8q_silu_mul_quant(h, I, q=qh, scales=sh)
+        fq.fp8q_scaled_mm(qh, d_pt, sh.view(-1), sd_pt, y=out_pt, workspace=ws["d"])
+        fq.fp8q_rmsnorm_quant(xin, w_norm, EPS, 128, q=qa_b, scales=sa_b, scale_layout="group_major")
+        fq.fp8q_scaled_mm_blockwise(qa_b, gu_bw, sa_b, sgu_bw, a_scale_layout="group_major", y=h_b,
+                                    workspace=ws["gub"])
+        fq.fp8q_silu_mul_quant(h_b, 128, q=qh_b, scales=sh_b, scale_layout="group_major")
+        fq.fp8q_scaled_mm_blockwise(qh_b, d_bw, sh_b, sd_bw, a_scale_layout="group_major", y=out_b,
+                                    workspace=ws["db"])
+
+    LAUNCHES_PER_STEP = 10
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        step(x)
+    torch.cuda.synchronize()
+    st = fq.fp8q_last_device_status()
+    if st != fq.OK:
+        raise RuntimeError(f"device status after warm-up: {fq.fp8q_status_string(st)}")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- timed: device-resident inputs
+    sampler = ClockSampler(local_rank)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    gu_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(args.steps):
+        flush.zero_()                                   # untimed L2 flush
+        starts[i].record(stream)
+        step(x, gu_ev[i])
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    gu_ms = [a.elapsed_time(b) for a, b in gu_ev]
+    total_ms = sum(step_ms)
+
+    # ---- timed: end to end through host buffers
+    out_pinned = torch.empty((2, M, H), dtype=torch.bfloat16).pin_memory()
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    xd = torch.empty_like(x)
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e_starts[i].record(stream)
+        xd.copy_(x_pinned, non_blocking=True)
+        step(xd)
+        out_pinned[0].copy_(out_pt, non_blocking=True)
+        out_pinned[1].copy_(out_b, non_blocking=True)
+        e_ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))
+    st = fq.fp8q_last_device_status()
+    if st != fq.OK:
+        raise RuntimeError(f"device status after timing: {fq.fp8q_status_string(st)}")
+
+    # ---- max over ranks
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = t.tolist()
+
+    flops_step = gemm_flops(M)
+    value = flops_step * args.steps * world / (total_ms * 1e-3) / 1e12
+    e2e_value = flops_step * args.steps * world / (e2e_ms * 1e-3) / 1e12
+    gu_flops = 2 * M * H * 2 * I
+    gu_avg_s = statistics.mean(gu_ms) * 1e-3
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except Exception:
+        pass
+    bf16_sust = peaks.get("bf16_tflops_sustained")
+    if bf16_sust:
+        peak, peak_src = 2.0 * bf16_sust, "of measured: 2 x bf16 sustained (fp8:bf16 nominal 4.5:2.25)"
+    else:
+        peak, peak_src = 2.0 * 1400.0, "of fallback: 2 x 1.4 PF bf16 sustained"
+    achieved = gu_flops / gu_avg_s / 1e12
+    qb = quant_bytes(M)
+    line = {
+        "metric": "FP8 quant+scaled_mm TFLOP/s (Qwen3-8B MLP block, per-token + blockwise)",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic (seeded Student-t(3) activations, N(0,0.02) weights)",
+        "config": workload_config(M, world),
+        "quant_hbm_gbs": round(qb * args.steps / (total_ms * 1e-3) / 1e9, 1),
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": M * H * 2, "d2h_bytes_per_step": 2 * M * H * 2},
+        "roofline": {"bound": "tensor", "kernel": "scaled_mm gate_up (per-token, 2048x24576x4096)",
+                     "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "peak_source": peak_src, "traffic": None},
+        "clocks": clocks,
+    }
+    return line
+
+
+# ------------------------------------------------------------------ oracle arm
+def run_reference(args):
+    """The CPU oracle, as it stands, on a bounded sample of the same workload:
+    all quant ops on `rows` tokens and both GEMM chains on those rows."""
+    import numpy as np
+
+    import fp8q_inputs as inp
+    import oracle
+
+    M = args.m
+    rows = int(os.environ.get("FP8Q_REF_ROWS", "16"))
+    x = inp.heavy_tailed_bf16(2000, rows, H)
+    w = inp.rms_weight_bf16(2001, H)
+    rng = np.random.default_rng(7)
+    # weights: per channel and per block, quantized by the oracle (setup, untimed)
+    Wgu = inp.to_bf16_bits(rng.normal(0, 0.02, (2 * I, H)))
+    Wd = inp.to_bf16_bits(rng.normal(0, 0.02, (H, I)))
+    gu_q, gu_s = oracle.group_quant(Wgu, H)
+    d_q, d_s = oracle.group_quant(Wd, I)
+
+    def blocks(Wb, N, K):
+        wf = inp.bf16_bits_to_f32(Wb).reshape(N // 128, 128, K // 128, 128)
+        s = oracle.scale(np.abs(wf).max(axis=(1, 3)).astype(np.float32))
+        q = oracle.e4m3_encode((wf / s[:, None, :, None]).astype(np.float32)).reshape(N, K)
+        return q, s
+
+    gu_bq, gu_bs = blocks(Wgu, 2 * I, H)
+    d_bq, d_bs = blocks(Wd, H, I)
+
+    def step():
+        oracle.group_quant(x, H)
+        oracle.group_quant(x, 128)
+        qa, sa = oracle.rmsnorm_quant(x, w, EPS, H)
+        h, _ = oracle.scaled_mm(qa, gu_q, sa.reshape(-1), gu_s.reshape(-1))
+        hb = inp.to_bf16_bits(h)
+        qh, sh = oracle.silu_mul_quant(hb, I)
+        oracle.scaled_mm(qh, d_q, sh.reshape(-1), d_s.reshape(-1))
+        qa, sa = oracle.rmsnorm_quant(x, w, EPS, 128)
+        h, _ = oracle.scaled_mm_blockwise(qa, gu_bq, sa, gu_bs)
+        qh, sh = oracle.silu_mul_quant(inp.to_bf16_bits(h), 128)
+        oracle.scaled_mm_blockwise(qh, d_bq, sh, d_bs)
+
+    for _ in range(max(1, min(args.warmup, 1))):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    flops = gemm_flops(rows) * args.steps
+    value = flops / dt / 1e12
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = (f"{rows} of {M} tokens per step (all ops of the step on those tokens; "
+              f"value = their GEMM FLOPs / oracle time)")
+    return {
+        "metric": "FP8 quant+scaled_mm TFLOP/s (Qwen3-8B MLP block, per-token + blockwise)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(M, 1), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def cpu_baseline_leg(args):
+    """Oracle timed on a bounded sample (rank 0, N=1 only)."""
+    os.environ.setdefault("FP8Q_REF_ROWS", "64")
+    a = argparse.Namespace(**vars(args))
+    a.steps, a.warmup = 1, 0
+    r = run_reference(a)
+    return {"value": r["value"], "unit": "TFLOP/s", "cores": r["cpu_baseline"]["cores"],
+            "kind": "oracle", "sample": r["cpu_baseline"]["sample"] + ", 1 step"}
+
+
+def main():
+    args = parse()
+    os.environ.setdefault("OMP_NUM_THREADS", str(os.cpu_count() or 1))
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    line = run_native(args, rank, world, local_rank)
+    if rank == 0:
+        if world == 1:
+            line["cpu_baseline"] = cpu_baseline_leg(args)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,278 @@
+"""Python binding of libfp8q, the B200 (sm_100a) FP8 W8A8 linear-layer path.
+
+Argument marshalling only: every entry point takes torch CUDA tensors, checks
+dtypes and shapes enough to pass the right pointers, and calls the C ABI of
+``include/fp8q.h`` with the current CUDA stream.  All arithmetic runs in the
+library's kernels; there is no CPU or PyTorch fallback, and importing this
+package fails loudly if ``libfp8q.so`` is missing (build it with
+``python -m fp8_quantized_linear_rms_b200.build``).
+
+The names match the C ABI:
+  fp8q_group_quant, fp8q_rmsnorm_quant, fp8q_silu_mul_quant   (activation quant)
+  fp8q_scaled_mm, fp8q_scaled_mm_blockwise                      (scaled FP8 GEMMs)
+  fp8q_workspace_bytes, fp8q_select_gemm_variant, fp8q_force_gemm_variant,
+  fp8q_last_device_status, fp8q_status_string, fp8q_version
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfp8q.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fp8q.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libfp8q.so not found at {LIB_PATH}; build it with "
+                      "`python -m fp8_quantized_linear_rms_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(5)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+
+
+class GemmVariant(ctypes.Structure):
+    """fp8q_gemm_variant: swap_ab, split_k, block_n."""
+    _fields_ = [("swap_ab", ctypes.c_int), ("split_k", ctypes.c_int), ("block_n", ctypes.c_int)]
+
+    def as_dict(self):
+        return {"swap_ab": self.swap_ab, "split_k": self.split_k, "block_n": self.block_n}
+
+
+_SIGS = {
+    "fp8q_group_quant": (_INT, [_P, _I64, _I64, _I64, _INT, _INT, _P, _I64, _P, _I64, _I64, _P]),
+    "fp8q_rmsnorm_quant": (_INT, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _INT, _INT, _P, _I64,
+                                  _P, _I64, _I64, _P]),
+    "fp8q_silu_mul_quant": (_INT, [_P, _I64, _I64, _I64, _INT, _INT, _P, _I64, _P, _I64, _I64,
+                                   _P]),
+    "fp8q_scaled_mm": (_INT, [_P, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P, _I64, _P,
+                              ctypes.c_size_t, _P]),
+    "fp8q_scaled_mm_blockwise": (_INT, [_P, _P, _P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I64,
+                                        _P, ctypes.c_size_t, _P]),
+    "fp8q_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, _INT]),
+    "fp8q_select_gemm_variant": (_INT, [_I64, _I64, _I64, _INT, ctypes.POINTER(GemmVariant)]),
+    "fp8q_force_gemm_variant": (_INT, [ctypes.POINTER(GemmVariant)]),
+    "fp8q_last_device_status": (_INT, [_P]),
+    "fp8q_status_string": (ctypes.c_char_p, [_INT]),
+    "fp8q_version": (ctypes.c_char_p, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class Fp8qError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {lib.fp8q_status_string(status).decode()} ({status})")
+
+
+def header_functions() -> list[str]:
+    """Names of every function include/fp8q.h declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return re.findall(r"^FP8Q_API\s+[\w\s\*]+?\b(fp8q_\w+)\s*\(", text, flags=re.M)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(fn: str, status: int) -> None:
+    if status != OK:
+        raise Fp8qError(fn, status)
+
+
+def _need(t: torch.Tensor, dtype, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _rowmajor(t: torch.Tensor, name: str) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be 2-D with unit column stride")
+    return t.stride(0)
+
+
+def _scales_out(M, L, group, layout, device, scales):
+    G = L // group if group > 0 and L % group == 0 else 0
+    if scales is None:
+        if layout == "group_major":
+            scales = torch.empty((G, M), dtype=torch.float32, device=device)
+        else:
+            scales = torch.empty((M, G), dtype=torch.float32, device=device)
+    if layout == "group_major":
+        return scales, 1, M
+    return scales, G, 1
+
+
+# --------------------------------------------------------------- activation quant
+def fp8q_group_quant(x: torch.Tensor, group_size: int, ue8m0: bool = False, q=None, scales=None,
+                     scale_layout: str = "row_major", stream=None):
+    """per_token_group_fp8_quant (group_size=128) / per-token quant (group_size=K).
+
+    x: bf16 [M, K].  Returns (q float8_e4m3fn [M, K], scales fp32 [M, K/g]
+    (row_major) or [K/g, M] (group_major)).
+    """
+    _need(x, torch.bfloat16, "x")
+    ldx = _rowmajor(x, "x")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    scales, ssm, ssg = _scales_out(M, K, group_size, scale_layout, x.device, scales)
+    st = lib.fp8q_group_quant(x.data_ptr(), M, K, ldx, group_size, int(ue8m0), q.data_ptr(),
+                              _rowmajor(q, "q"), scales.data_ptr(), ssm, ssg, _stream(stream))
+    _check("fp8q_group_quant", st)
+    return q, scales
+
+
+def fp8q_rmsnorm_quant(x: torch.Tensor, w: torch.Tensor, eps: float, group_size: int,
+                       ue8m0: bool = False, q=None, scales=None, scale_layout: str = "row_major",
+                       stream=None):
+    """rms_norm_dynamic_per_token_quant (group_size=H) / rms_norm_per_block_quant (128)."""
+    _need(x, torch.bfloat16, "x")
+    _need(w, torch.bfloat16, "w")
+    ldx = _rowmajor(x, "x")
+    M, H = x.shape
+    if q is None:
+        q = torch.empty((M, H), dtype=torch.float8_e4m3fn, device=x.device)
+    scales, ssm, ssg = _scales_out(M, H, group_size, scale_layout, x.device, scales)
+    st = lib.fp8q_rmsnorm_quant(x.data_ptr(), w.data_ptr(), ctypes.c_float(eps), M, H, ldx,
+                                group_size, int(ue8m0), q.data_ptr(), _rowmajor(q, "q"),
+                                scales.data_ptr(), ssm, ssg, _stream(stream))
+    _check("fp8q_rmsnorm_quant", st)
+    return q, scales
+
+
+def fp8q_silu_mul_quant(x: torch.Tensor, group_size: int, ue8m0: bool = False, q=None,
+                        scales=None, scale_layout: str = "row_major", stream=None):
+    """silu_and_mul_dynamic_per_token_quant (group_size=I) / silu_and_mul_per_block_quant (128).
+
+    x: bf16 [M, 2I] = [gate | up].
+    """
+    _need(x, torch.bfloat16, "x")
+    ldx = _rowmajor(x, "x")
+    M, I2 = x.shape
+    I = I2 // 2
+    if q is None:
+        q = torch.empty((M, I), dtype=torch.float8_e4m3fn, device=x.device)
+    scales, ssm, ssg = _scales_out(M, I, group_size, scale_layout, x.device, scales)
+    st = lib.fp8q_silu_mul_quant(x.data_ptr(), M, I, ldx, group_size, int(ue8m0), q.data_ptr(),
+                                 _rowmajor(q, "q"), scales.data_ptr(), ssm, ssg, _stream(stream))
+    _check("fp8q_silu_mul_quant", st)
+    return q, scales
+
+
+# --------------------------------------------------------------------- GEMMs
+def fp8q_workspace_bytes(M: int, N: int, K: int, blockwise: bool) -> int:
+    return int(lib.fp8q_workspace_bytes(M, N, K, int(blockwise)))
+
+
+def make_workspace(M: int, N: int, K: int, blockwise: bool, device="cuda") -> torch.Tensor | None:
+    """A zero-filled workspace for a GEMM of this shape (None if it needs none)."""
+    n = fp8q_workspace_bytes(M, N, K, blockwise)
+    return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
+
+
+def _ws(ws, M, N, K, blockwise, device):
+    """Pointer/size of the caller's workspace; when none is given and the shape
+    needs one, a fresh zero-filled buffer (the C ABI itself never allocates)."""
+    if ws is None:
+        ws = make_workspace(M, N, K, blockwise, device)
+    return (ws.data_ptr(), ws.numel() * ws.element_size(), ws) if ws is not None else (None, 0, None)
+
+
+def fp8q_scaled_mm(a_q: torch.Tensor, b_q: torch.Tensor, a_scale: torch.Tensor,
+                   b_scale: torch.Tensor, y=None, workspace=None, stream=None):
+    """y [M, N] bf16 = sa * sb * (a_q [M, K] @ b_q [N, K]^T).
+
+    a_scale: fp32 [M] (per token) or [1]; b_scale: fp32 [N] (per channel) or [1].
+    """
+    for t, n in ((a_q, "a_q"), (b_q, "b_q")):
+        _need(t, torch.float8_e4m3fn, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _need(a_scale, torch.float32, "a_scale")
+    _need(b_scale, torch.float32, "b_scale")
+    M, K = a_q.shape
+    N = b_q.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_q.device)
+    if a_scale.numel() not in (1, M) or b_scale.numel() not in (1, N):
+        raise ValueError("a_scale must have 1 or M entries, b_scale 1 or N")
+    wp, wn, _keep = _ws(workspace, M, N, K, False, a_q.device)
+    st = lib.fp8q_scaled_mm(a_q.data_ptr(), b_q.data_ptr(), a_scale.data_ptr(),
+                            int(a_scale.numel() == M), b_scale.data_ptr(),
+                            int(b_scale.numel() == N), M, N, K, y.data_ptr(), _rowmajor(y, "y"),
+                            wp, wn, _stream(stream))
+    _check("fp8q_scaled_mm", st)
+    return y
+
+
+def fp8q_scaled_mm_blockwise(a_q: torch.Tensor, b_q: torch.Tensor, a_scale: torch.Tensor,
+                             b_scale: torch.Tensor, a_scale_layout: str = "row_major", y=None,
+                             workspace=None, stream=None):
+    """Block-scaled GEMM: a_scale one fp32 per 1x128 group of A ([M, K/128] row_major or
+    [K/128, M] group_major), b_scale fp32 [N/128, K/128]."""
+    for t, n in ((a_q, "a_q"), (b_q, "b_q")):
+        _need(t, torch.float8_e4m3fn, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _need(a_scale, torch.float32, "a_scale")
+    _need(b_scale, torch.float32, "b_scale")
+    M, K = a_q.shape
+    N = b_q.shape[0]
+    if a_scale_layout == "group_major":
+        sm, skb = 1, M
+    else:
+        sm, skb = K // 128, 1
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_q.device)
+    wp, wn, _keep = _ws(workspace, M, N, K, True, a_q.device)
+    st = lib.fp8q_scaled_mm_blockwise(a_q.data_ptr(), b_q.data_ptr(), a_scale.data_ptr(), sm, skb,
+                                      b_scale.data_ptr(), M, N, K, y.data_ptr(),
+                                      _rowmajor(y, "y"), wp, wn, _stream(stream))
+    _check("fp8q_scaled_mm_blockwise", st)
+    return y
+
+
+def fp8q_select_gemm_variant(M: int, N: int, K: int, blockwise: bool) -> dict:
+    v = GemmVariant()
+    _check("fp8q_select_gemm_variant", lib.fp8q_select_gemm_variant(M, N, K, int(blockwise),
+                                                                    ctypes.byref(v)))
+    return v.as_dict()
+
+
+def fp8q_force_gemm_variant(swap_ab: int | None = None, split_k: int = 1, block_n: int = 128):
+    """Force a GEMM variant for the following calls (testing/tuning); no args = automatic."""
+    if swap_ab is None:
+        _check("fp8q_force_gemm_variant", lib.fp8q_force_gemm_variant(None))
+        return
+    v = GemmVariant(int(swap_ab), int(split_k), int(block_n))
+    _check("fp8q_force_gemm_variant", lib.fp8q_force_gemm_variant(ctypes.byref(v)))
+
+
+def fp8q_last_device_status(stream=None) -> int:
+    return int(lib.fp8q_last_device_status(_stream(stream)))
+
+
+def fp8q_status_string(status: int) -> str:
+    return lib.fp8q_status_string(status).decode()
+
+
+def fp8q_version() -> str:
+    return lib.fp8q_version().decode()

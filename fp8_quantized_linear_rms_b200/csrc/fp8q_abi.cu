@@ -1,0 +1,58 @@
+// fp8q_abi.cu -- status, version and device-query entry points of libfp8q.
+#include <mutex>
+
+#include "fp8q_common.cuh"
+
+namespace fp8q {
+
+__device__ int g_device_status = 0;
+
+int* device_status_ptr() {
+  static int* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int*>(p);
+  }
+  return cache[dev];
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace fp8q
+
+extern "C" fp8q_status fp8q_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP8Q_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, fp8q::g_device_status, sizeof(int)) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(fp8q::g_device_status, &zero, sizeof(int)) != cudaSuccess)
+    return FP8Q_ERR_CUDA;
+  return static_cast<fp8q_status>(v);
+}
+
+extern "C" const char* fp8q_status_string(fp8q_status s) {
+  switch (s) {
+    case FP8Q_OK: return "ok";
+    case FP8Q_ERR_INVALID_ARG: return "invalid argument";
+    case FP8Q_ERR_UNSUPPORTED: return "unsupported shape or configuration";
+    case FP8Q_ERR_CUDA: return "CUDA error";
+    case FP8Q_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+extern "C" const char* fp8q_version(void) { return "fp8q 0.1 sm_100a"; }

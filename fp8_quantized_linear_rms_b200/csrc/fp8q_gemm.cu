@@ -1,0 +1,734 @@
+// fp8q_gemm.cu -- scaled FP8 GEMMs on the 5th-generation tensor cores (sm_100a).
+//
+//   scaled_mm            y = bf16(sa(m) sb(n) sum_k qa[m,k] qb[n,k])
+//   scaled_mm_blockwise  y = bf16(sum_kb sa[m,kb] sb[n/128,kb] P_kb[m,n])
+// ("Helion in vLLM" (24-ai.news), section "Kernels integrated into vLLM",
+// items 8 and 9; the FP8_Dynamic and Block_FP8 schemes of "Helion linear
+// backend" (aihirek.info), section "Autotuning selects the variant").
+//
+// One persistent kernel template, one CTA per SM, warp-specialized:
+//   warp 0      TMA producer: 128-row x 128-byte e4m3 tiles of both operands,
+//               128B-swizzled, into a STAGES-deep shared-memory ring guarded
+//               by full/empty mbarriers;
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//               (kind::f8f6f4, M = 128, N = BN, K = 32 per instruction);
+//   warps 2..   epilogue: tcgen05.ld of the fp32 accumulator, scales, bf16.
+// Per-token/per-channel scales: the accumulator of a whole tile lives in one
+// of two TMEM buffers, so the epilogue of tile t overlaps the mainloop of
+// tile t+1.  Blockwise scales: each 128-deep K block accumulates into its own
+// TMEM partial buffer (4 rotating buffers); the epilogue promotes every partial
+// into fp32 registers with its scale sa[m,kb]*sb[nb,kb].
+//
+// Variants ("Helion linear backend" (aihirek.info), section "Single GEMM
+// implementation handles several algorithms"):
+//   Swap-AB  the weight rows fill the MMA's 128-row M slot and the tokens its
+//            N slot (BN = 16..128), for small M;
+//   Split-K  the K loop of a tile is cut into `split` ranges run by different
+//            CTAs; each writes a scaled fp32 partial to the workspace and the
+//            last one to arrive (per-warp atomic counter) sums the partials in
+//            split order (deterministic) and writes y.
+// No TMA multicast is used: every CTA loads its own tiles.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+#include <unordered_map>
+
+#include "fp8q_common.cuh"
+#include "fp8q_sm100.cuh"
+
+namespace fp8q {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;       // MMA M = TMEM lanes per tile
+constexpr int BK = 128;       // K bytes (e4m3 elements) per pipeline stage
+constexpr int UMMA_K = 32;    // K per tcgen05.mma for 8-bit operands
+constexpr int A_BYTES = BM * BK;
+constexpr int kSmemBudget = 200 * 1024;
+
+struct GemmArgs {
+  int rows_a, rows_b, K;              // MMA-A rows (TMEM lanes), MMA-B rows (columns)
+  int kblocks, tiles_a, tiles_b, split, kb_per_split, units;
+  int M, N;                           // logical output shape
+  const float* sa;                    // activation scales: sa[m*sa_sm + kb*sa_skb]
+  int64_t sa_sm, sa_skb;
+  const float* sb;                    // weight scales: per channel sb[n*sb_sn];
+  int64_t sb_sn, sb_snb, sb_skb;      //   blockwise sb[(n/128)*sb_snb + kb*sb_skb]
+  uint16_t* y;                        // bf16 [M, ldy]
+  int64_t ldy;
+  float* ws;                          // split-K partials
+  int* counters;                      // split-K arrival counters (zero between calls)
+  int* status;                        // device status word
+};
+
+template <int BN, bool SWAP, bool BW>
+struct Cfg {
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int EPI_WARPS = (BW && BN >= 128) ? 8 : 4;
+  static constexpr int COL_GROUPS = EPI_WARPS / 4;        // column slices per TMEM lane quadrant
+  static constexpr int CPT = BN / COL_GROUPS;              // columns per epilogue thread
+  static constexpr int CHUNK = CPT < 32 ? CPT : 32;        // columns per tcgen05.ld
+  static constexpr int NBUF = BW ? 4 : 2;                  // TMEM accumulator buffers
+  static constexpr int TMEM_NEED = NBUF * BN;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
+                                 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * NBUF + 1) + 16;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static_assert(STAGES >= 2, "pipeline too shallow");
+  static_assert(TMEM_NEED <= 512, "accumulators exceed TMEM");
+  static_assert(CPT % CHUNK == 0 && (CHUNK == 16 || CHUNK == 32), "chunking");
+  static_assert(B_BYTES % 1024 == 0, "B tiles must stay 1024-byte aligned");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+__device__ __forceinline__ void unit_coords(const GemmArgs& p, int u, int& ta, int& tb, int& s,
+                                            int& kb0, int& kb1) {
+  ta = u % p.tiles_a;
+  const int r = u / p.tiles_a;
+  tb = r % p.tiles_b;
+  s = r / p.tiles_b;
+  kb0 = s * p.kb_per_split;
+  kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+}
+
+// Bounded wait that ignores the abort flag: used only to drain in-flight
+// asynchronous work before the CTA exits.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int BN, bool SWAP, bool BW>
+__global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmArgs p) {
+  using C = Cfg<BN, SWAP, BW>;
+  constexpr int S = C::STAGES;
+  constexpr int NB = C::NBUF;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * C::B_BYTES);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + NB;
+  uint64_t* drain = tempty + NB;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < NB; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], C::EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+        int ta, tb, s, kb0, kb1;
+        unit_coords(p, u, ta, tb, s, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int st = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+          tma_load_2d(sA + st * A_BYTES, &tmA, &full[st], kb * BK, ta * BM);
+          tma_load_2d(sB + st * C::B_BYTES, &tmB, &full[st], kb * BK, tb * BN);
+        }
+      }
+      if (!ok) {
+        // Let every copy already issued land before the CTA can exit.
+        const int first = it - S > 0 ? it - S : 0;
+        for (int j = first; j < it; ++j) drain_wait(&full[j % S], (j / S) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      int it = 0, t = 0, pc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+        int ta, tb, s, kb0, kb1;
+        unit_coords(p, u, ta, tb, s, kb0, kb1);
+        uint32_t d = tmem_base;
+        int buf = 0;
+        if (!BW) {
+          buf = t & 1;
+          if (!mbar_wait(&tempty[buf], ((t >> 1) & 1) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          d = tmem_base + buf * BN;
+        }
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int st = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!mbar_wait(&full[st], ph, abort_flag, p.status)) { ok = false; break; }
+          int pb = 0;
+          if (BW) {
+            pb = pc % NB;
+            if (!mbar_wait(&tempty[pb], ((pc / NB) & 1) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+            d = tmem_base + pb * BN;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_kmajor_sw128(sA + st * A_BYTES);
+          const uint64_t bdesc = smem_desc_kmajor_sw128(sB + st * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            const uint32_t acc = BW ? (k > 0) : (kb > kb0 || k > 0);
+            mma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);  // +32 bytes of K
+          }
+          mma_commit(&empty[st]);
+          if (BW) {
+            mma_commit(&tfull[pb]);
+            ++pc;
+          }
+        }
+        if (!ok) break;
+        if (!BW) {
+          mma_commit(&tfull[buf]);
+          ++t;
+        }
+      }
+      // Every MMA issued so far has completed once `drain` flips.
+      mma_commit(drain);
+      drain_wait(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;
+    const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
+    const int cg = e >> 2;                     // column slice
+    const int row = quad * 32 + lane;          // MMA-A row within the tile
+    const int col0 = cg * C::CPT;
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    int t = 0, pc = 0;
+    bool ok = true;
+
+    for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+      int ta, tb, s, kb0, kb1;
+      unit_coords(p, u, ta, tb, s, kb0, kb1);
+      const int a_idx = ta * BM + row;                         // m (no swap) or n (swap)
+      const int b_base = tb * BN;                              // first column's n or m
+      const bool a_valid = a_idx < (SWAP ? p.N : p.M);
+      const int tile_id = tb * p.tiles_a + ta;
+      float* ws_tile = p.ws + (static_cast<int64_t>(tile_id) * p.split) * (BN * BM);
+
+      // Store one chunk of CHUNK final values v[] for columns col..col+CHUNK-1.
+      auto emit = [&](int col, const float* v) {
+        if (!a_valid) return;
+        if (!SWAP) {
+          const int m = a_idx;
+          uint16_t* yr = p.y + static_cast<int64_t>(m) * p.ldy;
+#pragma unroll
+          for (int g = 0; g < C::CHUNK; g += 8) {
+            const int n = b_base + col + g;
+            if (n < p.N) {
+              uint4 o;
+              o.x = pack_bf16x2(v[g + 0], v[g + 1]);
+              o.y = pack_bf16x2(v[g + 2], v[g + 3]);
+              o.z = pack_bf16x2(v[g + 4], v[g + 5]);
+              o.w = pack_bf16x2(v[g + 6], v[g + 7]);
+              *reinterpret_cast<uint4*>(yr + n) = o;
+            }
+          }
+        } else {
+          const int n = a_idx;
+#pragma unroll
+          for (int i = 0; i < C::CHUNK; ++i) {
+            const int m = b_base + col + i;
+            if (m < p.M)
+              p.y[static_cast<int64_t>(m) * p.ldy + n] =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
+          }
+        }
+      };
+      auto stash = [&](int col, const float* v) {    // fp32 partial of split s
+        float* w = ws_tile + static_cast<int64_t>(s) * (BN * BM);
+#pragma unroll
+        for (int i = 0; i < C::CHUNK; ++i) w[(col + i) * BM + row] = v[i];
+      };
+      auto finish_split = [&]() {                    // last arrival sums the partials in order
+        __threadfence();
+        __syncwarp();
+        int old = 0;
+        if (lane == 0) old = atomicAdd(&p.counters[tile_id * C::EPI_WARPS + e], 1);
+        old = __shfl_sync(0xFFFFFFFFu, old, 0);
+        if (old != p.split - 1) return;
+        if (lane == 0) p.counters[tile_id * C::EPI_WARPS + e] = 0;
+        __threadfence();
+        for (int c = col0; c < col0 + C::CPT; c += C::CHUNK) {
+          float v[C::CHUNK];
+#pragma unroll
+          for (int i = 0; i < C::CHUNK; ++i) v[i] = 0.0f;
+          for (int ss = 0; ss < p.split; ++ss) {
+            const float* w = ws_tile + static_cast<int64_t>(ss) * (BN * BM);
+#pragma unroll
+            for (int i = 0; i < C::CHUNK; ++i) v[i] += __ldcg(w + (c + i) * BM + row);
+          }
+          emit(c, v);
+        }
+      };
+
+      if (!BW) {
+        // -------- per-token / per-channel scales: one accumulator per tile
+        const int buf = t & 1;
+        float srow;
+        if (!SWAP) srow = a_valid ? __ldg(p.sa + a_idx * p.sa_sm) : 0.0f;
+        else srow = a_valid ? __ldg(p.sb + a_idx * p.sb_sn) : 0.0f;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[buf], (t >> 1) & 1, abort_flag, p.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int c = col0; c < col0 + C::CPT; c += C::CHUNK) {
+          float v[C::CHUNK];
+          const uint32_t taddr = tmem_base + lane_addr + buf * BN + c;
+          if (C::CHUNK == 32) tmem_ld_32x32b_x32(taddr, v);
+          else tmem_ld_32x32b_x16(taddr, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < C::CHUNK; ++i) {
+            const int b_idx = b_base + c + i;
+            float sc;
+            if (!SWAP) sc = b_idx < p.N ? __ldg(p.sb + b_idx * p.sb_sn) : 0.0f;
+            else sc = b_idx < p.M ? __ldg(p.sa + b_idx * p.sa_sm) : 0.0f;
+            v[i] = v[i] * (srow * sc);
+          }
+          if (p.split == 1) emit(c, v);
+          else stash(c, v);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+        ++t;
+        if (p.split > 1) finish_split();
+      } else {
+        // -------- blockwise scales: promote each K-block partial into registers
+        float acc[C::CPT];
+#pragma unroll
+        for (int i = 0; i < C::CPT; ++i) acc[i] = 0.0f;
+        const int nb = SWAP ? ta : (tb * BN) / 128;   // weight block row (constant per tile)
+        for (int kb = kb0; kb < kb1; ++kb) {
+          const int pb = pc % NB;
+          const float sbk = __ldg(p.sb + nb * p.sb_snb + kb * p.sb_skb);
+          float srow = 0.0f;
+          if (!SWAP) srow = a_valid ? __ldg(p.sa + a_idx * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[pb], (pc / NB) & 1, abort_flag, p.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < C::CPT; c += C::CHUNK) {
+            float v[C::CHUNK];
+            const uint32_t taddr = tmem_base + lane_addr + pb * BN + col0 + c;
+            if (C::CHUNK == 32) tmem_ld_32x32b_x32(taddr, v);
+            else tmem_ld_32x32b_x16(taddr, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < C::CHUNK; ++i) {
+              float sc = srow;
+              if (SWAP) {
+                const int m = b_base + col0 + c + i;
+                sc = m < p.M ? __ldg(p.sa + m * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
+              }
+              acc[c + i] = fmaf(v[i], sc, acc[c + i]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[pb]);
+          ++pc;
+        }
+        if (!ok) break;
+#pragma unroll
+        for (int c = 0; c < C::CPT; c += C::CHUNK) {
+          if (p.split == 1) emit(col0 + c, acc + c);
+          else stash(col0 + c, acc + c);
+        }
+        if (p.split > 1) finish_split();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+struct MapKey {
+  const void* ptr;
+  int64_t rows, k;
+  int box_rows, dev;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && rows == o.rows && k == o.k && box_rows == o.box_rows && dev == o.dev;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    size_t h = reinterpret_cast<uintptr_t>(k.ptr);
+    h ^= static_cast<size_t>(k.rows) * 0x9E3779B97F4A7C15ull;
+    h ^= static_cast<size_t>(k.k) * 0xC2B2AE3D27D4EB4Full;
+    h ^= static_cast<size_t>(k.box_rows) * 0x165667B19E3779F9ull + static_cast<size_t>(k.dev);
+    return h;
+  }
+};
+
+// Tensor map of an e4m3 [rows, k] row-major matrix, box = box_rows x 128
+// bytes, 128-byte swizzle, zero fill outside the matrix.  Cached per
+// (pointer, shape, box, device).
+bool tensor_map(const void* ptr, int64_t rows, int64_t k, int box_rows, CUtensorMap* out) {
+  static std::mutex mu;
+  static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const MapKey key{ptr, rows, k, box_rows, dev};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *out = it->second;
+      return true;
+    }
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  CUtensorMap m;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(k)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), gdim,
+                        gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() > 4096) cache.clear();
+  cache.emplace(key, m);
+  *out = m;
+  return true;
+}
+
+template <int BN, bool SWAP, bool BW>
+fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
+                        cudaStream_t stream) {
+  using C = Cfg<BN, SWAP, BW>;
+  CUtensorMap ma, mb;
+  if (!tensor_map(a_op, p.rows_a, p.K, BM, &ma) || !tensor_map(b_op, p.rows_b, p.K, BN, &mb))
+    return FP8Q_ERR_CUDA;
+  static int attr_done[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(gemm_kernel<BN, SWAP, BW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return FP8Q_ERR_CUDA;
+    attr_done[dev] = 1;
+  }
+  const int grid = p.units < num_sms() ? p.units : num_sms();
+  gemm_kernel<BN, SWAP, BW><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, p);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- dispatch
+
+std::mutex g_force_mu;
+bool g_forced = false;
+fp8q_gemm_variant g_force{0, 1, 128};
+
+bool variant_supported(const fp8q_gemm_variant& v, int blockwise) {
+  if (v.split_k < 1 || v.split_k > 64) return false;
+  if (v.swap_ab) return v.block_n == 16 || v.block_n == 32 || v.block_n == 64 || v.block_n == 128;
+  if (blockwise) return v.block_n == 128;
+  return v.block_n == 128 || v.block_n == 256;
+}
+
+int epi_warps(const fp8q_gemm_variant& v, int blockwise) {
+  return (blockwise && v.block_n >= 128) ? 8 : 4;
+}
+
+// Split count that spreads tiles over the SMs: the smallest split whose last
+// wave is at least 90% full, capped so that every split keeps >= 2 K blocks
+// and the fp32 partial traffic stays under a quarter of the weight bytes.
+int choose_split(int64_t tiles, int64_t kblocks, int64_t M, int64_t N, int64_t K, int bn,
+                 int sms) {
+  if (tiles >= sms) return 1;
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= 16; ++s) {
+    if (s > 1 && kblocks / s < 2) break;
+    const double ws_traffic = 2.0 * s * tiles * BM * bn * 4.0;
+    if (s > 1 && ws_traffic > 0.25 * static_cast<double>(N) * static_cast<double>(K)) break;
+    const int64_t units = tiles * s;
+    const int64_t waves = (units + sms - 1) / sms;
+    const double eff = static_cast<double>(units) / static_cast<double>(waves * sms);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = s;
+    }
+    if (eff >= 0.9) break;
+  }
+  (void)M;
+  return best;
+}
+
+fp8q_gemm_variant auto_variant(int64_t M, int64_t N, int64_t K, int blockwise) {
+  fp8q_gemm_variant v;
+  if (M <= 64) {
+    v.swap_ab = 1;
+    v.block_n = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  } else if (M <= 128) {
+    v.swap_ab = 1;
+    v.block_n = 128;
+  } else {
+    v.swap_ab = 0;
+    v.block_n = blockwise ? 128 : 256;
+  }
+  const int64_t rows_a = v.swap_ab ? N : M, rows_b = v.swap_ab ? M : N;
+  const int64_t tiles = ((rows_a + BM - 1) / BM) * ((rows_b + v.block_n - 1) / v.block_n);
+  v.split_k = choose_split(tiles, (K + BK - 1) / BK, M, N, K, v.block_n, num_sms());
+  return v;
+}
+
+fp8q_gemm_variant pick_variant(int64_t M, int64_t N, int64_t K, int blockwise) {
+  {
+    std::lock_guard<std::mutex> lock(g_force_mu);
+    if (g_forced) return g_force;
+  }
+  return auto_variant(M, N, K, blockwise);
+}
+
+struct Plan {
+  fp8q_gemm_variant v;
+  int tiles_a, tiles_b, kblocks, split, kb_per_split, units;
+  size_t counter_bytes, ws_bytes;
+};
+
+Plan make_plan(int64_t M, int64_t N, int64_t K, int blockwise, const fp8q_gemm_variant& v) {
+  Plan pl;
+  pl.v = v;
+  const int64_t rows_a = v.swap_ab ? N : M, rows_b = v.swap_ab ? M : N;
+  pl.tiles_a = static_cast<int>((rows_a + BM - 1) / BM);
+  pl.tiles_b = static_cast<int>((rows_b + v.block_n - 1) / v.block_n);
+  pl.kblocks = static_cast<int>((K + BK - 1) / BK);
+  int split = v.split_k < pl.kblocks ? v.split_k : pl.kblocks;
+  if (split < 1) split = 1;
+  pl.kb_per_split = (pl.kblocks + split - 1) / split;
+  pl.split = (pl.kblocks + pl.kb_per_split - 1) / pl.kb_per_split;   // every split non-empty
+  const int64_t tiles = static_cast<int64_t>(pl.tiles_a) * pl.tiles_b;
+  pl.units = static_cast<int>(tiles * pl.split);
+  if (pl.split > 1) {
+    pl.counter_bytes = ((static_cast<size_t>(tiles) * epi_warps(v, blockwise) * sizeof(int) + 255) / 256) * 256;
+    pl.ws_bytes = pl.counter_bytes + static_cast<size_t>(tiles) * pl.split * BM * v.block_n * sizeof(float);
+  } else {
+    pl.counter_bytes = 0;
+    pl.ws_bytes = 0;
+  }
+  return pl;
+}
+
+template <bool BW>
+fp8q_status run_gemm(const void* a_q, const void* b_q, GemmArgs& p, const Plan& pl, void* ws,
+                     cudaStream_t stream) {
+  p.tiles_a = pl.tiles_a;
+  p.tiles_b = pl.tiles_b;
+  p.kblocks = pl.kblocks;
+  p.split = pl.split;
+  p.kb_per_split = pl.kb_per_split;
+  p.units = pl.units;
+  p.counters = pl.split > 1 ? static_cast<int*>(ws) : nullptr;
+  p.ws = pl.split > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.counter_bytes) : nullptr;
+  p.status = device_status_ptr();
+  const int bn = pl.v.block_n;
+  if (pl.v.swap_ab) {
+    p.rows_a = p.N;
+    p.rows_b = p.M;
+    switch (bn) {
+      case 16: return launch_gemm<16, true, BW>(b_q, a_q, p, stream);
+      case 32: return launch_gemm<32, true, BW>(b_q, a_q, p, stream);
+      case 64: return launch_gemm<64, true, BW>(b_q, a_q, p, stream);
+      case 128: return launch_gemm<128, true, BW>(b_q, a_q, p, stream);
+      default: return FP8Q_ERR_UNSUPPORTED;
+    }
+  }
+  p.rows_a = p.M;
+  p.rows_b = p.N;
+  if (bn == 128) return launch_gemm<128, false, BW>(a_q, b_q, p, stream);
+  if (!BW && bn == 256) return launch_gemm<256, false, false>(a_q, b_q, p, stream);
+  return FP8Q_ERR_UNSUPPORTED;
+}
+
+constexpr int64_t kMaxDim = (1LL << 31) - 512;
+
+fp8q_status check_gemm(const void* a_q, const void* b_q, const void* sa, const void* sb,
+                       int64_t M, int64_t N, int64_t K, const void* y, int64_t ldy) {
+  if (M < 0 || N <= 0 || K <= 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
+    return FP8Q_ERR_INVALID_ARG;
+  if (N % 16 != 0 || K % 16 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (ldy < N || ldy % 8 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (M == 0) return FP8Q_OK;  // nothing is read or written: pointers may be null
+  if (!a_q || !b_q || !sa || !sb || !y) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(a_q, 16) || !aligned(b_q, 16) || !aligned(y, 16) || !aligned(sa, 4) ||
+      !aligned(sb, 4))
+    return FP8Q_ERR_INVALID_ARG;
+  return FP8Q_OK;
+}
+
+}  // namespace
+}  // namespace fp8q
+
+using namespace fp8q;
+
+extern "C" fp8q_status fp8q_select_gemm_variant(int64_t M, int64_t N, int64_t K, int blockwise,
+                                                fp8q_gemm_variant* out) {
+  if (!out || M < 0 || N <= 0 || K <= 0) return FP8Q_ERR_INVALID_ARG;
+  *out = pick_variant(M, N, K, blockwise);
+  const Plan pl = make_plan(M, N, K, blockwise, *out);
+  out->split_k = pl.split;
+  return FP8Q_OK;
+}
+
+extern "C" fp8q_status fp8q_force_gemm_variant(const fp8q_gemm_variant* v) {
+  std::lock_guard<std::mutex> lock(g_force_mu);
+  if (!v) {
+    g_forced = false;
+    return FP8Q_OK;
+  }
+  if (!variant_supported(*v, 0) && !variant_supported(*v, 1)) return FP8Q_ERR_INVALID_ARG;
+  g_force = *v;
+  g_forced = true;
+  return FP8Q_OK;
+}
+
+extern "C" size_t fp8q_workspace_bytes(int64_t M, int64_t N, int64_t K, int blockwise) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  const fp8q_gemm_variant v = pick_variant(M, N, K, blockwise);
+  return make_plan(M, N, K, blockwise, v).ws_bytes;
+}
+
+extern "C" fp8q_status fp8q_scaled_mm(const void* a_q, const void* b_q, const float* a_scale,
+                                      int a_per_token, const float* b_scale, int b_per_channel,
+                                      int64_t M, int64_t N, int64_t K, void* y, int64_t ldy,
+                                      void* workspace, size_t ws_bytes, void* stream) {
+  fp8q_status st = check_gemm(a_q, b_q, a_scale, b_scale, M, N, K, y, ldy);
+  if (st != FP8Q_OK) return st;
+  if ((a_per_token != 0 && a_per_token != 1) || (b_per_channel != 0 && b_per_channel != 1))
+    return FP8Q_ERR_INVALID_ARG;
+  if (M == 0) return FP8Q_OK;
+  const fp8q_gemm_variant v = pick_variant(M, N, K, 0);
+  if (!variant_supported(v, 0)) return FP8Q_ERR_UNSUPPORTED;
+  const Plan pl = make_plan(M, N, K, 0, v);
+  if (pl.ws_bytes > 0 && (!workspace || ws_bytes < pl.ws_bytes || !aligned(workspace, 256)))
+    return FP8Q_ERR_INVALID_ARG;
+  GemmArgs p{};
+  p.K = static_cast<int>(K);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.sa = a_scale;
+  p.sa_sm = a_per_token ? 1 : 0;
+  p.sa_skb = 0;
+  p.sb = b_scale;
+  p.sb_sn = b_per_channel ? 1 : 0;
+  p.sb_snb = 0;
+  p.sb_skb = 0;
+  p.y = static_cast<uint16_t*>(y);
+  p.ldy = ldy;
+  return run_gemm<false>(a_q, b_q, p, pl, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fp8q_status fp8q_scaled_mm_blockwise(const void* a_q, const void* b_q,
+                                                const float* a_scale, int64_t as_stride_m,
+                                                int64_t as_stride_kb, const float* b_scale,
+                                                int64_t M, int64_t N, int64_t K, void* y,
+                                                int64_t ldy, void* workspace, size_t ws_bytes,
+                                                void* stream) {
+  fp8q_status st = check_gemm(a_q, b_q, a_scale, b_scale, M, N, K, y, ldy);
+  if (st != FP8Q_OK) return st;
+  if (N % 128 != 0 || K % 128 != 0 || as_stride_m < 0 || as_stride_kb < 0)
+    return FP8Q_ERR_INVALID_ARG;
+  if (M == 0) return FP8Q_OK;
+  const fp8q_gemm_variant v = pick_variant(M, N, K, 1);
+  if (!variant_supported(v, 1)) return FP8Q_ERR_UNSUPPORTED;
+  const Plan pl = make_plan(M, N, K, 1, v);
+  if (pl.ws_bytes > 0 && (!workspace || ws_bytes < pl.ws_bytes || !aligned(workspace, 256)))
+    return FP8Q_ERR_INVALID_ARG;
+  GemmArgs p{};
+  p.K = static_cast<int>(K);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.sa = a_scale;
+  p.sa_sm = as_stride_m;
+  p.sa_skb = as_stride_kb;
+  p.sb = b_scale;
+  p.sb_sn = 0;
+  p.sb_snb = K / 128;
+  p.sb_skb = 1;
+  p.y = static_cast<uint16_t*>(y);
+  p.ldy = ldy;
+  return run_gemm<true>(a_q, b_q, p, pl, workspace, static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,216 @@
+/*
+ * fp8q.h -- C ABI of libfp8q, the B200 (sm_100a) FP8 W8A8 linear-layer path:
+ * dynamic activation quantization fused with its producer, and the scaled FP8
+ * GEMMs it feeds.
+ *
+ * The ops are the ones listed in "Helion in vLLM" (24-ai.news), section
+ * "Kernels integrated into vLLM": items 1-3 and 5-7 (quantization) and 8-9
+ * (GEMMs).  The pages name them but do not write out their arithmetic; this
+ * library fixes it as follows.
+ *
+ *   scale      s = fl32(max(amax, 1e-10) / 448), amax = max |y| over the group
+ *   UE8M0      (ue8m0 = 1) s is rounded up to the next power of two (a power of
+ *              two is kept); the scale is still stored as fp32
+ *   codes      q = e4m3fn(fl32(y / s)), IEEE fp32 division, round to nearest
+ *              even, saturating to +-448; the sign of zero is kept
+ *   groups     contiguous 1x128 chunks of a row (group_size = 128), or the
+ *              whole row (group_size = row length: "per token")
+ *   y          the value quantized: x itself (group quant); bf16(bf16(x*r)*w)
+ *              with r = 1/sqrt(mean(x^2)+eps) (RMSNorm); bf16(silu(g)*u)
+ *              (SiLU*mul) -- one round-to-nearest-even to bf16 at each step
+ *   GEMM       y[m,n] = bf16_rn(sum_k (qa[m,k] sa)(qb[n,k] sb)), fp32 accumulate
+ *
+ * Conventions shared by every entry point.
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The
+ *     library allocates no device memory in any call: scratch space is the
+ *     caller's `workspace` (sized by fp8q_workspace_bytes).
+ *   - bf16 tensors are raw IEEE bfloat16 bit patterns; codes are float8
+ *     e4m3fn bytes; scales are fp32.  Matrices are row-major with a leading
+ *     dimension `ld*` given in ELEMENTS.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Calls are asynchronous: they enqueue kernels and return; no
+ *     call synchronizes the host except fp8q_last_device_status.
+ *   - Argument errors are found on the host before anything is launched; the
+ *     call then returns FP8Q_ERR_INVALID_ARG (or FP8Q_ERR_UNSUPPORTED) and
+ *     launches nothing.  A launch failure returns FP8Q_ERR_CUDA.  A GEMM
+ *     whose internal pipeline wait runs past its time limit (about one
+ *     second) stops, records FP8Q_ERR_TIMEOUT in a device status word and
+ *     returns; read it with fp8q_last_device_status.  No C++ exception
+ *     crosses this interface.
+ *   - Pointers to bf16 / code tensors must be 16-byte aligned; scale pointers
+ *     4-byte aligned.  With M = 0 a call validates its sizes and returns
+ *     FP8Q_OK without touching memory; its pointers may then be NULL.
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP8Q_API __attribute__((visibility("default")))
+#else
+#define FP8Q_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8Q_OK = 0,
+    FP8Q_ERR_INVALID_ARG = 1,  /* null pointer, bad size, stride or alignment */
+    FP8Q_ERR_UNSUPPORTED = 2,  /* valid request this build does not handle    */
+    FP8Q_ERR_CUDA = 3,         /* a CUDA runtime / driver call failed          */
+    FP8Q_ERR_TIMEOUT = 4       /* a device-side wait gave up (device status)   */
+} fp8q_status;
+
+/* ------------------------------------------------------------------------ */
+/* Activation quantization                                                   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * fp8q_group_quant -- per_token_group_fp8_quant (group_size = 128) and
+ * dynamic_per_token_scaled_fp8_quant (group_size = K) ("Helion in vLLM",
+ * "Kernels integrated into vLLM", items 5 and 1).  Also quantizes weights per
+ * output channel: a row of W [N, K] is one channel.
+ *
+ *   x        bf16 [M, K], leading dimension ldx (>= K, multiple of 8)
+ *   M, K     M >= 0 (M = 0 is a no-op), K > 0 and a multiple of 16
+ *   group_size  128 (K must then be a multiple of 128) or K
+ *   ue8m0    0 or 1 (round scales up to powers of two)
+ *   q        e4m3 codes [M, K], leading dimension ldq (>= K, multiple of 16)
+ *   scales   fp32, scale of group g of row m at scales[m*s_stride_m + g*s_stride_g]
+ *            (row-major [M, K/group]: s_stride_m = K/group, s_stride_g = 1;
+ *            group-major [K/group, M]: s_stride_m = 1, s_stride_g = M)
+ */
+FP8Q_API fp8q_status fp8q_group_quant(const void* x, int64_t M, int64_t K, int64_t ldx, int group_size,
+                             int ue8m0, void* q, int64_t ldq, float* scales,
+                             int64_t s_stride_m, int64_t s_stride_g, void* stream);
+
+/*
+ * fp8q_rmsnorm_quant -- rms_norm_dynamic_per_token_quant (group_size = H)
+ * and rms_norm_per_block_quant (group_size = 128) ("Helion in vLLM",
+ * "Kernels integrated into vLLM", items 2 and 6).  The norm is taken over the
+ * whole row of H elements; the scales per group.
+ *   y = bf16(bf16(x * r) * w),  r = 1 / sqrt(sum(x^2)/H + eps)
+ *
+ *   x [M, H] bf16 (ldx), w [H] bf16, eps >= 0; other arguments as in
+ *   fp8q_group_quant with K = H.
+ */
+FP8Q_API fp8q_status fp8q_rmsnorm_quant(const void* x, const void* w, float eps, int64_t M, int64_t H,
+                               int64_t ldx, int group_size, int ue8m0, void* q, int64_t ldq,
+                               float* scales, int64_t s_stride_m, int64_t s_stride_g,
+                               void* stream);
+
+/*
+ * fp8q_silu_mul_quant -- silu_and_mul_dynamic_per_token_quant (group_size = I)
+ * and silu_and_mul_per_block_quant (group_size = 128) ("Helion in vLLM",
+ * "Kernels integrated into vLLM", items 3 and 7).
+ *   row m of x is [gate (I) | up (I)];  y = bf16(silu(gate) * up),
+ *   silu(t) = t / (1 + exp(-t))
+ *
+ *   x [M, 2I] bf16 (ldx >= 2I, multiple of 8); q [M, I] (ldq); other
+ *   arguments as in fp8q_group_quant with K = I.
+ */
+FP8Q_API fp8q_status fp8q_silu_mul_quant(const void* x, int64_t M, int64_t I, int64_t ldx, int group_size,
+                                int ue8m0, void* q, int64_t ldq, float* scales,
+                                int64_t s_stride_m, int64_t s_stride_g, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Scaled FP8 GEMMs                                                          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * fp8q_scaled_mm -- scaled_mm ("Helion in vLLM", "Kernels integrated into
+ * vLLM", item 8; the FP8_Dynamic scheme of "Helion linear backend"
+ * (aihirek.info), section "Autotuning selects the variant").
+ *   y[m, n] = bf16_rn( sa(m) * sb(n) * sum_k qa[m, k] * qb[n, k] )
+ *
+ *   a_q      e4m3 [M, K], rows contiguous (row stride K)
+ *   b_q      e4m3 [N, K], rows contiguous (nn.Linear weight layout)
+ *   a_scale  fp32: [M] if a_per_token else [1]
+ *   b_scale  fp32: [N] if b_per_channel else [1]
+ *   M >= 0 (M = 0 is a no-op), N > 0 a multiple of 16, K > 0 a multiple of 16
+ *   y        bf16 [M, N], leading dimension ldy (>= N, multiple of 8)
+ *   workspace / ws_bytes  device scratch of at least
+ *            fp8q_workspace_bytes(M, N, K, 0) bytes (may be NULL when that
+ *            is 0).  It must be zero-filled before its first use.  A call
+ *            whose kernels finish normally leaves the part that must start
+ *            at zero (the split-K arrival counters) at zero again, so the
+ *            same workspace can be reused without clearing; after
+ *            FP8Q_ERR_TIMEOUT, zero-fill it again.  Calls that share one
+ *            workspace must not overlap in time.
+ */
+FP8Q_API fp8q_status fp8q_scaled_mm(const void* a_q, const void* b_q, const float* a_scale,
+                           int a_per_token, const float* b_scale, int b_per_channel, int64_t M,
+                           int64_t N, int64_t K, void* y, int64_t ldy, void* workspace,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * fp8q_scaled_mm_blockwise -- scaled_mm_blockwise ("Helion in vLLM",
+ * "Kernels integrated into vLLM", item 9; the Block_FP8 scheme of "Helion
+ * linear backend" (aihirek.info), section "Autotuning selects the variant").
+ *   y[m, n] = bf16_rn( sum_kb sa[m, kb] * sb[n/128, kb] * P_kb[m, n] ),
+ *   P_kb = fp32 sum over k in [128 kb, 128 kb + 128) of qa[m, k] * qb[n, k]
+ *
+ *   a_scale  fp32, one scale per 1x128 group of A: sa[m, kb] at
+ *            a_scale[m*as_stride_m + kb*as_stride_kb]
+ *   b_scale  fp32 [N/128, K/128] row-major, one scale per 128x128 block of B
+ *   N and K multiples of 128; other arguments as in fp8q_scaled_mm, with
+ *   fp8q_workspace_bytes(M, N, K, 1).
+ */
+FP8Q_API fp8q_status fp8q_scaled_mm_blockwise(const void* a_q, const void* b_q, const float* a_scale,
+                                     int64_t as_stride_m, int64_t as_stride_kb,
+                                     const float* b_scale, int64_t M, int64_t N, int64_t K,
+                                     void* y, int64_t ldy, void* workspace, size_t ws_bytes,
+                                     void* stream);
+
+/* Bytes of scratch the GEMM of this shape needs (0 if none); blockwise = 0/1.
+ * Depends only on the shape and the variant the library picks for it. */
+FP8Q_API size_t fp8q_workspace_bytes(int64_t M, int64_t N, int64_t K, int blockwise);
+
+/* ------------------------------------------------------------------------ */
+/* GEMM variant selection (Split-K / Swap-AB / tile width)                   */
+/* ------------------------------------------------------------------------ */
+
+/* A GEMM variant ("Helion linear backend" (aihirek.info), section "Single
+ * GEMM implementation handles several algorithms"): swap_ab = 1 computes
+ * (B A^T)^T so the tokens sit in the MMA's N slot; split_k > 1 divides the K
+ * loop among that many CTAs per output tile; block_n is the MMA N extent. */
+typedef struct {
+    int swap_ab;
+    int split_k;
+    int block_n;
+} fp8q_gemm_variant;
+
+/* The variant the library would run for this shape.  Returns FP8Q_OK. */
+FP8Q_API fp8q_status fp8q_select_gemm_variant(int64_t M, int64_t N, int64_t K, int blockwise,
+                                     fp8q_gemm_variant* out);
+
+/* Force a variant for every following GEMM call in this process (testing and
+ * tuning only; not thread-safe).  NULL restores automatic selection.  Returns
+ * FP8Q_ERR_INVALID_ARG if the variant is malformed (block_n not one of
+ * 16, 32, 64, 128, 256; split_k < 1). */
+FP8Q_API fp8q_status fp8q_force_gemm_variant(const fp8q_gemm_variant* v);
+
+/* ------------------------------------------------------------------------ */
+/* Status                                                                    */
+/* ------------------------------------------------------------------------ */
+
+/* Synchronizes `stream`, then returns and clears the device status word of
+ * the current device (FP8Q_OK, or FP8Q_ERR_TIMEOUT if a kernel gave up on a
+ * wait since the last read).  FP8Q_ERR_CUDA if the synchronization failed. */
+FP8Q_API fp8q_status fp8q_last_device_status(void* stream);
+
+/* Static description of a status code (never NULL). */
+FP8Q_API const char* fp8q_status_string(fp8q_status s);
+
+/* Library version string, e.g. "fp8q 0.1 sm_100a". */
+FP8Q_API const char* fp8q_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */

@@ -1,0 +1,77 @@
+"""The C-ABI library: it loads, exports every function include/fp8q.h declares,
+and validates arguments on the host (no kernel is launched by these calls, so
+they run without a GPU)."""
+import ctypes
+
+import pytest
+
+import fp8_quantized_linear_rms_b200 as fq
+
+
+def test_library_exports_every_declared_function():
+    names = fq.header_functions()
+    assert len(names) == 11
+    for n in names:
+        assert hasattr(fq.lib, n), n
+        assert callable(getattr(fq, n)), f"binding lacks {n}"
+
+
+def test_status_strings_and_version():
+    assert fq.fp8q_version().startswith("fp8q")
+    for s in range(5):
+        assert fq.fp8q_status_string(s)
+    assert fq.fp8q_status_string(99) == "unknown status"
+
+
+def test_invalid_arguments_rejected_before_launch():
+    L = fq.lib
+    fake = 1 << 20   # a 16-byte-aligned address that is never dereferenced
+    # null pointers with M > 0
+    assert L.fp8q_group_quant(None, 4, 256, 256, 128, 0, fake, 256, fake, 2, 1, None) == fq.ERR_INVALID_ARG
+    # group size not 128 or K; K not a multiple of 16; ldx too small; bad ue8m0
+    assert L.fp8q_group_quant(fake, 4, 256, 256, 64, 0, fake, 256, fake, 2, 1, None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_group_quant(fake, 4, 200, 208, 200, 0, fake, 208, fake, 1, 1, None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_group_quant(fake, 4, 256, 128, 128, 0, fake, 256, fake, 2, 1, None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_group_quant(fake, 4, 256, 256, 128, 3, fake, 256, fake, 2, 1, None) == fq.ERR_INVALID_ARG
+    # misaligned input
+    assert L.fp8q_group_quant(fake + 2, 4, 256, 256, 128, 0, fake, 256, fake, 2, 1, None) == fq.ERR_INVALID_ARG
+    # negative eps, silu ldx < 2I
+    assert L.fp8q_rmsnorm_quant(fake, fake, ctypes.c_float(-1.0), 4, 256, 256, 128, 0, fake, 256, fake,
+                                2, 1, None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_silu_mul_quant(fake, 4, 256, 256, 128, 0, fake, 256, fake, 2, 1, None) == fq.ERR_INVALID_ARG
+    # GEMMs: N % 16, K % 16, ldy < N, blockwise K % 128 and N % 128
+    assert L.fp8q_scaled_mm(fake, fake, fake, 1, fake, 1, 4, 24, 256, fake, 24, None, 0, None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_scaled_mm(fake, fake, fake, 1, fake, 1, 4, 32, 40, fake, 32, None, 0, None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_scaled_mm(fake, fake, fake, 1, fake, 1, 4, 32, 256, fake, 16, None, 0, None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_scaled_mm_blockwise(fake, fake, fake, 2, 1, fake, 4, 128, 200, fake, 128, None, 0,
+                                      None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_scaled_mm_blockwise(fake, fake, fake, 2, 1, fake, 4, 192, 256, fake, 192, None, 0,
+                                      None) == fq.ERR_INVALID_ARG
+
+
+def test_zero_rows_is_a_noop_without_pointers():
+    L = fq.lib
+    assert L.fp8q_group_quant(None, 0, 256, 256, 128, 0, None, 256, None, 2, 1, None) == fq.OK
+    assert L.fp8q_scaled_mm(None, None, None, 1, None, 1, 0, 256, 256, None, 256, None, 0, None) == fq.OK
+    assert L.fp8q_scaled_mm_blockwise(None, None, None, 2, 1, None, 0, 256, 256, None, 256, None, 0,
+                                      None) == fq.OK
+
+
+def test_variant_selection_host_logic():
+    # small M: Swap-AB with tokens padded to 16/32/64; large M: no swap
+    assert fq.fp8q_select_gemm_variant(1, 10240, 5120, True)["swap_ab"] == 1
+    assert fq.fp8q_select_gemm_variant(1, 10240, 5120, True)["block_n"] == 16
+    assert fq.fp8q_select_gemm_variant(33, 10240, 5120, True)["block_n"] == 64
+    v = fq.fp8q_select_gemm_variant(8192, 51200, 5120, False)
+    assert v["swap_ab"] == 0 and v["split_k"] == 1
+    # Split-K only where tiles cannot fill the SMs; every split non-empty
+    v = fq.fp8q_select_gemm_variant(16, 5120, 25600, True)
+    assert v["split_k"] > 1
+    assert fq.fp8q_workspace_bytes(16, 5120, 25600, True) > 0
+    assert fq.fp8q_workspace_bytes(8192, 51200, 5120, False) == 0
+    # forcing
+    fq.fp8q_force_gemm_variant(0, 2, 256)
+    assert fq.fp8q_select_gemm_variant(8192, 51200, 5120, False) == {"swap_ab": 0, "split_k": 2, "block_n": 256}
+    fq.fp8q_force_gemm_variant()
+    with pytest.raises(fq.Fp8qError):
+        fq.fp8q_force_gemm_variant(0, 1, 48)
