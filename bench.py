@@ -41,10 +41,13 @@ EPS = 1e-6
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=1500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--m", type=int, default=2048)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--sweep", default=None,
+                    help="per-op timing instead of the step: quant, gemm8b, decode32b, prefill32b, all")
+    ap.add_argument("--reps", type=int, default=20)
     return ap.parse_args()
 
 
@@ -384,12 +387,138 @@ def cpu_baseline_leg(args):
             "kind": "oracle", "sample": r["cpu_baseline"]["sample"] + ", 1 step"}
 
 
+# ------------------------------------------------------------------ per-op sweep
+def run_sweep(args):
+    """Time every op of the path on the config shapes, one JSON line per case:
+    device time per launch (CUDA events, median of --reps, L2 flushed before each
+    rep), achieved GB/s or TFLOP/s and the fraction of the measured peak."""
+    import numpy as np
+    import torch
+
+    import fp8_quantized_linear_rms_b200 as fq
+    import fp8q_inputs as inp
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except Exception:
+        pass
+    hbm = peaks.get("hbm_gbs", 6650.0)
+    fp8_peak = 2.0 * peaks.get("bf16_tflops", 1590.0)      # burst: kernels timed alone
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timeit(fn):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.reps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e-3)
+        assert fq.fp8q_last_device_status() == fq.OK
+        return float(np.median(ts))
+
+    def emit(d):
+        print(json.dumps(d), flush=True)
+
+    def bf16_rand(shape, seed, heavy=True):
+        g = torch.Generator(device=dev).manual_seed(seed)
+        x = torch.randn(shape, generator=g, device=dev)
+        if heavy:
+            x = x * (1.0 + 19.0 * (torch.rand(shape[-1], generator=g, device=dev) < 0.01))
+        return x.to(torch.bfloat16)
+
+    which = args.sweep
+    if which in ("quant", "all"):
+        w = {h: bf16_rand((h,), 1, False) * 0.1 + 1.0 for h in (4096, 5120)}
+        for M in (16, 128, 2048, 8192):
+            cases = [("group_quant", 4096), ("rmsnorm_quant", 4096), ("rmsnorm_quant", 5120),
+                     ("silu_mul_quant", 12288), ("silu_mul_quant", 25600)]
+            for op, L in cases:
+                for g in (L, 128):
+                    if op == "silu_mul_quant":
+                        x = bf16_rand((M, 2 * L), 3)
+                        fn = lambda: fq.fp8q_silu_mul_quant(x, g)
+                        nbytes = M * (4 * L + L + 4 * (L // g))
+                    elif op == "rmsnorm_quant":
+                        x = bf16_rand((M, L), 4)
+                        fn = lambda: fq.fp8q_rmsnorm_quant(x, w[L], 1e-6, g)
+                        nbytes = M * (2 * L + L + 4 * (L // g)) + 2 * L
+                    else:
+                        x = bf16_rand((M, L), 5)
+                        fn = lambda: fq.fp8q_group_quant(x, g)
+                        nbytes = M * (2 * L + L + 4 * (L // g))
+                    t = timeit(fn)
+                    emit({"op": op, "M": M, "L": L, "group": g, "us": round(t * 1e6, 2),
+                          "GB/s": round(nbytes / t / 1e9, 1),
+                          "frac_hbm": round(nbytes / t / 1e9 / hbm, 3)})
+                    del x
+
+    def gemm_case(tag, M, N, K, blockwise):
+        a = torch.randint(0, 126, (M, K), dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
+        b = torch.randint(0, 126, (N, K), dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
+        if blockwise:
+            sa = torch.rand((K // 128, M), device=dev) * 1e-3 + 1e-4
+            sb = torch.rand((N // 128, K // 128), device=dev) * 1e-3 + 1e-4
+            ws = fq.make_workspace(M, N, K, True, dev)
+            fn = lambda: fq.fp8q_scaled_mm_blockwise(a, b, sa, sb, a_scale_layout="group_major",
+                                                     workspace=ws)
+        else:
+            sa = torch.rand(M, device=dev) * 1e-3 + 1e-4
+            sb = torch.rand(N, device=dev) * 1e-3 + 1e-4
+            ws = fq.make_workspace(M, N, K, False, dev)
+            fn = lambda: fq.fp8q_scaled_mm(a, b, sa, sb, workspace=ws)
+        t = timeit(fn)
+        flops = 2.0 * M * N * K
+        nbytes = M * K + N * K + 2 * M * N
+        v = fq.fp8q_select_gemm_variant(M, N, K, blockwise)
+        emit({"op": "scaled_mm_blockwise" if blockwise else "scaled_mm", "shape": tag, "M": M,
+              "N": N, "K": K, "variant": v, "us": round(t * 1e6, 2),
+              "TFLOP/s": round(flops / t / 1e12, 1), "frac_fp8_peak": round(flops / t / 1e12 / fp8_peak, 3),
+              "GB/s": round(nbytes / t / 1e9, 1), "frac_hbm": round(nbytes / t / 1e9 / hbm, 3)})
+
+    if which in ("gemm8b", "all"):
+        sh = inp.linear_shapes(inp.QWEN3_8B)
+        for M in (1, 16, 128, 2048):
+            for layer in ("gate_up", "down"):
+                K, N = sh[layer]
+                gemm_case(f"qwen3-8b {layer}", M, N, K, False)
+        for M in (1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096):
+            for layer in ("qkv", "o", "gate_up", "down"):
+                K, N = sh[layer]
+                gemm_case(f"qwen3-8b {layer}", M, N, K, True)
+    if which in ("decode32b", "all"):
+        sh = inp.linear_shapes(inp.QWEN3_32B)
+        for M in (1, 2, 4, 8, 16, 32, 64):
+            for layer in ("qkv", "o", "gate_up", "down"):
+                K, N = sh[layer]
+                gemm_case(f"qwen3-32b {layer}", M, N, K, True)
+    if which in ("prefill32b", "all"):
+        sh = inp.linear_shapes(inp.QWEN3_32B)
+        for bw in (False, True):
+            for layer in ("qkv", "o", "gate_up", "down"):
+                K, N = sh[layer]
+                gemm_case(f"qwen3-32b {layer}", 8192, N, K, bw)
+    return 0
+
+
 def main():
     args = parse()
     os.environ.setdefault("OMP_NUM_THREADS", str(os.cpu_count() or 1))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.sweep:
+        return run_sweep(args)
     if args.impl == "reference":
         if rank != 0:
             return 0

@@ -73,7 +73,7 @@ struct Cfg {
   static constexpr int COL_GROUPS = EPI_WARPS / 4;        // column slices per TMEM lane quadrant
   static constexpr int CPT = BN / COL_GROUPS;              // columns per epilogue thread
   static constexpr int CHUNK = CPT < 32 ? CPT : 32;        // columns per tcgen05.ld
-  static constexpr int NBUF = BW ? 4 : 2;                  // TMEM accumulator buffers
+  static constexpr int NBUF = (BW && BN < 256) ? 4 : 2;    // TMEM accumulator buffers
   static constexpr int TMEM_NEED = NBUF * BN;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                  : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
@@ -97,13 +97,14 @@ __device__ __forceinline__ void unit_coords(const GemmArgs& p, int u, int& ta, i
   kb1 = min(p.kblocks, kb0 + p.kb_per_split);
 }
 
-// Bounded wait that ignores the abort flag: used only to drain in-flight
-// asynchronous work before the CTA exits.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
-  }
+// (a0, a1) += (v0, v1) * (s0, s1) with one paired fp32 FMA (sm_100 f32x2).
+__device__ __forceinline__ void ffma2(float& a0, float& a1, float v0, float v1, float s0, float s1) {
+  uint64_t a, v, sc;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(v0), "f"(v1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(sc) : "f"(s0), "f"(s1));
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a) : "l"(v), "l"(sc));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(a));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -313,29 +314,37 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
 
       if (!BW) {
         // -------- per-token / per-channel scales: one accumulator per tile
+        // Column scales: lane l of the warp loads the scale of column c + l of
+        // every chunk (one load per 32 columns, issued before the wait), and the
+        // products broadcast it with a shuffle.
+        constexpr int NCH = C::CPT / C::CHUNK;
         const int buf = t & 1;
         float srow;
         if (!SWAP) srow = a_valid ? __ldg(p.sa + a_idx * p.sa_sm) : 0.0f;
         else srow = a_valid ? __ldg(p.sb + a_idx * p.sb_sn) : 0.0f;
+        float colsc[NCH];
+#pragma unroll
+        for (int j = 0; j < NCH; ++j) {
+          const int b_idx = b_base + col0 + j * C::CHUNK + lane;
+          if (!SWAP) colsc[j] = (lane < C::CHUNK && b_idx < p.N) ? __ldg(p.sb + b_idx * p.sb_sn) : 0.0f;
+          else colsc[j] = (lane < C::CHUNK && b_idx < p.M) ? __ldg(p.sa + b_idx * p.sa_sm) : 0.0f;
+        }
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[buf], (t >> 1) & 1, abort_flag, p.status))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int c = col0; c < col0 + C::CPT; c += C::CHUNK) {
+#pragma unroll
+        for (int j = 0; j < NCH; ++j) {
+          const int c = col0 + j * C::CHUNK;
           float v[C::CHUNK];
           const uint32_t taddr = tmem_base + lane_addr + buf * BN + c;
           if (C::CHUNK == 32) tmem_ld_32x32b_x32(taddr, v);
           else tmem_ld_32x32b_x16(taddr, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < C::CHUNK; ++i) {
-            const int b_idx = b_base + c + i;
-            float sc;
-            if (!SWAP) sc = b_idx < p.N ? __ldg(p.sb + b_idx * p.sb_sn) : 0.0f;
-            else sc = b_idx < p.M ? __ldg(p.sa + b_idx * p.sa_sm) : 0.0f;
-            v[i] = v[i] * (srow * sc);
-          }
+          for (int i = 0; i < C::CHUNK; ++i)
+            v[i] = v[i] * (srow * __shfl_sync(0xFFFFFFFFu, colsc[j], i));
           if (p.split == 1) emit(c, v);
           else stash(c, v);
         }
@@ -345,36 +354,58 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
         ++t;
         if (p.split > 1) finish_split();
       } else {
-        // -------- blockwise scales: promote each K-block partial into registers
+        // -------- blockwise scales: promote each K-block partial into registers.
+        // The scales of K block kb+1 are loaded while block kb is processed, so
+        // their latency stays off the per-block critical path.  Swap-AB: the
+        // scale varies per column (token); lane l holds that of column c + l.
+        constexpr int NCH = C::CPT / C::CHUNK;
         float acc[C::CPT];
 #pragma unroll
         for (int i = 0; i < C::CPT; ++i) acc[i] = 0.0f;
-        const int nb = SWAP ? ta : (tb * BN) / 128;   // weight block row (constant per tile)
+        // Weight block row of this thread's columns: the whole tile (Swap-AB) or
+        // this warp's 128-column slice (a slice never straddles a block row).
+        const int nb = SWAP ? ta : (tb * BN + col0) / 128;
+        const bool slice_valid = SWAP || (tb * BN + col0) < p.N;
+        float srow_n = 0.0f, colsc_n[NCH];
+        auto load_scales = [&](int kb) {
+          const float sbk = slice_valid ? __ldg(p.sb + nb * p.sb_snb + kb * p.sb_skb) : 0.0f;
+          if (!SWAP) {
+            srow_n = (a_valid && slice_valid) ? __ldg(p.sa + a_idx * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
+          } else {
+#pragma unroll
+            for (int j = 0; j < NCH; ++j) {
+              const int m = b_base + col0 + j * C::CHUNK + lane;
+              colsc_n[j] = (lane < C::CHUNK && m < p.M)
+                               ? __ldg(p.sa + m * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
+            }
+          }
+        };
+        load_scales(kb0);
         for (int kb = kb0; kb < kb1; ++kb) {
           const int pb = pc % NB;
-          const float sbk = __ldg(p.sb + nb * p.sb_snb + kb * p.sb_skb);
-          float srow = 0.0f;
-          if (!SWAP) srow = a_valid ? __ldg(p.sa + a_idx * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
+          const float srow = srow_n;
+          float colsc[NCH];
+#pragma unroll
+          for (int j = 0; j < NCH; ++j) colsc[j] = SWAP ? colsc_n[j] : 0.0f;
+          if (kb + 1 < kb1) load_scales(kb + 1);
           if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[pb], (pc / NB) & 1, abort_flag, p.status))) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < C::CPT; c += C::CHUNK) {
+          for (int j = 0; j < NCH; ++j) {
+            const int c = j * C::CHUNK;
             float v[C::CHUNK];
             const uint32_t taddr = tmem_base + lane_addr + pb * BN + col0 + c;
             if (C::CHUNK == 32) tmem_ld_32x32b_x32(taddr, v);
             else tmem_ld_32x32b_x16(taddr, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < C::CHUNK; ++i) {
-              float sc = srow;
-              if (SWAP) {
-                const int m = b_base + col0 + c + i;
-                sc = m < p.M ? __ldg(p.sa + m * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
-              }
-              acc[c + i] = fmaf(v[i], sc, acc[c + i]);
+            for (int i = 0; i < C::CHUNK; i += 2) {
+              const float s0 = SWAP ? __shfl_sync(0xFFFFFFFFu, colsc[j], i) : srow;
+              const float s1 = SWAP ? __shfl_sync(0xFFFFFFFFu, colsc[j], i + 1) : srow;
+              ffma2(acc[c + i], acc[c + i + 1], v[i], v[i + 1], s0, s1);
             }
           }
           tc_fence_before();
@@ -504,7 +535,7 @@ fp8q_gemm_variant g_force{0, 1, 128};
 bool variant_supported(const fp8q_gemm_variant& v, int blockwise) {
   if (v.split_k < 1 || v.split_k > 64) return false;
   if (v.swap_ab) return v.block_n == 16 || v.block_n == 32 || v.block_n == 64 || v.block_n == 128;
-  if (blockwise) return v.block_n == 128;
+  if (blockwise) return v.block_n == 128 || v.block_n == 256;
   return v.block_n == 128 || v.block_n == 256;
 }
 
@@ -547,7 +578,7 @@ fp8q_gemm_variant auto_variant(int64_t M, int64_t N, int64_t K, int blockwise) {
     v.block_n = 128;
   } else {
     v.swap_ab = 0;
-    v.block_n = blockwise ? 128 : 256;
+    v.block_n = 256;
   }
   const int64_t rows_a = v.swap_ab ? N : M, rows_b = v.swap_ab ? M : N;
   const int64_t tiles = ((rows_a + BM - 1) / BM) * ((rows_b + v.block_n - 1) / v.block_n);
@@ -619,7 +650,7 @@ fp8q_status run_gemm(const void* a_q, const void* b_q, GemmArgs& p, const Plan& 
   p.rows_a = p.M;
   p.rows_b = p.N;
   if (bn == 128) return launch_gemm<128, false, BW>(a_q, b_q, p, stream);
-  if (!BW && bn == 256) return launch_gemm<256, false, false>(a_q, b_q, p, stream);
+  if (bn == 256) return launch_gemm<256, false, BW>(a_q, b_q, p, stream);
   return FP8Q_ERR_UNSUPPORTED;
 }
 

@@ -23,7 +23,7 @@ if torch.cuda.is_available():
     import fp8_quantized_linear_rms_b200 as fq   # fails loudly if libfp8q.so is missing
 
 PT_VARIANTS = [(0, 128), (0, 256), (1, 16), (1, 32), (1, 64), (1, 128)]
-BW_VARIANTS = [(0, 128), (1, 16), (1, 32), (1, 64), (1, 128)]
+BW_VARIANTS = [(0, 128), (0, 256), (1, 16), (1, 32), (1, 64), (1, 128)]
 
 
 @pytest.fixture(autouse=True)
