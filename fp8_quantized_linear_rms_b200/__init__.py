@@ -5,7 +5,7 @@ dtypes and shapes enough to pass the right pointers, and calls the C ABI of
 ``include/fp8q.h`` with the current CUDA stream.  All arithmetic runs in the
 library's kernels; there is no CPU or PyTorch fallback, and importing this
 package fails loudly if ``libfp8q.so`` is missing (build it with
-``python -m fp8_quantized_linear_rms_b200.build``).
+``python fp8_quantized_linear_rms_b200/build.py``).
 
 The names match the C ABI:
   fp8q_group_quant, fp8q_rmsnorm_quant, fp8q_silu_mul_quant   (activation quant)
@@ -27,7 +27,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fp8q.h")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libfp8q.so not found at {LIB_PATH}; build it with "
-                      "`python -m fp8_quantized_linear_rms_b200.build`")
+                      "`python fp8_quantized_linear_rms_b200/build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -56,6 +56,8 @@ _SIGS = {
                               ctypes.c_size_t, _P]),
     "fp8q_scaled_mm_blockwise": (_INT, [_P, _P, _P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I64,
                                         _P, ctypes.c_size_t, _P]),
+    "fp8q_scaled_mm_blockwise_noalloc": (_INT, [_P, _P, _P, _I64, _I64, _P, _I64, _I64, _I64, _P,
+                                                _I64, _P]),
     "fp8q_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, _INT]),
     "fp8q_select_gemm_variant": (_INT, [_I64, _I64, _I64, _INT, ctypes.POINTER(GemmVariant)]),
     "fp8q_force_gemm_variant": (_INT, [ctypes.POINTER(GemmVariant)]),
@@ -247,6 +249,32 @@ def fp8q_scaled_mm_blockwise(a_q: torch.Tensor, b_q: torch.Tensor, a_scale: torc
                                       b_scale.data_ptr(), M, N, K, y.data_ptr(),
                                       _rowmajor(y, "y"), wp, wn, _stream(stream))
     _check("fp8q_scaled_mm_blockwise", st)
+    return y
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def fp8q_scaled_mm_blockwise_noalloc(a_q: torch.Tensor, b_q: torch.Tensor, a_scale: torch.Tensor,
+                                     b_scale: torch.Tensor, a_scale_layout: str = "row_major",
+                                     y=None, stream=None):
+    """fp8q_scaled_mm_blockwise without a workspace: the library's fixed 16 MiB
+    scratch array is used instead (calls that overlap on the GPU race)."""
+    for t, n in ((a_q, "a_q"), (b_q, "b_q")):
+        _need(t, torch.float8_e4m3fn, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _need(a_scale, torch.float32, "a_scale")
+    _need(b_scale, torch.float32, "b_scale")
+    M, K = a_q.shape
+    N = b_q.shape[0]
+    sm, skb = (1, M) if a_scale_layout == "group_major" else (K // 128, 1)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_q.device)
+    st = lib.fp8q_scaled_mm_blockwise_noalloc(a_q.data_ptr(), b_q.data_ptr(), a_scale.data_ptr(),
+                                              sm, skb, b_scale.data_ptr(), M, N, K, y.data_ptr(),
+                                              _rowmajor(y, "y"), _stream(stream))
+    _check("fp8q_scaled_mm_blockwise_noalloc", st)
     return y
 
 

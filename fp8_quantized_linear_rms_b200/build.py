@@ -1,6 +1,6 @@
 """Build libfp8q.so in-tree with nvcc for sm_100a (B200).
 
-    python -m fp8_quantized_linear_rms_b200.build [--force]
+    python fp8_quantized_linear_rms_b200/build.py [--force]
 
 Objects go to ``_build/`` at the repository root; the shared library to
 ``fp8_quantized_linear_rms_b200/libfp8q.so``.  Only stale objects are rebuilt.

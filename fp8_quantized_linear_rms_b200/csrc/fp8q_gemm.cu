@@ -763,3 +763,64 @@ extern "C" fp8q_status fp8q_scaled_mm_blockwise(const void* a_q, const void* b_q
   p.ldy = ldy;
   return run_gemm<true>(a_q, b_q, p, pl, workspace, static_cast<cudaStream_t>(stream));
 }
+
+// ------------------------------------------------------------ no-allocation path
+// Split-K scratch of fp8q_scaled_mm_blockwise_noalloc: one fixed device array,
+// shared by every call on a device, so the call allocates nothing.  Host code
+// must not pass the symbol itself to a kernel (on the host it names a
+// stand-in, not device memory): its device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+namespace {
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FP8Q_NOALLOC_SCRATCH_BYTES];
+
+void* noalloc_scratch_ptr() {
+  static std::mutex mu;
+  static void* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    cache[dev] = p;
+  }
+  return cache[dev];
+}
+}  // namespace
+
+extern "C" fp8q_status fp8q_scaled_mm_blockwise_noalloc(const void* a_q, const void* b_q,
+                                                        const float* a_scale, int64_t as_stride_m,
+                                                        int64_t as_stride_kb, const float* b_scale,
+                                                        int64_t M, int64_t N, int64_t K, void* y,
+                                                        int64_t ldy, void* stream) {
+  fp8q_status st = check_gemm(a_q, b_q, a_scale, b_scale, M, N, K, y, ldy);
+  if (st != FP8Q_OK) return st;
+  if (N % 128 != 0 || K % 128 != 0 || as_stride_m < 0 || as_stride_kb < 0)
+    return FP8Q_ERR_INVALID_ARG;
+  if (M == 0) return FP8Q_OK;
+  const fp8q_gemm_variant v = pick_variant(M, N, K, 1);
+  if (!variant_supported(v, 1)) return FP8Q_ERR_UNSUPPORTED;
+  const Plan pl = make_plan(M, N, K, 1, v);
+  if (pl.ws_bytes > FP8Q_NOALLOC_SCRATCH_BYTES) return FP8Q_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pl.ws_bytes > 0) {
+    scratch = noalloc_scratch_ptr();
+    if (!scratch) return FP8Q_ERR_CUDA;
+    if (cudaMemsetAsync(scratch, 0, pl.counter_bytes, s) != cudaSuccess) return FP8Q_ERR_CUDA;
+  }
+  GemmArgs p{};
+  p.K = static_cast<int>(K);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.sa = a_scale;
+  p.sa_sm = as_stride_m;
+  p.sa_skb = as_stride_kb;
+  p.sb = b_scale;
+  p.sb_sn = 0;
+  p.sb_snb = K / 128;
+  p.sb_skb = 1;
+  p.y = static_cast<uint16_t*>(y);
+  p.ldy = ldy;
+  return run_gemm<true>(a_q, b_q, p, pl, scratch, s);
+}

@@ -166,6 +166,38 @@ FP8Q_API fp8q_status fp8q_scaled_mm_blockwise(const void* a_q, const void* b_q, 
                                      void* y, int64_t ldy, void* workspace, size_t ws_bytes,
                                      void* stream);
 
+/*
+ * fp8q_scaled_mm_blockwise_noalloc -- the same GEMM as
+ * fp8q_scaled_mm_blockwise, for callers that cannot hand the library any
+ * device memory beyond their inputs and outputs.  (The pages have no
+ * counterpart; this is a deployment convenience of this library.)
+ *
+ * Some callers cannot allocate: an inference engine that reserved all free
+ * HBM for its KV cache at start-up, a plugin interface that gives a kernel
+ * only its input and output buffers, or a latency-critical path where
+ * cudaMalloc / cudaFree (which can synchronize the device) are not allowed.
+ * This entry point allocates nothing.  Its split-K scratch is one fixed
+ * device array of FP8Q_NOALLOC_SCRATCH_BYTES (16 MiB) inside the library,
+ * which every GPU that loads the library holds until the process exits.
+ *
+ *   Arguments are those of fp8q_scaled_mm_blockwise without the workspace.
+ *   Returns FP8Q_ERR_UNSUPPORTED, launching nothing, when the shape's split-K
+ *   scratch (fp8q_workspace_bytes(M, N, K, 1)) exceeds
+ *   FP8Q_NOALLOC_SCRATCH_BYTES.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   Every call clears the part of the array that must start at zero (the
+ *   split-K arrival counters) with cudaMemsetAsync on its stream.
+ *   All calls on a device share the one array: calls that can overlap on the
+ *   GPU (different streams without ordering) race and give wrong results.
+ */
+#define FP8Q_NOALLOC_SCRATCH_BYTES (16u << 20)
+FP8Q_API fp8q_status fp8q_scaled_mm_blockwise_noalloc(const void* a_q, const void* b_q,
+                                                      const float* a_scale, int64_t as_stride_m,
+                                                      int64_t as_stride_kb, const float* b_scale,
+                                                      int64_t M, int64_t N, int64_t K, void* y,
+                                                      int64_t ldy, void* stream);
+
 /* Bytes of scratch the GEMM of this shape needs (0 if none); blockwise = 0/1.
  * Depends only on the shape and the variant the library picks for it. */
 FP8Q_API size_t fp8q_workspace_bytes(int64_t M, int64_t N, int64_t K, int blockwise);

@@ -10,7 +10,7 @@ import fp8_quantized_linear_rms_b200 as fq
 
 def test_library_exports_every_declared_function():
     names = fq.header_functions()
-    assert len(names) == 11
+    assert len(names) == 12
     for n in names:
         assert hasattr(fq.lib, n), n
         assert callable(getattr(fq, n)), f"binding lacks {n}"

@@ -1,0 +1,70 @@
+"""fp8q_scaled_mm_blockwise_noalloc, the GEMM entry point for callers that
+cannot allocate device memory (an engine that pre-reserved all free HBM, a
+plugin that is handed only its inputs and outputs, a path where cudaMalloc's
+possible device synchronization is not allowed).  It runs the blockwise GEMM
+with the library's fixed 16 MiB scratch array instead of a caller workspace.
+
+Called through the C ABI, on split-K shapes (so the scratch is really used),
+twice in a row per shape: both calls must agree with the workspace entry point
+fp8q_scaled_mm_blockwise within the GEMM tolerance of the other tests
+(|y - y_ref| <= 2^-8 |y_ref| + 1e-3 sum_k |a_k b_k|).  This file is collected
+last on purpose, and passes alone in a fresh process as well.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fp8q_inputs as inp
+import oracle
+from helpers import bf16_to_np, gemm_tolerance_check, to_dev_codes
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import fp8_quantized_linear_rms_b200 as fq   # fails loudly if libfp8q.so is missing
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 5120, 25600), (1, 10240, 5120), (64, 4096, 12288)])
+def test_noalloc_matches_workspace_entry_point(M, N, K):
+    fq.fp8q_force_gemm_variant()
+    v = fq.fp8q_select_gemm_variant(M, N, K, True)
+    assert v["split_k"] > 1, "the shape must exercise the split-K scratch"
+    assert 0 < fq.fp8q_workspace_bytes(M, N, K, True) <= fq.NOALLOC_SCRATCH_BYTES
+    a = to_dev_codes(inp.random_e4m3_codes(M + 1, (M, K)))
+    b = to_dev_codes(inp.random_e4m3_codes(N + 2, (N, K)))
+    sa = torch.from_numpy(inp.random_scales(3, (M, K // 128))).cuda()
+    sb = torch.from_numpy(inp.random_scales(4, (N // 128, K // 128))).cuda()
+    y_ws = fq.fp8q_scaled_mm_blockwise(a, b, sa, sb, workspace=fq.make_workspace(M, N, K, True))
+    torch.cuda.synchronize()
+    # |a_k b_k| sums for the tolerance, from the oracle on every row
+    _, absdot = oracle.scaled_mm_blockwise(a.view(torch.uint8).cpu().numpy(),
+                                           b.view(torch.uint8).cpu().numpy(),
+                                           sa.cpu().numpy(), sb.cpu().numpy())
+    ref = bf16_to_np(y_ws).astype(np.float64)
+    stream = torch.cuda.current_stream().cuda_stream
+    for call in range(2):
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        st = fq.lib.fp8q_scaled_mm_blockwise_noalloc(a.data_ptr(), b.data_ptr(), sa.data_ptr(),
+                                                     K // 128, 1, sb.data_ptr(), M, N, K,
+                                                     y.data_ptr(), N, stream)
+        assert st == fq.OK, fq.fp8q_status_string(st)
+        torch.cuda.synchronize()
+        assert fq.fp8q_last_device_status() == fq.OK
+        gemm_tolerance_check(bf16_to_np(y), ref, absdot, f"noalloc call {call + 1}")
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    M, N, K = 256, 4096, 12288
+    fq.fp8q_force_gemm_variant(0, 16, 256)      # 16 x 32 tiles x 16 splits of 128x256 fp32
+    try:
+        assert fq.fp8q_workspace_bytes(M, N, K, True) > fq.NOALLOC_SCRATCH_BYTES
+        a = torch.zeros((M, K), dtype=torch.uint8, device="cuda")
+        b = torch.zeros((N, K), dtype=torch.uint8, device="cuda")
+        s = torch.ones(N * K // 128, dtype=torch.float32, device="cuda")
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        st = fq.lib.fp8q_scaled_mm_blockwise_noalloc(a.data_ptr(), b.data_ptr(), s.data_ptr(),
+                                                     K // 128, 1, s.data_ptr(), M, N, K,
+                                                     y.data_ptr(), N, None)
+        assert st == fq.ERR_UNSUPPORTED
+    finally:
+        fq.fp8q_force_gemm_variant()
