@@ -69,10 +69,10 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
-  static constexpr int EPI_WARPS = (BW && BN >= 128) ? 8 : 4;
+  static constexpr int EPI_WARPS = (BW && BN >= 256) ? 16 : ((BW && BN >= 128) ? 8 : 4);
   static constexpr int COL_GROUPS = EPI_WARPS / 4;        // column slices per TMEM lane quadrant
   static constexpr int CPT = BN / COL_GROUPS;              // columns per epilogue thread
-  static constexpr int CHUNK = CPT < 32 ? CPT : 32;        // columns per tcgen05.ld
+  static constexpr int CHUNK = (EPI_WARPS == 16 || CPT < 32) ? 16 : 32;  // columns per tcgen05.ld
   static constexpr int NBUF = (BW && BN < 256) ? 4 : 2;    // TMEM accumulator buffers
   static constexpr int TMEM_NEED = NBUF * BN;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
@@ -97,14 +97,24 @@ __device__ __forceinline__ void unit_coords(const GemmArgs& p, int u, int& ta, i
   kb1 = min(p.kblocks, kb0 + p.kb_per_split);
 }
 
-// (a0, a1) += (v0, v1) * (s0, s1) with one paired fp32 FMA (sm_100 f32x2).
-__device__ __forceinline__ void ffma2(float& a0, float& a1, float v0, float v1, float s0, float s1) {
-  uint64_t a, v, sc;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(v0), "f"(v1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(sc) : "f"(s0), "f"(s1));
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a) : "l"(v), "l"(sc));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(a));
+// acc += (r0, r1) * sc: one paired fp32 FMA (sm_100 .f32x2) on a 64-bit
+// accumulator pair; r0, r1 are adjacent registers of a tcgen05.ld.
+__device__ __forceinline__ void ffma2_acc(uint64_t& acc, uint32_t r0, uint32_t r1, uint64_t sc) {
+  asm("{\n\t.reg .b64 v;\n\t"
+      "mov.b64 v, {%1, %2};\n\t"
+      "fma.rn.f32x2 %0, v, %3, %0;\n\t}"
+      : "+l"(acc)
+      : "r"(r0), "r"(r1), "l"(sc));
+}
+
+__device__ __forceinline__ uint64_t pair_f32(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void unpair_f32(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -359,35 +369,48 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
         // their latency stays off the per-block critical path.  Swap-AB: the
         // scale varies per column (token); lane l holds that of column c + l.
         constexpr int NCH = C::CPT / C::CHUNK;
-        float acc[C::CPT];
+        uint64_t acc[C::CPT / 2];                      // fp32 pairs, columns 2i, 2i+1
 #pragma unroll
-        for (int i = 0; i < C::CPT; ++i) acc[i] = 0.0f;
+        for (int i = 0; i < C::CPT / 2; ++i) acc[i] = 0ull;
         // Weight block row of this thread's columns: the whole tile (Swap-AB) or
         // this warp's 128-column slice (a slice never straddles a block row).
         const int nb = SWAP ? ta : (tb * BN + col0) / 128;
         const bool slice_valid = SWAP || (tb * BN + col0) < p.N;
-        float srow_n = 0.0f, colsc_n[NCH];
-        auto load_scales = [&](int kb) {
-          const float sbk = slice_valid ? __ldg(p.sb + nb * p.sb_snb + kb * p.sb_skb) : 0.0f;
+        // Scales of the next SD K blocks are kept in flight in a register ring
+        // (stage 0 = the block being promoted), so the global-load latency of
+        // a block's scales overlaps the promotion of the SD-1 blocks before it.
+        constexpr int SD = 4;
+        float srow_q[SD], colsc_q[SD][NCH];
+        auto load_scales = [&](int kb, float& srow_o, float* colsc_o) {
+          const bool in = kb < kb1;
+          const float sbk = (in && slice_valid) ? __ldg(p.sb + nb * p.sb_snb + kb * p.sb_skb) : 0.0f;
           if (!SWAP) {
-            srow_n = (a_valid && slice_valid) ? __ldg(p.sa + a_idx * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
+            srow_o = (in && a_valid && slice_valid) ? __ldg(p.sa + a_idx * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
           } else {
+            srow_o = 0.0f;
 #pragma unroll
             for (int j = 0; j < NCH; ++j) {
               const int m = b_base + col0 + j * C::CHUNK + lane;
-              colsc_n[j] = (lane < C::CHUNK && m < p.M)
+              colsc_o[j] = (in && lane < C::CHUNK && m < p.M)
                                ? __ldg(p.sa + m * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
             }
           }
         };
-        load_scales(kb0);
+#pragma unroll
+        for (int q = 0; q < SD; ++q) load_scales(kb0 + q, srow_q[q], colsc_q[q]);
         for (int kb = kb0; kb < kb1; ++kb) {
           const int pb = pc % NB;
-          const float srow = srow_n;
+          const uint64_t srow2 = pair_f32(srow_q[0], srow_q[0]);
           float colsc[NCH];
 #pragma unroll
-          for (int j = 0; j < NCH; ++j) colsc[j] = SWAP ? colsc_n[j] : 0.0f;
-          if (kb + 1 < kb1) load_scales(kb + 1);
+          for (int j = 0; j < NCH; ++j) colsc[j] = SWAP ? colsc_q[0][j] : 0.0f;
+#pragma unroll
+          for (int q = 0; q + 1 < SD; ++q) {
+            srow_q[q] = srow_q[q + 1];
+#pragma unroll
+            for (int j = 0; j < NCH; ++j) colsc_q[q][j] = colsc_q[q + 1][j];
+          }
+          load_scales(kb + SD, srow_q[SD - 1], colsc_q[SD - 1]);
           if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[pb], (pc / NB) & 1, abort_flag, p.status))) {
             ok = false;
             break;
@@ -395,17 +418,17 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int j = 0; j < NCH; ++j) {
-            const int c = j * C::CHUNK;
-            float v[C::CHUNK];
-            const uint32_t taddr = tmem_base + lane_addr + pb * BN + col0 + c;
-            if (C::CHUNK == 32) tmem_ld_32x32b_x32(taddr, v);
-            else tmem_ld_32x32b_x16(taddr, v);
+            uint32_t r[C::CHUNK];
+            const uint32_t taddr = tmem_base + lane_addr + pb * BN + col0 + j * C::CHUNK;
+            if (C::CHUNK == 32) tmem_ld_32x32b_x32_raw(taddr, r);
+            else tmem_ld_32x32b_x16_raw(taddr, r);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < C::CHUNK; i += 2) {
-              const float s0 = SWAP ? __shfl_sync(0xFFFFFFFFu, colsc[j], i) : srow;
-              const float s1 = SWAP ? __shfl_sync(0xFFFFFFFFu, colsc[j], i + 1) : srow;
-              ffma2(acc[c + i], acc[c + i + 1], v[i], v[i + 1], s0, s1);
+              const uint64_t sc = SWAP ? pair_f32(__shfl_sync(0xFFFFFFFFu, colsc[j], i),
+                                                  __shfl_sync(0xFFFFFFFFu, colsc[j], i + 1))
+                                       : srow2;
+              ffma2_acc(acc[(j * C::CHUNK + i) / 2], r[i], r[i + 1], sc);
             }
           }
           tc_fence_before();
@@ -416,8 +439,11 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
         if (!ok) break;
 #pragma unroll
         for (int c = 0; c < C::CPT; c += C::CHUNK) {
-          if (p.split == 1) emit(col0 + c, acc + c);
-          else stash(col0 + c, acc + c);
+          float v[C::CHUNK];
+#pragma unroll
+          for (int i = 0; i < C::CHUNK; i += 2) unpair_f32(acc[(c + i) / 2], v[i], v[i + 1]);
+          if (p.split == 1) emit(col0 + c, v);
+          else stash(col0 + c, v);
         }
         if (p.split > 1) finish_split();
       }
@@ -540,6 +566,7 @@ bool variant_supported(const fp8q_gemm_variant& v, int blockwise) {
 }
 
 int epi_warps(const fp8q_gemm_variant& v, int blockwise) {
+  if (blockwise && v.block_n >= 256) return 16;
   return (blockwise && v.block_n >= 128) ? 8 : 4;
 }
 

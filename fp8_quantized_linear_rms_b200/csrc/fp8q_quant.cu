@@ -109,19 +109,54 @@ __device__ __forceinline__ uint32_t f2_to_e4m3x2(uint64_t v) {
 // ends p(1 - delta) and p(1 + delta) (each one more rounding) bracket v.
 // Rounding to nearest is monotone, so if both ends round to the same code, v
 // rounds to it as well; otherwise the element takes the exact slow path.
-constexpr float kBf16Lo = 1.0f - 0x1p-20f, kBf16Hi = 1.0f + 0x1p-20f;   // errors <= 2^-21
+constexpr float kBf16Lo = 1.0f - 0x1p-20f, kBf16Hi = 1.0f + 0x1p-20f;   // errors < 2^-21.7
+constexpr float kSiluLo = 1.0f - 0x1p-19f, kSiluHi = 1.0f + 0x1p-19f;   // errors <= 2^-20.6
 constexpr float kE4m3Lo = 1.0f - 0x1p-21f, kE4m3Hi = 1.0f + 0x1p-21f;   // errors <= 2^-22
+constexpr float kTiny = 0x1p-100f;  // below this fp32 products may lose relative precision
 
-// Either bf16 half nonzero with |v| < 2^-100: fp32 products there may have
-// lost relative precision, so the bracket is not trusted.
-__device__ __forceinline__ bool bf2_tiny(uint32_t h) {
-  const uint32_t e = h & 0x7F807F80u;
-  return __vcmpltu2(__vsub2(e, 0x00800080u), 0x0D000D00u) != 0u;
+// Two fp32 values -> bf16x2 word (element 0 in the low half), nearest even.
+__device__ __forceinline__ uint32_t bf2_rn(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Hardware approximations with error bounds measured exhaustively (every
+// fp32 input of the ranges used, against fp64): ex2.approx.ftz <= 2^-22.7
+// relative on [-126, 128); rcp.approx.ftz <= 2^-23.3 relative.
+__device__ __forceinline__ float ex2_approx(float a) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(a));
+  return r;
+}
+__device__ __forceinline__ float rcp_approx(float s) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+  return r;
+}
+
+// e^x for |x| <= 87 as 2^(x log2 e) with the exponent split exactly
+// (Cody & Waite argument splitting): a = fl(x * L2E) plus the exact FMA
+// residual of that product and x times the error of L2E itself; then
+// 2^a * (1 + lo ln 2).  Relative error <= 2^-22.2 (measured exhaustively
+// over every fp32 x in [-87, 87]).
+__device__ __forceinline__ float exp_fast(float x) {
+  const float L2E = 1.44269502f;           // fl32(log2 e)
+  const float L2E_LO = 1.925963e-8f;       // log2 e - L2E
+  const float a = __fmul_rn(x, L2E);
+  const float lo = __fmaf_rn(x, L2E_LO, __fmaf_rn(x, L2E, -a));
+  const float e = ex2_approx(a);
+  return __fmaf_rn(e, __fmul_rn(lo, 0.693147182f), e);
 }
 
 // The rare exact paths, kept out of line: inlined into every unrolled element
 // position they would overflow the instruction cache.
-__device__ __noinline__ uint32_t rms_pair_f64(uint32_t xw, double r) {
+// r = 1 / sqrt(mean(x^2) + eps) in fp64 from the fp64 row sum of squares.
+__device__ __forceinline__ double rms_inv_f64(double ss, int64_t L, float eps) {
+  return 1.0 / sqrt(ss / static_cast<double>(L) + static_cast<double>(eps));
+}
+
+__device__ __noinline__ uint32_t rms_pair_f64(uint32_t xw, double ss, int64_t L, float eps) {
+  const double r = rms_inv_f64(ss, L, eps);
   const uint32_t lo = f64_to_bf16_bits_rn(static_cast<double>(bf16_bits_to_f32(xw & 0xFFFFu)) * r);
   const uint32_t hi = f64_to_bf16_bits_rn(static_cast<double>(bf16_bits_to_f32(xw >> 16)) * r);
   return lo | (hi << 16);
@@ -138,39 +173,58 @@ __device__ __noinline__ uint32_t silu_pair_f64(uint32_t gw, uint32_t uw) {
   return out;
 }
 
-// RMSNorm pair: n = bf16(x * r), y = bf16(n * w).  Fast path: p = fl(x * fl(r)),
-// relative error <= 2^-23 (two roundings); bracket +-2^-20.  n * w is one
-// exactly rounded bf16 multiply (the product of two 8-bit significands is
-// exact before its single rounding).
-__device__ __forceinline__ uint32_t rms_pair(uint32_t xw, uint32_t ww, uint64_t r2, double r) {
-  const uint64_t p = mul2(bf2_to_f2(xw), r2);
-  const uint32_t nlo = f2_to_bf2_rn(mul2(p, pk2(kBf16Lo, kBf16Lo)));
-  const uint32_t nhi = f2_to_bf2_rn(mul2(p, pk2(kBf16Hi, kBf16Hi)));
-  const uint32_t n = (nlo == nhi && !bf2_tiny(nlo)) ? nlo : rms_pair_f64(xw, r);
-  const __nv_bfloat162 y = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&n),
-                                   *reinterpret_cast<const __nv_bfloat162*>(&ww));
-  return *reinterpret_cast<const uint32_t*>(&y);
-}
-
-// SiLU*mul pair: y = bf16(silu(g) * u), silu(g) = g / (1 + e^-g) evaluated
-// as g * fl(1/fl(1 + e)) * u.  Error of the fp32 value: expf <= 2 ulp
-// (2^-22 relative), then four IEEE roundings: <= 2^-21; bracket +-2^-20.
-// Gates below -85 make e^-g overflow fp32: always the exact path.
-__device__ __forceinline__ uint32_t silu_pair(uint32_t gw, uint32_t uw) {
-  const float g0 = __uint_as_float(gw << 16), g1 = __uint_as_float(gw & 0xFFFF0000u);
-  const uint64_t d = add2(pk2(expf(-g0), expf(-g1)), pk2(1.0f, 1.0f));
-  float d0, d1;
-  up2(d, d0, d1);
-  const uint64_t sl = mul2(pk2(g0, g1), pk2(__frcp_rn(d0), __frcp_rn(d1)));
-  const uint64_t p = mul2(sl, bf2_to_f2(uw));
-  const uint32_t lo = f2_to_bf2_rn(mul2(p, pk2(kBf16Lo, kBf16Lo)));
-  const uint32_t hi = f2_to_bf2_rn(mul2(p, pk2(kBf16Hi, kBf16Hi)));
-  if (lo != hi || bf2_tiny(lo) || fminf(g0, g1) < -85.0f) return silu_pair_f64(gw, uw);
+// RMSNorm pair, fast path: n = bf16(x * r) from p = fl(x * r32) with r32 the
+// fp32 rsqrt (relative error < 2^-21.7 in all), bracket +-2^-20.  `unsafe` is set when the
+// bracket does not decide the rounding or |p| is tiny; the caller then
+// recomputes the pair exactly (rms_pair_f64).
+__device__ __forceinline__ uint32_t rms_n_fast(uint32_t xw, float r32, bool& unsafe) {
+  const float p0 = __fmul_rn(__uint_as_float(xw << 16), r32);
+  const float p1 = __fmul_rn(__uint_as_float(xw & 0xFFFF0000u), r32);
+  const uint32_t lo = bf2_rn(__fmul_rn(p0, kBf16Lo), __fmul_rn(p1, kBf16Lo));
+  const uint32_t hi = bf2_rn(__fmul_rn(p0, kBf16Hi), __fmul_rn(p1, kBf16Hi));
+  unsafe = (lo != hi) || fminf(fabsf(p0), fabsf(p1)) < kTiny;
   return lo;
 }
 
+// y = bf16(n * w): one exactly rounded bf16 multiply per half (the product of
+// two 8-bit significands is exact before its single rounding).
+__device__ __forceinline__ uint32_t bf2_mul(uint32_t n, uint32_t w) {
+  const __nv_bfloat162 y = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&n),
+                                   *reinterpret_cast<const __nv_bfloat162*>(&w));
+  return *reinterpret_cast<const uint32_t*>(&y);
+}
+
+// SiLU*mul element, fast: silu(g) * u = g * (1 / (1 + e^-g)) * u with
+// exp_fast (<= 2^-22.2), one rounding of 1 + e, rcp_approx (<= 2^-23.3) and
+// two multiplications: relative error <= 2^-20.6.
+__device__ __forceinline__ float silu_mul_fast(float g, float u) {
+  const float d = __fadd_rn(1.0f, exp_fast(-g));
+  return __fmul_rn(__fmul_rn(g, rcp_approx(d)), u);
+}
+
+// SiLU*mul pair: bracket +-2^-19; gates below -85 (e^-g beyond the fast
+// exp's range) and tiny results take the exact path.
+__device__ __forceinline__ uint32_t silu_pair_fast(uint32_t gw, uint32_t uw, bool& unsafe) {
+  const float g0 = __uint_as_float(gw << 16), g1 = __uint_as_float(gw & 0xFFFF0000u);
+  const float p0 = silu_mul_fast(g0, __uint_as_float(uw << 16));
+  const float p1 = silu_mul_fast(g1, __uint_as_float(uw & 0xFFFF0000u));
+  const uint32_t lo = bf2_rn(__fmul_rn(p0, kSiluLo), __fmul_rn(p1, kSiluLo));
+  const uint32_t hi = bf2_rn(__fmul_rn(p0, kSiluHi), __fmul_rn(p1, kSiluHi));
+  unsafe = (lo != hi) || fminf(fabsf(p0), fabsf(p1)) < kTiny || fminf(g0, g1) < -85.0f;
+  return lo;
+}
+
+// Scale of a group: fl32(max(amax, 1e-10) / 448), UE8M0: rounded up to a
+// power of two.  The quotient is q0 = a * fl(1/448) corrected once by its
+// exact FMA residual (Markstein's correction step); amax is a bf16 value, and
+// the GPU tests check this against IEEE division for every positive bf16 amax.
+constexpr float kInv448 = 1.0f / 448.0f;
+
 __device__ __forceinline__ float group_scale(float amax, int ue8m0) {
-  float s = __fdiv_rn(fmaxf(amax, 1e-10f), 448.0f);
+  const float a = fmaxf(amax, 1e-10f);
+  const float q0 = __fmul_rn(a, kInv448);
+  const float r = __fmaf_rn(-448.0f, q0, a);
+  float s = __fmaf_rn(r, kInv448, q0);
   if (ue8m0) {
     uint32_t u = __float_as_uint(s);          // s >= 2.2e-13: a positive normal
     if (u & 0x007FFFFFu) u = (u & 0xFF800000u) + 0x00800000u;
@@ -191,30 +245,33 @@ __device__ __noinline__ uint2 quantize_chunk_ieee(const uint4 y, float s) {
   return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
-// 8 bf16 values (one chunk) -> 8 e4m3 codes of fl32(y / s).  Fast path:
-// t = y * fl(1/s) is within 1.5 * 2^-23 of fl32(y/s); bracket +-2^-21.
-// `rcp` = __frcp_rn(s).
-__device__ __forceinline__ uint2 quantize_chunk(const uint4& y, float s, float rcp) {
+// 8 bf16 values (one chunk) -> 8 e4m3 codes of fl32(y / s), fast path:
+// t = y * rcp with rcp within 2^-23.3 of 1/s is within 2^-22 of fl32(y/s);
+// bracket +-2^-21.  `unsafe` asks the caller for quantize_chunk_ieee.
+__device__ __forceinline__ uint2 quantize_chunk_fast(const uint4& y, float rcp, bool& unsafe) {
   const uint32_t w[4] = {y.x, y.y, y.z, y.w};
-  const uint64_t r2 = pk2(rcp, rcp);
   uint32_t c[4];
   bool slow = false;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint64_t t = mul2(bf2_to_f2(w[j]), r2);
-    c[j] = f2_to_e4m3x2(mul2(t, pk2(kE4m3Lo, kE4m3Lo)));
-    slow |= c[j] != f2_to_e4m3x2(mul2(t, pk2(kE4m3Hi, kE4m3Hi)));
+    const float t0 = __fmul_rn(__uint_as_float(w[j] << 16), rcp);
+    const float t1 = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), rcp);
+    c[j] = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
+        make_float2(__fmul_rn(t0, kE4m3Lo), __fmul_rn(t1, kE4m3Lo)), __NV_SATFINITE, __NV_E4M3));
+    const uint32_t chi = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
+        make_float2(__fmul_rn(t0, kE4m3Hi), __fmul_rn(t1, kE4m3Hi)), __NV_SATFINITE, __NV_E4M3));
+    slow |= c[j] != chi;
   }
-  if (slow) return quantize_chunk_ieee(y, s);
+  unsafe = slow;
   return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
 __device__ __forceinline__ float chunk_amax(const uint4& y) {
-  // |bf16| max on the bit patterns (sign cleared; magnitudes order as
-  // integers), two halves per SIMD max.
-  uint32_t m = __vmaxu2(y.x & 0x7FFF7FFFu, y.y & 0x7FFF7FFFu);
-  m = __vmaxu2(m, __vmaxu2(y.z & 0x7FFF7FFFu, y.w & 0x7FFF7FFFu));
-  return bf16_bits_to_f32(max(m & 0xFFFFu, m >> 16));
+  // max |y| of 8 bf16 values with packed bf16 max (|.| = sign bits cleared)
+  const uint32_t w[4] = {y.x & 0x7FFF7FFFu, y.y & 0x7FFF7FFFu, y.z & 0x7FFF7FFFu, y.w & 0x7FFF7FFFu};
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(w);
+  const __nv_bfloat162 m = __hmax2(__hmax2(h[0], h[1]), __hmax2(h[2], h[3]));
+  return fmaxf(__low2float(m), __high2float(m));
 }
 
 __device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
@@ -269,16 +326,22 @@ template <int OP, bool PER_TOKEN, int CH, typename Src, typename Release>
 __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, const Src& src,
                                             int tid, int T, int bar_id, double* red_d,
                                             float* red_f, Release release) {
+  static_assert(CH * 4 <= 32, "one mask bit per bf16 pair");
   const int64_t nchunks = p.L >> 3;
   uint4 y[CH];
   bool valid[CH];
 #pragma unroll
   for (int i = 0; i < CH; ++i) valid[i] = (tid + static_cast<int64_t>(i) * T) < nchunks;
+  auto off = [&](int i) { return (tid + static_cast<int64_t>(i) * T) * 8; };
 
+  // Hot loops compute every value on the fast path and only flag the rare
+  // pairs / chunks whose rounding the fast path cannot decide; the exact
+  // recomputation of those runs afterwards, outside the hot loops.
+  uint32_t fix = 0;  // bit 4i + j: pair j of chunk i needs the exact path
   if constexpr (OP == OP_PLAIN) {
 #pragma unroll
     for (int i = 0; i < CH; ++i)
-      if (valid[i]) y[i] = src.ld((tid + static_cast<int64_t>(i) * T) * 8);
+      if (valid[i]) y[i] = src.ld(off(i));
     release();
   } else if constexpr (OP == OP_SILU) {
     // gate and up chunks are read in batches of SB chunks to bound registers.
@@ -289,9 +352,8 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
 #pragma unroll
       for (int i = 0; i < SB; ++i) {
         if (valid[i0 + i]) {
-          const int64_t off = (tid + static_cast<int64_t>(i0 + i) * T) * 8;
-          g[i] = src.ld(off);
-          u[i] = src.ld(p.L + off);
+          g[i] = src.ld(off(i0 + i));
+          u[i] = src.ld(p.L + off(i0 + i));
         }
       }
 #pragma unroll
@@ -301,8 +363,26 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
           const uint32_t uw[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
           uint32_t o[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) o[j] = silu_pair(gw[j], uw[j]);
+          for (int j = 0; j < 4; ++j) {
+            bool bad;
+            o[j] = silu_pair_fast(gw[j], uw[j], bad);
+            fix |= static_cast<uint32_t>(bad) << (4 * (i0 + i) + j);
+          }
           y[i0 + i] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+    if (fix) {  // rare: re-read the flagged chunks and recompute their pairs exactly
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        if ((fix >> (4 * i)) & 0xFu) {
+          const uint4 g = src.ld(off(i)), u = src.ld(p.L + off(i));
+          uint32_t* yw = reinterpret_cast<uint32_t*>(&y[i]);
+          const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+          const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if ((fix >> (4 * i + j)) & 1u) yw[j] = silu_pair_f64(gw[j], uw[j]);
         }
       }
     }
@@ -311,7 +391,7 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
     uint4 xv[CH];
 #pragma unroll
     for (int i = 0; i < CH; ++i)
-      if (valid[i]) xv[i] = src.ld((tid + static_cast<int64_t>(i) * T) * 8);
+      if (valid[i]) xv[i] = src.ld(off(i));
     release();
     // Sum of squares: squares of bf16 values are exact in fp32; they are
     // accumulated with paired TwoSum (Knuth, TAOCP vol. 2, 4.2.2), a running
@@ -338,23 +418,46 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
     double ss = (static_cast<double>(s0) + static_cast<double>(s1f)) +
                 (static_cast<double>(c0) + static_cast<double>(c1));
     ss = team_reduce(ss, SumOp(), red_d, tid, T, bar_id);
-    const double r = 1.0 / sqrt(ss / static_cast<double>(p.L) + static_cast<double>(p.eps));
-    const uint64_t r2 = pk2(static_cast<float>(r), static_cast<float>(r));
+    // Fast path: r32 = rsqrtf(fl32(mean + eps)): <= 2 ulp + half an ulp from
+    // the conversion, < 2^-21.9 relative; the fp64 r is computed only by the
+    // exact path.
+    const float r32 = rsqrtf(static_cast<float>(ss / static_cast<double>(p.L) + static_cast<double>(p.eps)));
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
       if (valid[i]) {
-        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.w + (tid + static_cast<int64_t>(i) * T) * 8));
         const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.w + off(i)));
         const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
         uint32_t o[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) o[j] = rms_pair(xw[j], ww[j], r2, r);
+        for (int j = 0; j < 4; ++j) {
+          bool bad;
+          o[j] = bf2_mul(rms_n_fast(xw[j], r32, bad), ww[j]);
+          fix |= static_cast<uint32_t>(bad) << (4 * i + j);
+        }
         y[i] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    if (fix) {  // rare: exact bf16(x * r) for the flagged pairs, then y again
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        if ((fix >> (4 * i)) & 0xFu) {
+          const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+          const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.w + off(i)));
+          const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+          uint32_t* yw = reinterpret_cast<uint32_t*>(&y[i]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if ((fix >> (4 * i + j)) & 1u) yw[j] = bf2_mul(rms_pair_f64(xw[j], ss, p.L, p.eps), ww[j]);
+        }
       }
     }
   }
 
+  // Codes are stored as soon as they are made; a flagged chunk is stored
+  // again, from IEEE division, after the loop.
   uint8_t* qr = p.q + row * p.ldq;
+  uint32_t qfix = 0;  // bit i: chunk i needs IEEE division
   if constexpr (PER_TOKEN) {
     float amax = 0.0f;
 #pragma unroll
@@ -362,29 +465,42 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
       if (valid[i]) amax = fmaxf(amax, chunk_amax(y[i]));
     amax = team_reduce(amax, MaxOp(), red_f, tid, T, bar_id);
     const float s = group_scale(amax, p.ue8m0);
-    const float rcp = __frcp_rn(s);
+    const float rcp = rcp_approx(s);
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
       if (valid[i]) {
-        const int64_t c = tid + static_cast<int64_t>(i) * T;
-        *reinterpret_cast<uint2*>(qr + c * 8) = quantize_chunk(y[i], s, rcp);
+        bool bad;
+        *reinterpret_cast<uint2*>(qr + off(i)) = quantize_chunk_fast(y[i], rcp, bad);
+        qfix |= static_cast<uint32_t>(bad) << i;
       }
     }
     if (tid == 0) p.s[row * p.s_sm] = s;
+    if (qfix) {
+#pragma unroll
+      for (int i = 0; i < CH; ++i)
+        if ((qfix >> i) & 1u) *reinterpret_cast<uint2*>(qr + off(i)) = quantize_chunk_ieee(y[i], s);
+    }
   } else {
     // 128-wide groups: the 16 threads tid & ~15 .. +15 own one group per i
     // (T is a multiple of 32 and L of 128, so whole half-warps are valid or not).
+    float sc[CH];
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
       float a = valid[i] ? chunk_amax(y[i]) : 0.0f;
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+      sc[i] = group_scale(a, p.ue8m0);
       if (valid[i]) {
-        const int64_t c = tid + static_cast<int64_t>(i) * T;
-        const float s = group_scale(a, p.ue8m0);
-        *reinterpret_cast<uint2*>(qr + c * 8) = quantize_chunk(y[i], s, __frcp_rn(s));
-        if ((tid & 15) == 0) p.s[row * p.s_sm + (c >> 4) * p.s_sg] = s;
+        bool bad;
+        *reinterpret_cast<uint2*>(qr + off(i)) = quantize_chunk_fast(y[i], rcp_approx(sc[i]), bad);
+        qfix |= static_cast<uint32_t>(bad) << i;
+        if ((tid & 15) == 0) p.s[row * p.s_sm + (off(i) >> 7) * p.s_sg] = sc[i];
       }
+    }
+    if (qfix) {
+#pragma unroll
+      for (int i = 0; i < CH; ++i)
+        if ((qfix >> i) & 1u) *reinterpret_cast<uint2*>(qr + off(i)) = quantize_chunk_ieee(y[i], sc[i]);
     }
   }
 }
@@ -402,21 +518,29 @@ __global__ void __launch_bounds__(kMaxThreads, (CH <= 4 ? 2 : 1)) quant_rows_ker
 
 // Ring kernel: persistent CTAs; warp 0 (one lane) streams whole input rows
 // into a ring of NBUF shared-memory buffers with cp.async.bulk (completion on
-// the slot's mbarrier), so HBM reads stay in flight while the T compute
-// threads quantize earlier rows from shared memory.  Every wait is bounded; a
-// wait that gives up records FP8Q_ERR_TIMEOUT, the compute team leaves
-// together (vote on a named barrier) and the producer lets its copies land.
-constexpr int kRingMaxBuf = 8;
+// the slot's mbarrier), while NT teams of T compute threads each quantize a
+// different row from shared memory (team t takes the CTA's rows i = t, t+NT,
+// ...; NBUF is a multiple of NT, so a slot always serves the same team).  HBM
+// reads stay in flight independently of the compute.  Every wait is bounded; a
+// wait that gives up records FP8Q_ERR_TIMEOUT, the team leaves together (vote
+// on its named barrier) and the producer lets its copies land.
+constexpr int kRingMaxBuf = 16;
+
+// CTA size cap of the ring kernel (it sets the register budget per thread):
+// SiLU needs more registers than the other ops, 8 chunks per thread more still.
+__host__ __device__ constexpr int ring_max_threads(int op, int ch) {
+  return ch == 8 ? 512 : (op == OP_SILU ? 800 : 1024);
+}
 
 template <int OP, bool PER_TOKEN, int CH>
-__global__ void __launch_bounds__(kMaxThreads + 32, 1)
-    quant_ring_kernel(const QuantParams p, int nbuf, int row_stride_bytes, int* status) {
+__global__ void __launch_bounds__(ring_max_threads(OP, CH), 1)
+    quant_ring_kernel(const QuantParams p, int nbuf, int nteams, int T, int row_stride_bytes,
+                      int* status) {
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ uint64_t full[kRingMaxBuf], empty[kRingMaxBuf];
-  __shared__ double red_d[32];
-  __shared__ float red_f[32];
+  __shared__ double red_d[8][32];
+  __shared__ float red_f[8][32];
   __shared__ volatile int abort_flag;
-  const int T = blockDim.x - 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t copy_bytes = static_cast<uint32_t>((OP == OP_SILU ? 4 : 2) * p.L);
 
@@ -452,14 +576,17 @@ __global__ void __launch_bounds__(kMaxThreads + 32, 1)
     return;
   }
 
-  const int tid = threadIdx.x - 32;
-  int i = 0;
-  for (int64_t row = blockIdx.x; row < p.M; row += gridDim.x, ++i) {
+  const int team = (threadIdx.x - 32) / T;
+  const int tid = (threadIdx.x - 32) - team * T;
+  const int bar = 1 + team;
+  int i = team;
+  for (int64_t row = blockIdx.x + static_cast<int64_t>(team) * gridDim.x; row < p.M;
+       row += static_cast<int64_t>(nteams) * gridDim.x, i += nteams) {
     const int slot = i % nbuf;
     const bool ok = sm100::mbar_wait(&full[slot], (i / nbuf) & 1, &abort_flag, status);
-    if (sm100::team_any(!ok, 1, T)) break;
+    if (sm100::team_any(!ok, bar, T)) break;
     const uint16_t* src = reinterpret_cast<const uint16_t*>(ring + static_cast<size_t>(slot) * row_stride_bytes);
-    process_row<OP, PER_TOKEN, CH>(p, row, SmemRow{src}, tid, T, 1, red_d, red_f, [&] {
+    process_row<OP, PER_TOKEN, CH>(p, row, SmemRow{src}, tid, T, bar, red_d[team], red_f[team], [&] {
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&empty[slot]);
     });
@@ -474,19 +601,32 @@ inline int threads_for(int64_t nchunks, int ch) {
   return static_cast<int>(t < 32 ? 32 : t);
 }
 
-constexpr int kRingSmemTarget = 96 * 1024;    // ring bytes aimed at per CTA
-constexpr int kRingSmemMax = 200 * 1024;      // larger rows use the register kernel
+constexpr int kRingSmemMax = 200 * 1024;   // ring bytes per CTA (one CTA per SM)
+
+// Ring geometry: as many teams as fit the CTA size cap (at most 8), and
+// the deepest ring (a multiple of the team count, >= 2 slots per team) that
+// fits the shared memory.  Returns false when even one team with two slots
+// does not fit.
+bool ring_geometry(int64_t row_bytes, int T, int max_threads, int* nteams, int* nbuf, int* stride) {
+  *stride = static_cast<int>(((row_bytes + 127) / 128) * 128);
+  int nt = (max_threads - 32) / T;
+  nt = nt > 8 ? 8 : nt;
+  while (nt >= 1 && 2LL * nt * *stride > kRingSmemMax) --nt;
+  if (nt < 1) return false;
+  int per = static_cast<int>(kRingSmemMax / (static_cast<int64_t>(nt) * *stride));
+  if (per * nt > kRingMaxBuf) per = kRingMaxBuf / nt;
+  if (per < 2) return false;
+  *nteams = nt;
+  *nbuf = per * nt;
+  return true;
+}
 
 template <int OP, bool PER_TOKEN, int CH>
-fp8q_status launch_ring(const QuantParams& p, int T, cudaStream_t stream) {
-  const int64_t row_bytes = (OP == OP_SILU ? 4 : 2) * p.L;
-  const int stride = static_cast<int>(((row_bytes + 127) / 128) * 128);
-  int nbuf = static_cast<int>(kRingSmemTarget / stride);
-  nbuf = nbuf < 2 ? 2 : (nbuf > kRingMaxBuf ? kRingMaxBuf : nbuf);
+fp8q_status launch_ring(const QuantParams& p, int T, int nteams, int nbuf, int stride,
+                        cudaStream_t stream) {
   const int smem = nbuf * stride;
   auto kern = quant_ring_kernel<OP, PER_TOKEN, CH>;
   static int attr_done[64] = {0};
-  static int occ_cache[64][2] = {{0}};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
@@ -495,18 +635,10 @@ fp8q_status launch_ring(const QuantParams& p, int T, cudaStream_t stream) {
       return FP8Q_ERR_CUDA;
     attr_done[dev] = 1;
   }
-  int occ = 0;
-  if (occ_cache[dev][0] == (T << 20 | smem >> 7) + 1) {
-    occ = occ_cache[dev][1];
-  } else {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, T + 32, smem) != cudaSuccess || occ < 1)
-      occ = 1;
-    occ_cache[dev][0] = (T << 20 | smem >> 7) + 1;
-    occ_cache[dev][1] = occ;
-  }
-  int64_t grid = static_cast<int64_t>(num_sms()) * occ;
+  int64_t grid = num_sms();
   if (grid > p.M) grid = p.M;
-  kern<<<static_cast<unsigned>(grid), T + 32, smem, stream>>>(p, nbuf, stride, device_status_ptr());
+  kern<<<static_cast<unsigned>(grid), 32 + nteams * T, smem, stream>>>(p, nbuf, nteams, T, stride,
+                                                                       device_status_ptr());
   return launch_status();
 }
 
@@ -519,11 +651,15 @@ fp8q_status launch_quant(const QuantParams& p, cudaStream_t stream) {
   const int ch = nchunks > 4 * kMaxThreads ? 8 : 4;
   const int T = threads_for(nchunks, ch);
   if (T > kMaxThreads) return FP8Q_ERR_UNSUPPORTED;
-  // Long rows (8 chunks per thread, few rows per SM) stream through the
-  // shared-memory ring; shorter rows run many CTAs per SM on registers alone.
+  // Long rows (8 chunks per thread) stream through the shared-memory ring;
+  // shorter rows run many CTAs per SM on registers alone.
   const int64_t row_bytes = (OP == OP_SILU ? 4 : 2) * p.L;
-  if (ch == 8 && 2 * ((row_bytes + 127) / 128) * 128 <= kRingSmemMax)
-    return per_token ? launch_ring<OP, true, 8>(p, T, stream) : launch_ring<OP, false, 8>(p, T, stream);
+  int nteams = 0, nbuf = 0, stride = 0;
+  // (Measured: for rows of <= 2048 chunks the register kernel, with many
+  // CTAs per SM, is faster than the ring.)
+  if (ch == 8 && ring_geometry(row_bytes, T, ring_max_threads(OP, ch), &nteams, &nbuf, &stride))
+    return per_token ? launch_ring<OP, true, 8>(p, T, nteams, nbuf, stride, stream)
+                     : launch_ring<OP, false, 8>(p, T, nteams, nbuf, stride, stream);
   const int64_t grid = p.M < (1LL << 30) ? p.M : (1LL << 30);
   const dim3 g(static_cast<unsigned>(grid)), b(T);
   if (ch == 8) {

@@ -164,3 +164,25 @@ def test_quant_deterministic():
         b = fq.fp8q_rmsnorm_quant(x, w, 1e-6, 128)
         assert torch.equal(a[0].view(torch.uint8), b[0].view(torch.uint8))
         assert torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("ue8m0", [False, True])
+def test_group_scale_for_every_bf16_amax(ue8m0):
+    # Every positive finite bf16 value is the amax of one 128-group (plus one
+    # all-zero group): the kernel's scale must equal the oracle's IEEE division
+    # fl32(max(amax, 1e-10)/448) (and its UE8M0 rounding) for every one of them,
+    # and the codes of the group's other, smaller random elements must match.
+    amax_bits = np.arange(1, 0x7F80, dtype=np.int64)            # 1 .. largest finite
+    G = amax_bits.size + 1                                       # + an all-zero group
+    g = np.random.default_rng(99)
+    groups = np.zeros((G, 128), np.int64)
+    groups[:-1] = g.integers(0, amax_bits[:, None], size=(G - 1, 128))  # smaller magnitudes
+    groups[:-1, :] |= g.integers(0, 2, size=(G - 1, 128)) << 15        # random signs
+    pos = g.integers(0, 128, size=G - 1)
+    groups[np.arange(G - 1), pos] = amax_bits | (g.integers(0, 2, size=G - 1) << 15)
+    x = groups.astype(np.uint16).reshape(G // 8, 8 * 128)
+    q_ref, s_ref = oracle.group_quant(x, 128, ue8m0)
+    q, s = fq.fp8q_group_quant(to_dev_bf16(x), 128, ue8m0)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(s.cpu().numpy(), s_ref)
+    np.testing.assert_array_equal(codes_np(q), q_ref)
