@@ -440,6 +440,9 @@ def run_sweep(args):
         ts = []
         for _ in range(args.reps):
             flush.zero_()
+            # keep the GPU busy while the host enqueues fn, so that host-side
+            # launch overhead does not leak into the device time of fn
+            torch.cuda._sleep(200_000)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)

@@ -50,7 +50,10 @@ constexpr int kSmemBudget = 200 * 1024;
 
 struct GemmArgs {
   int rows_a, rows_b, K;              // MMA-A rows (TMEM lanes), MMA-B rows (columns)
-  int kblocks, tiles_a, tiles_b, split, kb_per_split, units;
+  int kblocks, tiles_a, tiles_b, split, kb_per_split, units;  // classic: tiles x split units
+  int streamk;                        // 1: stream-K ranges instead of units
+  int seg_len, total_iters;           // stream-K: K-block iterations per CTA, tiles x kblocks
+  int max_contrib;                    // partial slots per tile in the workspace
   int M, N;                           // logical output shape
   const float* sa;                    // activation scales: sa[m*sa_sm + kb*sa_skb]
   int64_t sa_sm, sa_skb;
@@ -96,6 +99,51 @@ __device__ __forceinline__ void unit_coords(const GemmArgs& p, int u, int& ta, i
   kb0 = s * p.kb_per_split;
   kb1 = min(p.kblocks, kb0 + p.kb_per_split);
 }
+
+// One piece of work of a CTA: K blocks [kb0, kb1) of tile (ta, tb), written
+// to partial slot `slot` of the tile's `ncontrib` contributors (1: the piece
+// is the whole tile and goes straight to y).
+struct Seg {
+  int ta, tb, kb0, kb1, slot, ncontrib;
+};
+
+// The CTA's pieces in order.  Classic: units blockIdx.x, + gridDim.x, ...
+// (tile-major, `split` equal K ranges per tile).  Stream-K: one contiguous
+// range of seg_len (tile, K block) iterations per CTA, so every CTA streams
+// the same number of K blocks; a tile cut by range boundaries is summed from
+// the partials of the CTAs that cover it, in CTA order.
+struct SegIter {
+  int cur, end;
+  __device__ explicit SegIter(const GemmArgs& p) {
+    if (p.streamk) {
+      cur = blockIdx.x * p.seg_len;
+      end = min(p.total_iters, cur + p.seg_len);
+    } else {
+      cur = blockIdx.x;
+      end = p.units;
+    }
+  }
+  __device__ bool next(const GemmArgs& p, Seg& g) {
+    if (cur >= end) return false;
+    if (!p.streamk) {
+      unit_coords(p, cur, g.ta, g.tb, g.slot, g.kb0, g.kb1);
+      g.ncontrib = p.split;
+      cur += gridDim.x;
+      return true;
+    }
+    const int tile = cur / p.kblocks;
+    g.kb0 = cur - tile * p.kblocks;
+    g.kb1 = min(p.kblocks, g.kb0 + (end - cur));
+    g.ta = tile % p.tiles_a;
+    g.tb = tile / p.tiles_a;
+    const int first = static_cast<int>((static_cast<int64_t>(tile) * p.kblocks) / p.seg_len);
+    const int last = static_cast<int>((static_cast<int64_t>(tile + 1) * p.kblocks - 1) / p.seg_len);
+    g.ncontrib = last - first + 1;
+    g.slot = static_cast<int>(blockIdx.x) - first;
+    cur += g.kb1 - g.kb0;
+    return true;
+  }
+};
 
 // acc += (r0, r1) * sc: one paired fp32 FMA (sm_100 .f32x2) on a 64-bit
 // accumulator pair; r0, r1 are adjacent registers of a tcgen05.ld.
@@ -175,16 +223,16 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
     if (lane == 0) {
       int it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-        int ta, tb, s, kb0, kb1;
-        unit_coords(p, u, ta, tb, s, kb0, kb1);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+      SegIter si(p);
+      Seg g;
+      while (ok && si.next(p, g)) {
+        for (int kb = g.kb0; kb < g.kb1; ++kb, ++it) {
           const int st = it % S;
           const uint32_t ph = (it / S) & 1;
           if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
-          tma_load_2d(sA + st * A_BYTES, &tmA, &full[st], kb * BK, ta * BM);
-          tma_load_2d(sB + st * C::B_BYTES, &tmB, &full[st], kb * BK, tb * BN);
+          tma_load_2d(sA + st * A_BYTES, &tmA, &full[st], kb * BK, g.ta * BM);
+          tma_load_2d(sB + st * C::B_BYTES, &tmB, &full[st], kb * BK, g.tb * BN);
         }
       }
       if (!ok) {
@@ -200,9 +248,10 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
       constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
       int it = 0, t = 0, pc = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-        int ta, tb, s, kb0, kb1;
-        unit_coords(p, u, ta, tb, s, kb0, kb1);
+      SegIter si(p);
+      Seg g;
+      while (ok && si.next(p, g)) {
+        const int kb0 = g.kb0, kb1 = g.kb1;
         uint32_t d = tmem_base;
         int buf = 0;
         if (!BW) {
@@ -257,14 +306,15 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
     int t = 0, pc = 0;
     bool ok = true;
 
-    for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
-      int ta, tb, s, kb0, kb1;
-      unit_coords(p, u, ta, tb, s, kb0, kb1);
+    SegIter si(p);
+    Seg g;
+    while (ok && si.next(p, g)) {
+      const int ta = g.ta, tb = g.tb, kb0 = g.kb0, kb1 = g.kb1;
       const int a_idx = ta * BM + row;                         // m (no swap) or n (swap)
       const int b_base = tb * BN;                              // first column's n or m
       const bool a_valid = a_idx < (SWAP ? p.N : p.M);
       const int tile_id = tb * p.tiles_a + ta;
-      float* ws_tile = p.ws + (static_cast<int64_t>(tile_id) * p.split) * (BN * BM);
+      float* ws_tile = p.ws + (static_cast<int64_t>(tile_id) * p.max_contrib) * (BN * BM);
 
       // Store one chunk of CHUNK final values v[] for columns col..col+CHUNK-1.
       auto emit = [&](int col, const float* v) {
@@ -295,10 +345,22 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
           }
         }
       };
-      auto stash = [&](int col, const float* v) {    // fp32 partial of split s
-        float* w = ws_tile + static_cast<int64_t>(s) * (BN * BM);
+      // Partial layout inside a slot.  VEC: [col/4][row][4] fp32, each lane
+      // moving 16 bytes, a warp's access 512 contiguous bytes.  Otherwise
+      // (the 16-warp variant, whose register budget is tight): [col][row],
+      // 4 bytes a lane, 128 contiguous bytes a warp.
+      constexpr bool VEC = C::EPI_WARPS < 16;
+      auto stash = [&](int col, const float* v) {    // fp32 partial of this piece
+        float* w = ws_tile + static_cast<int64_t>(g.slot) * (BN * BM);
+        if (VEC) {
 #pragma unroll
-        for (int i = 0; i < C::CHUNK; ++i) w[(col + i) * BM + row] = v[i];
+          for (int i = 0; i < C::CHUNK; i += 4)
+            __stcg(reinterpret_cast<float4*>(w) + ((col + i) >> 2) * BM + row,
+                   make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < C::CHUNK; ++i) __stcg(w + (col + i) * BM + row, v[i]);
+        }
       };
       auto finish_split = [&]() {                    // last arrival sums the partials in order
         __threadfence();
@@ -306,17 +368,47 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
         int old = 0;
         if (lane == 0) old = atomicAdd(&p.counters[tile_id * C::EPI_WARPS + e], 1);
         old = __shfl_sync(0xFFFFFFFFu, old, 0);
-        if (old != p.split - 1) return;
+        if (old != g.ncontrib - 1) return;
         if (lane == 0) p.counters[tile_id * C::EPI_WARPS + e] = 0;
         __threadfence();
+        // Slots are added in slot order (VEC: two slots' loads in flight at once).
+        constexpr int Q = C::CHUNK / 4;
+        constexpr int64_t SLOT = BN * BM;
         for (int c = col0; c < col0 + C::CPT; c += C::CHUNK) {
           float v[C::CHUNK];
 #pragma unroll
           for (int i = 0; i < C::CHUNK; ++i) v[i] = 0.0f;
-          for (int ss = 0; ss < p.split; ++ss) {
-            const float* w = ws_tile + static_cast<int64_t>(ss) * (BN * BM);
+          if (VEC) {
+            const float4* wc = reinterpret_cast<const float4*>(ws_tile) + (c >> 2) * BM + row;
+            int ss = 0;
+            for (; ss + 1 < g.ncontrib; ss += 2) {
+              float4 x0[Q], x1[Q];
 #pragma unroll
-            for (int i = 0; i < C::CHUNK; ++i) v[i] += __ldcg(w + (c + i) * BM + row);
+              for (int i = 0; i < Q; ++i) x0[i] = __ldcg(wc + ss * (SLOT / 4) + i * BM);
+#pragma unroll
+              for (int i = 0; i < Q; ++i) x1[i] = __ldcg(wc + (ss + 1) * (SLOT / 4) + i * BM);
+#pragma unroll
+              for (int i = 0; i < Q; ++i) {
+                v[4 * i + 0] += x0[i].x; v[4 * i + 1] += x0[i].y; v[4 * i + 2] += x0[i].z; v[4 * i + 3] += x0[i].w;
+              }
+#pragma unroll
+              for (int i = 0; i < Q; ++i) {
+                v[4 * i + 0] += x1[i].x; v[4 * i + 1] += x1[i].y; v[4 * i + 2] += x1[i].z; v[4 * i + 3] += x1[i].w;
+              }
+            }
+            if (ss < g.ncontrib) {
+#pragma unroll
+              for (int i = 0; i < Q; ++i) {
+                const float4 x = __ldcg(wc + ss * (SLOT / 4) + i * BM);
+                v[4 * i + 0] += x.x; v[4 * i + 1] += x.y; v[4 * i + 2] += x.z; v[4 * i + 3] += x.w;
+              }
+            }
+          } else {
+            for (int ss = 0; ss < g.ncontrib; ++ss) {
+              const float* w = ws_tile + ss * SLOT;
+#pragma unroll
+              for (int i = 0; i < C::CHUNK; ++i) v[i] += __ldcg(w + (c + i) * BM + row);
+            }
           }
           emit(c, v);
         }
@@ -355,14 +447,14 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
 #pragma unroll
           for (int i = 0; i < C::CHUNK; ++i)
             v[i] = v[i] * (srow * __shfl_sync(0xFFFFFFFFu, colsc[j], i));
-          if (p.split == 1) emit(c, v);
+          if (g.ncontrib == 1) emit(c, v);
           else stash(c, v);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);
         ++t;
-        if (p.split > 1) finish_split();
+        if (g.ncontrib > 1) finish_split();
       } else {
         // -------- blockwise scales: promote each K-block partial into registers.
         // The scales of K block kb+1 are loaded while block kb is processed, so
@@ -442,10 +534,10 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
           float v[C::CHUNK];
 #pragma unroll
           for (int i = 0; i < C::CHUNK; i += 2) unpair_f32(acc[(c + i) / 2], v[i], v[i + 1]);
-          if (p.split == 1) emit(col0 + c, v);
+          if (g.ncontrib == 1) emit(col0 + c, v);
           else stash(col0 + c, v);
         }
-        if (p.split > 1) finish_split();
+        if (g.ncontrib > 1) finish_split();
       }
     }
   }
@@ -547,7 +639,9 @@ fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
       return FP8Q_ERR_CUDA;
     attr_done[dev] = 1;
   }
-  const int grid = p.units < num_sms() ? p.units : num_sms();
+  int grid;
+  if (p.streamk) grid = (p.total_iters + p.seg_len - 1) / p.seg_len;
+  else grid = p.units < num_sms() ? p.units : num_sms();
   gemm_kernel<BN, SWAP, BW><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, p);
   return launch_status();
 }
@@ -559,7 +653,7 @@ bool g_forced = false;
 fp8q_gemm_variant g_force{0, 1, 128};
 
 bool variant_supported(const fp8q_gemm_variant& v, int blockwise) {
-  if (v.split_k < 1 || v.split_k > 64) return false;
+  if (v.split_k < 0 || v.split_k > 64) return false;   // 0: stream-K
   if (v.swap_ab) return v.block_n == 16 || v.block_n == 32 || v.block_n == 64 || v.block_n == 128;
   if (blockwise) return v.block_n == 128 || v.block_n == 256;
   return v.block_n == 128 || v.block_n == 256;
@@ -570,52 +664,78 @@ int epi_warps(const fp8q_gemm_variant& v, int blockwise) {
   return (blockwise && v.block_n >= 128) ? 8 : 4;
 }
 
-// Split count that spreads tiles over the SMs: the smallest split whose last
-// wave is at least 90% full, capped so that every split keeps >= 2 K blocks
-// and the fp32 partial traffic stays under a quarter of the weight bytes.
-int choose_split(int64_t tiles, int64_t kblocks, int64_t M, int64_t N, int64_t K, int bn,
-                 int sms) {
-  if (tiles >= sms) return 1;
-  int best = 1;
-  double best_eff = 0.0;
-  for (int s = 1; s <= 16; ++s) {
-    if (s > 1 && kblocks / s < 2) break;
-    const double ws_traffic = 2.0 * s * tiles * BM * bn * 4.0;
-    if (s > 1 && ws_traffic > 0.25 * static_cast<double>(N) * static_cast<double>(K)) break;
-    const int64_t units = tiles * s;
-    const int64_t waves = (units + sms - 1) / sms;
-    const double eff = static_cast<double>(units) / static_cast<double>(waves * sms);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best = s;
-    }
-    if (eff >= 0.9) break;
+// Measured variant table: for each (scheme, N, K) the fastest variant per
+// bucket of M, timed on a B200 by tune.py (which writes the included file).
+// A row applies to m_prev < M <= m_max, m_prev being the next smaller m_max
+// of the same (scheme, N, K); M above the largest bucket takes that bucket.
+struct TunedVariant {
+  int blockwise;
+  int64_t m_max, n, k;
+  int swap_ab, split_k, block_n;
+};
+constexpr TunedVariant kTuned[] = {
+#include "fp8q_variant_table.inc"
+    {-1, 0, 0, 0, 0, 0, 0},   // end marker
+};
+
+bool tuned_variant(int64_t M, int64_t N, int64_t K, int blockwise, fp8q_gemm_variant* out) {
+  const TunedVariant* best = nullptr;   // smallest m_max >= M
+  const TunedVariant* top = nullptr;    // largest m_max
+  for (const TunedVariant& t : kTuned) {
+    if (t.blockwise != blockwise || t.n != N || t.k != K) continue;
+    if (t.m_max >= M && (!best || t.m_max < best->m_max)) best = &t;
+    if (!top || t.m_max > top->m_max) top = &t;
   }
-  (void)M;
-  return best;
+  if (!best) best = top;
+  if (!best) return false;
+  out->swap_ab = best->swap_ab;
+  out->split_k = best->split_k;
+  out->block_n = best->block_n;
+  return variant_supported(*out, blockwise);
 }
 
-fp8q_gemm_variant auto_variant(int64_t M, int64_t N, int64_t K, int blockwise) {
+// Shapes outside the table: rules drawn from the same measurements.
+fp8q_gemm_variant heuristic_variant(int64_t M, int64_t N, int64_t K, int blockwise) {
   fp8q_gemm_variant v;
-  if (M <= 64) {
+  if (M <= 128) {
+    // Swap-AB: the weight rows fill the 128-row MMA slot, the tokens its N.
     v.swap_ab = 1;
-    v.block_n = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
-  } else if (M <= 128) {
-    v.swap_ab = 1;
-    v.block_n = 128;
+    v.block_n = M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128));
   } else {
     v.swap_ab = 0;
     v.block_n = 256;
   }
   const int64_t rows_a = v.swap_ab ? N : M, rows_b = v.swap_ab ? M : N;
   const int64_t tiles = ((rows_a + BM - 1) / BM) * ((rows_b + v.block_n - 1) / v.block_n);
-  v.split_k = choose_split(tiles, (K + BK - 1) / BK, M, N, K, v.block_n, num_sms());
+  const int64_t kblocks = (K + BK - 1) / BK;
+  const int64_t sms = num_sms();
+  if (tiles >= sms) {
+    v.split_k = 1;
+  } else if (blockwise && M > 16) {
+    // The per-K-block promotion makes each SM's share of the K loop the
+    // limit: stream-K spreads the K blocks over every SM.
+    v.split_k = 0;
+  } else {
+    // Whole K ranges: as many per tile as fit on the SMs in one wave,
+    // each at least 8 K blocks long.
+    int64_t s = sms / tiles;
+    if (s > kblocks / 8) s = kblocks / 8;
+    v.split_k = static_cast<int>(s < 1 ? 1 : s);
+  }
   return v;
 }
 
-fp8q_gemm_variant pick_variant(int64_t M, int64_t N, int64_t K, int blockwise) {
+fp8q_gemm_variant auto_variant(int64_t M, int64_t N, int64_t K, int blockwise) {
+  fp8q_gemm_variant v;
+  if (tuned_variant(M, N, K, blockwise, &v)) return v;
+  return heuristic_variant(M, N, K, blockwise);
+}
+
+fp8q_gemm_variant pick_variant(int64_t M, int64_t N, int64_t K, int blockwise,
+                               bool* forced = nullptr) {
   {
     std::lock_guard<std::mutex> lock(g_force_mu);
+    if (forced) *forced = g_forced;
     if (g_forced) return g_force;
   }
   return auto_variant(M, N, K, blockwise);
@@ -624,6 +744,7 @@ fp8q_gemm_variant pick_variant(int64_t M, int64_t N, int64_t K, int blockwise) {
 struct Plan {
   fp8q_gemm_variant v;
   int tiles_a, tiles_b, kblocks, split, kb_per_split, units;
+  int streamk, seg_len, total_iters, grid, max_contrib;
   size_t counter_bytes, ws_bytes;
 };
 
@@ -634,15 +755,36 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int blockwise, const fp8q_gemm_v
   pl.tiles_a = static_cast<int>((rows_a + BM - 1) / BM);
   pl.tiles_b = static_cast<int>((rows_b + v.block_n - 1) / v.block_n);
   pl.kblocks = static_cast<int>((K + BK - 1) / BK);
-  int split = v.split_k < pl.kblocks ? v.split_k : pl.kblocks;
-  if (split < 1) split = 1;
-  pl.kb_per_split = (pl.kblocks + split - 1) / split;
-  pl.split = (pl.kblocks + pl.kb_per_split - 1) / pl.kb_per_split;   // every split non-empty
   const int64_t tiles = static_cast<int64_t>(pl.tiles_a) * pl.tiles_b;
-  pl.units = static_cast<int>(tiles * pl.split);
-  if (pl.split > 1) {
+  pl.streamk = 0;
+  pl.seg_len = 0;
+  pl.total_iters = 0;
+  if (v.split_k == 0) {
+    // stream-K: equal K-block ranges over at most one CTA per SM
+    const int64_t total = tiles * pl.kblocks;
+    int64_t grid = num_sms();
+    if (grid > total) grid = total;
+    pl.streamk = 1;
+    pl.total_iters = static_cast<int>(total);
+    pl.seg_len = static_cast<int>((total + grid - 1) / grid);
+    pl.grid = static_cast<int>((total + pl.seg_len - 1) / pl.seg_len);
+    pl.max_contrib = (pl.kblocks + pl.seg_len - 1) / pl.seg_len + 1;
+    if (pl.max_contrib > pl.grid) pl.max_contrib = pl.grid;
+    pl.split = 1;
+    pl.kb_per_split = pl.kblocks;
+    pl.units = 0;
+  } else {
+    int split = v.split_k < pl.kblocks ? v.split_k : pl.kblocks;
+    if (split < 1) split = 1;
+    pl.kb_per_split = (pl.kblocks + split - 1) / split;
+    pl.split = (pl.kblocks + pl.kb_per_split - 1) / pl.kb_per_split;   // every split non-empty
+    pl.units = static_cast<int>(tiles * pl.split);
+    pl.grid = pl.units < num_sms() ? pl.units : num_sms();
+    pl.max_contrib = pl.split;
+  }
+  if (pl.max_contrib > 1) {
     pl.counter_bytes = ((static_cast<size_t>(tiles) * epi_warps(v, blockwise) * sizeof(int) + 255) / 256) * 256;
-    pl.ws_bytes = pl.counter_bytes + static_cast<size_t>(tiles) * pl.split * BM * v.block_n * sizeof(float);
+    pl.ws_bytes = pl.counter_bytes + static_cast<size_t>(tiles) * pl.max_contrib * BM * v.block_n * sizeof(float);
   } else {
     pl.counter_bytes = 0;
     pl.ws_bytes = 0;
@@ -659,8 +801,12 @@ fp8q_status run_gemm(const void* a_q, const void* b_q, GemmArgs& p, const Plan& 
   p.split = pl.split;
   p.kb_per_split = pl.kb_per_split;
   p.units = pl.units;
-  p.counters = pl.split > 1 ? static_cast<int*>(ws) : nullptr;
-  p.ws = pl.split > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.counter_bytes) : nullptr;
+  p.streamk = pl.streamk;
+  p.seg_len = pl.seg_len;
+  p.total_iters = pl.total_iters;
+  p.max_contrib = pl.max_contrib;
+  p.counters = pl.max_contrib > 1 ? static_cast<int*>(ws) : nullptr;
+  p.ws = pl.max_contrib > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.counter_bytes) : nullptr;
   p.status = device_status_ptr();
   const int bn = pl.v.block_n;
   if (pl.v.swap_ab) {
@@ -707,7 +853,7 @@ extern "C" fp8q_status fp8q_select_gemm_variant(int64_t M, int64_t N, int64_t K,
   if (!out || M < 0 || N <= 0 || K <= 0) return FP8Q_ERR_INVALID_ARG;
   *out = pick_variant(M, N, K, blockwise);
   const Plan pl = make_plan(M, N, K, blockwise, *out);
-  out->split_k = pl.split;
+  out->split_k = pl.streamk ? 0 : pl.split;
   return FP8Q_OK;
 }
 
@@ -825,9 +971,16 @@ extern "C" fp8q_status fp8q_scaled_mm_blockwise_noalloc(const void* a_q, const v
   if (N % 128 != 0 || K % 128 != 0 || as_stride_m < 0 || as_stride_kb < 0)
     return FP8Q_ERR_INVALID_ARG;
   if (M == 0) return FP8Q_OK;
-  const fp8q_gemm_variant v = pick_variant(M, N, K, 1);
+  bool forced = false;
+  fp8q_gemm_variant v = pick_variant(M, N, K, 1, &forced);
   if (!variant_supported(v, 1)) return FP8Q_ERR_UNSUPPORTED;
-  const Plan pl = make_plan(M, N, K, 1, v);
+  Plan pl = make_plan(M, N, K, 1, v);
+  if (pl.ws_bytes > FP8Q_NOALLOC_SCRATCH_BYTES && !forced) {
+    // The chosen split's partials do not fit the fixed array; whole-K tiles
+    // need no scratch at all.
+    v.split_k = 1;
+    pl = make_plan(M, N, K, 1, v);
+  }
   if (pl.ws_bytes > FP8Q_NOALLOC_SCRATCH_BYTES) return FP8Q_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -1,0 +1,186 @@
+"""Time every GEMM variant on this GPU and write the library's variant table.
+
+    python -m fp8_quantized_linear_rms_b200.tune [--out FILE] [--json FILE] [--reps N]
+
+For each scheme (per-token/per-channel scales, 1x128/128x128 block scales),
+each linear-layer shape (N, K) of the Qwen3-8B and Qwen3-32B models and each
+bucket of M, every candidate variant -- Swap-AB or not, tile width, whole-K
+tiles, split-K factors, stream-K -- is timed on the device, and the fastest
+goes into ``csrc/fp8q_variant_table.inc``, which ``fp8q_gemm.cu`` compiles in.
+Rebuild the library afterwards (``python fp8_quantized_linear_rms_b200/build.py``).
+
+Timing: CUDA events around a run of back-to-back calls, each on its own copy
+of the weight matrix, with enough copies (384 MiB in all, 2 to 64 of them) that every
+call reads its weights from HBM as a model's successive layers do; the time
+per call is the median over trials of the run's mean.
+
+Where variants come within 2% of the fastest, the simplest wins, in this
+order: whole-K tiles, split-K, stream-K (they need no / a fixed / a larger
+workspace).  Operands are random e4m3 codes and positive scales; the time of a
+variant does not depend on the values.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+
+import torch
+
+import fp8_quantized_linear_rms_b200 as fq
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+# (name, K, N) of the linear layers: Qwen3-8B (hidden 4096, intermediate 12288,
+# 32 query / 8 kv heads of 128), Qwen3-32B (hidden 5120, intermediate 25600,
+# 64 query / 8 kv heads of 128), and a square 2048 layer.
+SHAPES = [
+    ("qwen3-8b qkv", 4096, 6144), ("qwen3-8b o", 4096, 4096),
+    ("qwen3-8b gate_up", 4096, 24576), ("qwen3-8b down", 12288, 4096),
+    ("qwen3-32b qkv", 5120, 10240), ("qwen3-32b o", 8192, 5120),
+    ("qwen3-32b gate_up", 5120, 51200), ("qwen3-32b down", 25600, 5120),
+    ("square 2048", 2048, 2048),
+]
+M_BUCKETS = [1, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192]
+TIE = 1.02
+
+
+def _tiles(rows_a: int, rows_b: int, bn: int) -> int:
+    return -(-rows_a // 128) * -(-rows_b // bn)
+
+
+def _splits(tiles: int, kblocks: int, sms: int) -> list[int]:
+    out = [1]
+    if tiles < 2 * sms:
+        out.append(0)                       # stream-K
+    if tiles < sms:
+        fit = sms // tiles
+        for s in sorted({2, 3, 4, 6, 8, fit}):
+            if 1 < s <= min(fit, kblocks):
+                out.append(s)
+    return out
+
+
+def candidates(M: int, N: int, K: int, sms: int) -> list[tuple[int, int, int]]:
+    kb = K // 128
+    out = []
+    if M <= 128:
+        bn = next(b for b in (16, 32, 64, 128) if b >= M)
+        for b in sorted({bn, min(128, 2 * bn)}):
+            out += [(1, s, b) for s in _splits(_tiles(N, M, b), kb, sms)]
+    if M >= 32:
+        for b in (128, 256):
+            out += [(0, s, b) for s in _splits(_tiles(M, N, b), kb, sms)]
+    return out
+
+
+def _complexity(v):
+    return 0 if v[1] == 1 else (1 if v[1] > 1 else 2)
+
+
+def _time_run(fns, trials: int) -> float:
+    """Mean time per call (us) of calling fns[0], fns[1], ... back to back."""
+    for f in fns:
+        f()
+    torch.cuda.synchronize()
+    per = []
+    for _ in range(trials):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        # The GPU sleeps while the host queues the run, so host-side call
+        # overhead never leaves the GPU idle between the timed calls.
+        torch.cuda._sleep(50_000 * len(fns))
+        a.record()
+        for f in fns:
+            f()
+        b.record()
+        b.synchronize()
+        per.append(a.elapsed_time(b) * 1e3 / len(fns))
+    return statistics.median(per)
+
+
+def tune(reps: int = 5, shapes=SHAPES, buckets=M_BUCKETS, log=print):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    rows = []
+    for name, K, N in shapes:
+        copies = max(2, min(64, -(-(384 << 20) // (N * K))))
+        bs = [torch.randint(0, 0x7E, (N, K), dtype=torch.uint8, device=dev, generator=g)
+              .view(torch.float8_e4m3fn) for _ in range(copies)]
+        sb_ch = torch.rand(N, device=dev, generator=g) * 1e-3
+        sb_bl = torch.rand((N // 128, K // 128), device=dev, generator=g) * 1e-3
+        for M in buckets:
+            a = torch.randint(0, 0x7E, (M, K), dtype=torch.uint8, device=dev, generator=g)
+            a = a.view(torch.float8_e4m3fn)
+            sa_tok = torch.rand(M, device=dev, generator=g) * 1e-3
+            sa_grp = torch.rand((K // 128, M), device=dev, generator=g) * 1e-3
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            for bw in (0, 1):
+                times = {}
+                for v in candidates(M, N, K, sms):
+                    fq.fp8q_force_gemm_variant(*v)
+                    try:
+                        ws = fq.make_workspace(M, N, K, bool(bw), dev)
+                        if bw:
+                            fns = [lambda b=b: fq.fp8q_scaled_mm_blockwise(
+                                a, b, sa_grp, sb_bl, a_scale_layout="group_major", y=y,
+                                workspace=ws) for b in bs]
+                        else:
+                            fns = [lambda b=b: fq.fp8q_scaled_mm(a, b, sa_tok, sb_ch, y=y,
+                                                                 workspace=ws) for b in bs]
+                        times[v] = _time_run(fns, reps)
+                    finally:
+                        fq.fp8q_force_gemm_variant()
+                best_t = min(times.values())
+                best = min((v for v, t in times.items() if t <= best_t * TIE),
+                           key=lambda v: (_complexity(v), times[v]))
+                row = {"shape": name, "blockwise": bw, "m_max": M, "N": N, "K": K,
+                       "variant": list(best), "us": round(times[best], 2),
+                       "tflops": round(2.0 * M * N * K / times[best] / 1e6, 1),
+                       "all": {f"{v[0]},{v[1]},{v[2]}": round(t, 2) for v, t in times.items()}}
+                rows.append(row)
+                log(json.dumps(row))
+            del a, y
+        del bs
+    return rows
+
+
+def write_table(rows, path: str) -> None:
+    dev = torch.cuda.get_device_name()
+    with open(path, "w") as f:
+        f.write(f"// Measured GEMM variant table, written by tune.py on {dev}\n")
+        f.write(f"// ({datetime.date.today().isoformat()}): the fastest variant per scheme, (N, K)\n")
+        f.write("// and bucket of M (mean microseconds per call, weights read from HBM).\n")
+        f.write("// {blockwise, m_max, N, K, swap_ab, split_k (0 = stream-K), block_n}\n")
+        for r in rows:
+            s, k, n = r["variant"]
+            f.write(f"{{{r['blockwise']}, {r['m_max']}, {r['N']}, {r['K']}, {s}, {k}, {n}}},"
+                    f"  // {r['shape']}: {r['us']} us\n")
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--out", default=os.path.join(HERE, "csrc", "fp8q_variant_table.inc"))
+    ap.add_argument("--json", default=None, help="also write every timing as JSON lines")
+    ap.add_argument("--reps", type=int, default=5, help="trials per variant")
+    args = ap.parse_args()
+    jf = open(args.json, "w") if args.json else None
+
+    def log(line):
+        print(line, flush=True)
+        if jf:
+            jf.write(line + "\n")
+            jf.flush()
+
+    rows = tune(args.reps, log=log)
+    write_table(rows, args.out)
+    if jf:
+        jf.close()
+
+
+if __name__ == "__main__":
+    main()

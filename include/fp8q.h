@@ -181,9 +181,12 @@ FP8Q_API fp8q_status fp8q_scaled_mm_blockwise(const void* a_q, const void* b_q, 
  * which every GPU that loads the library holds until the process exits.
  *
  *   Arguments are those of fp8q_scaled_mm_blockwise without the workspace.
- *   Returns FP8Q_ERR_UNSUPPORTED, launching nothing, when the shape's split-K
- *   scratch (fp8q_workspace_bytes(M, N, K, 1)) exceeds
- *   FP8Q_NOALLOC_SCRATCH_BYTES.
+ *   When the automatically chosen variant's split-K scratch
+ *   (fp8q_workspace_bytes(M, N, K, 1)) exceeds FP8Q_NOALLOC_SCRATCH_BYTES,
+ *   the call runs that variant's tile shape with whole-K tiles (no scratch)
+ *   instead.  A variant set by fp8q_force_gemm_variant is not changed: if its
+ *   scratch does not fit, the call returns FP8Q_ERR_UNSUPPORTED and launches
+ *   nothing.
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress); make that first call before any stream capture.
  *   Every call clears the part of the array that must start at zero (the
@@ -209,21 +212,29 @@ FP8Q_API size_t fp8q_workspace_bytes(int64_t M, int64_t N, int64_t K, int blockw
 /* A GEMM variant ("Helion linear backend" (aihirek.info), section "Single
  * GEMM implementation handles several algorithms"): swap_ab = 1 computes
  * (B A^T)^T so the tokens sit in the MMA's N slot; split_k > 1 divides the K
- * loop among that many CTAs per output tile; block_n is the MMA N extent. */
+ * loop of every output tile among that many CTAs; split_k = 0 selects
+ * stream-K: every CTA (at most one per SM) takes an equal contiguous range of
+ * (tile, K block) iterations and tiles cut by range boundaries are summed
+ * from their pieces in a fixed order; block_n is the MMA N extent. */
 typedef struct {
     int swap_ab;
     int split_k;
     int block_n;
 } fp8q_gemm_variant;
 
-/* The variant the library would run for this shape.  Returns FP8Q_OK. */
+/* The variant the library would run for this shape: the row of its built-in
+ * table of variants measured fastest on a B200 (the shapes of the Qwen3-8B
+ * and Qwen3-32B linear layers, per bucket of M; written by the package's
+ * tune.py), else a rule drawn from the same measurements.  The split_k it
+ * reports is the one that runs (a split larger than the number of K blocks
+ * is reduced).  Returns FP8Q_OK. */
 FP8Q_API fp8q_status fp8q_select_gemm_variant(int64_t M, int64_t N, int64_t K, int blockwise,
                                      fp8q_gemm_variant* out);
 
 /* Force a variant for every following GEMM call in this process (testing and
  * tuning only; not thread-safe).  NULL restores automatic selection.  Returns
  * FP8Q_ERR_INVALID_ARG if the variant is malformed (block_n not one of
- * 16, 32, 64, 128, 256; split_k < 1). */
+ * 16, 32, 64, 128, 256; split_k < 0 or > 64). */
 FP8Q_API fp8q_status fp8q_force_gemm_variant(const fp8q_gemm_variant* v);
 
 /* ------------------------------------------------------------------------ */

@@ -2,10 +2,14 @@
 and validates arguments on the host (no kernel is launched by these calls, so
 they run without a GPU)."""
 import ctypes
+import os
+import re
 
 import pytest
 
 import fp8_quantized_linear_rms_b200 as fq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_library_exports_every_declared_function():
@@ -57,17 +61,55 @@ def test_zero_rows_is_a_noop_without_pointers():
                                       None) == fq.OK
 
 
+def _variant_table():
+    """Rows of the compiled-in variant table, read from its source text."""
+    path = os.path.join(ROOT, "fp8_quantized_linear_rms_b200", "csrc", "fp8q_variant_table.inc")
+    rows = []
+    for line in open(path):
+        m = re.match(r"\{(-?\d+), (\d+), (\d+), (\d+), (\d+), (\d+), (\d+)\},", line)
+        if m:
+            rows.append(tuple(int(x) for x in m.groups()))
+    return rows
+
+
+def test_variant_table_lookup():
+    rows = _variant_table()
+    assert len(rows) >= 100
+    keys = {}
+    for bw, m_max, n, k, swap, split, bn in rows:
+        keys.setdefault((bw, n, k), []).append(m_max)
+        want = {"swap_ab": swap, "split_k": split, "block_n": bn}
+        assert fq.fp8q_select_gemm_variant(m_max, n, k, bool(bw)) == want
+    # an M between buckets takes the next larger bucket; above all, the largest
+    for (bw, n, k), ms in keys.items():
+        ms = sorted(ms)
+        by_m = {r[1]: r for r in rows if (r[0], r[2], r[3]) == (bw, n, k)}
+        for lo, hi in zip(ms, ms[1:]):
+            if hi - lo > 1:
+                r = by_m[hi]
+                assert fq.fp8q_select_gemm_variant(lo + 1, n, k, bool(bw)) == \
+                    {"swap_ab": r[4], "split_k": r[5], "block_n": r[6]}
+        r = by_m[ms[-1]]
+        assert fq.fp8q_select_gemm_variant(ms[-1] * 4, n, k, bool(bw)) == \
+            {"swap_ab": r[4], "split_k": r[5], "block_n": r[6]}
+
+
 def test_variant_selection_host_logic():
-    # small M: Swap-AB with tokens padded to 16/32/64; large M: no swap
-    assert fq.fp8q_select_gemm_variant(1, 10240, 5120, True)["swap_ab"] == 1
-    assert fq.fp8q_select_gemm_variant(1, 10240, 5120, True)["block_n"] == 16
-    assert fq.fp8q_select_gemm_variant(33, 10240, 5120, True)["block_n"] == 64
-    v = fq.fp8q_select_gemm_variant(8192, 51200, 5120, False)
-    assert v["swap_ab"] == 0 and v["split_k"] == 1
-    # Split-K only where tiles cannot fill the SMs; every split non-empty
-    v = fq.fp8q_select_gemm_variant(16, 5120, 25600, True)
-    assert v["split_k"] > 1
-    assert fq.fp8q_workspace_bytes(16, 5120, 25600, True) > 0
+    # shapes outside the table: Swap-AB with tokens padded to 16/32/64/128 for
+    # small M, no swap for large M
+    N, K = 3072, 2560
+    assert fq.fp8q_select_gemm_variant(1, N, K, True)["swap_ab"] == 1
+    assert fq.fp8q_select_gemm_variant(1, N, K, True)["block_n"] == 16
+    assert fq.fp8q_select_gemm_variant(33, N, K, True)["block_n"] == 64
+    assert fq.fp8q_select_gemm_variant(100, N, K, False)["block_n"] == 128
+    v = fq.fp8q_select_gemm_variant(8192, N, K, False)
+    assert v == {"swap_ab": 0, "split_k": 1, "block_n": 256}
+    # 24 tiles: whole-K ranges split so that the tiles fill the SMs, each
+    # range at least 8 K blocks; blockwise with M > 16 takes stream-K
+    assert fq.fp8q_select_gemm_variant(16, N, K, False)["split_k"] == 2
+    assert fq.fp8q_select_gemm_variant(16, N, 8 * 128 * 6, False)["split_k"] == 6
+    assert fq.fp8q_select_gemm_variant(64, N, K, True)["split_k"] == 0
+    assert fq.fp8q_workspace_bytes(64, N, K, True) > 0
     assert fq.fp8q_workspace_bytes(8192, 51200, 5120, False) == 0
     # forcing
     fq.fp8q_force_gemm_variant(0, 2, 256)

@@ -52,7 +52,7 @@ def _run_bw(a, b, sa, sb, M, N, K, layout="row_major"):
     return bf16_to_np(y)
 
 
-@pytest.mark.parametrize("split", [1, 3])
+@pytest.mark.parametrize("split", [0, 1, 3])
 @pytest.mark.parametrize("swap,bn", PT_VARIANTS)
 @pytest.mark.parametrize("M,N,K", [(1, 256, 384), (100, 272, 400), (260, 384, 1024)])
 def test_scaled_mm_variants(M, N, K, swap, bn, split):
@@ -66,7 +66,7 @@ def test_scaled_mm_variants(M, N, K, swap, bn, split):
     gemm_tolerance_check(y, y_ref, ad, f"pt swap={swap} bn={bn} split={split}")
 
 
-@pytest.mark.parametrize("split", [1, 3])
+@pytest.mark.parametrize("split", [0, 1, 3])
 @pytest.mark.parametrize("swap,bn", BW_VARIANTS)
 @pytest.mark.parametrize("M,N,K", [(1, 256, 384), (100, 384, 512), (260, 256, 1024)])
 def test_scaled_mm_blockwise_variants(M, N, K, swap, bn, split):
@@ -116,9 +116,10 @@ def test_small_k_tail():
         gemm_tolerance_check(y, y_ref, ad, f"K tail swap={swap}")
 
 
+@pytest.mark.parametrize("split", [0, 4])
 @pytest.mark.parametrize("blockwise", [False, True])
 @pytest.mark.parametrize("swap,bn", [(0, 128), (1, 32)])
-def test_output_canaries_and_split_determinism(blockwise, swap, bn):
+def test_output_canaries_and_split_determinism(blockwise, swap, bn, split):
     # y is a view into a larger buffer (extra columns and rows): nothing outside
     # [M, N] may change; split-K results are bit-identical across runs and the
     # workspace is reusable without clearing.
@@ -127,7 +128,7 @@ def test_output_canaries_and_split_determinism(blockwise, swap, bn):
     b = inp.random_e4m3_codes(52, (N, K))
     sa = inp.random_scales(53, (M, K // 128) if blockwise else (M,))
     sb = inp.random_scales(54, (N // 128, K // 128) if blockwise else (N,))
-    fq.fp8q_force_gemm_variant(swap, 4, bn)
+    fq.fp8q_force_gemm_variant(swap, split, bn)
     ws = fq.make_workspace(M, N, K, blockwise)
     assert ws is not None
     big = torch.full((M + 3, N + 24), 7.0, dtype=torch.bfloat16, device="cuda")

@@ -28,19 +28,36 @@ if torch.cuda.is_available():
 def test_noalloc_matches_workspace_entry_point(M, N, K):
     fq.fp8q_force_gemm_variant()
     v = fq.fp8q_select_gemm_variant(M, N, K, True)
-    assert v["split_k"] > 1, "the shape must exercise the split-K scratch"
+    assert v["split_k"] != 1, "the shape must exercise the split-K / stream-K scratch"
     assert 0 < fq.fp8q_workspace_bytes(M, N, K, True) <= fq.NOALLOC_SCRATCH_BYTES
+    _compare_two_calls(M, N, K)
+
+
+def test_noalloc_runs_whole_k_tiles_when_the_split_scratch_does_not_fit():
+    # the automatic variant of this shape wants more split-K scratch than the
+    # fixed array holds: the call runs the same tiles with whole K ranges
+    M, N, K = 64, 24576, 4096
+    fq.fp8q_force_gemm_variant()
+    assert fq.fp8q_workspace_bytes(M, N, K, True) > fq.NOALLOC_SCRATCH_BYTES
+    _compare_two_calls(M, N, K)
+
+
+def _compare_two_calls(M, N, K):
     a = to_dev_codes(inp.random_e4m3_codes(M + 1, (M, K)))
     b = to_dev_codes(inp.random_e4m3_codes(N + 2, (N, K)))
     sa = torch.from_numpy(inp.random_scales(3, (M, K // 128))).cuda()
     sb = torch.from_numpy(inp.random_scales(4, (N // 128, K // 128))).cuda()
     y_ws = fq.fp8q_scaled_mm_blockwise(a, b, sa, sb, workspace=fq.make_workspace(M, N, K, True))
     torch.cuda.synchronize()
-    # |a_k b_k| sums for the tolerance, from the oracle on every row
-    _, absdot = oracle.scaled_mm_blockwise(a.view(torch.uint8).cpu().numpy(),
-                                           b.view(torch.uint8).cpu().numpy(),
-                                           sa.cpu().numpy(), sb.cpu().numpy())
-    ref = bf16_to_np(y_ws).astype(np.float64)
+    # the oracle's fp64 result and |a_k b_k| sums, on every row
+    ref, absdot = oracle.scaled_mm_blockwise(a.view(torch.uint8).cpu().numpy(),
+                                             b.view(torch.uint8).cpu().numpy(),
+                                             sa.cpu().numpy(), sb.cpu().numpy())
+    y_ws_np = bf16_to_np(y_ws)
+    gemm_tolerance_check(y_ws_np, ref, absdot, "workspace entry point")
+    # the same variant sums in the same order: bit-identical to the workspace entry
+    v = fq.fp8q_select_gemm_variant(M, N, K, True)
+    same_variant = fq.fp8q_workspace_bytes(M, N, K, True) <= fq.NOALLOC_SCRATCH_BYTES
     stream = torch.cuda.current_stream().cuda_stream
     for call in range(2):
         y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
@@ -50,7 +67,11 @@ def test_noalloc_matches_workspace_entry_point(M, N, K):
         assert st == fq.OK, fq.fp8q_status_string(st)
         torch.cuda.synchronize()
         assert fq.fp8q_last_device_status() == fq.OK
-        gemm_tolerance_check(bf16_to_np(y), ref, absdot, f"noalloc call {call + 1}")
+        got = bf16_to_np(y)
+        gemm_tolerance_check(got, ref, absdot, f"noalloc call {call + 1} ({v})")
+        if same_variant:
+            assert np.array_equal(got, y_ws_np), \
+                f"noalloc call {call + 1} differs from the workspace entry point"
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
