@@ -5,23 +5,30 @@
 //   items 2, 6  RMSNorm + per-token / per-block quant       -> fp8q_rmsnorm_quant
 //   items 3, 7  SiLU*mul + per-token / per-block quant      -> fp8q_silu_mul_quant
 //
-// One CTA owns one row.  Every thread loads its 16-byte chunks of the row
-// (8 bf16 each; chunk c of the row goes to thread c mod T, so a warp reads 512
-// contiguous bytes per load), all loads issued before any arithmetic.  The row
-// then stays in registers as packed bf16 y values: one HBM read, one write of
-// the codes.  Group amax = shuffle over the 16 threads that own one 128-wide
-// group; row amax and the RMSNorm sum of squares = warp shuffle + a shared-
-// memory pass over the warps.
+// One CTA (or, for long rows, one team of a CTA) owns one row.  Every thread
+// loads its 16-byte chunks of the row (8 bf16 each; chunk c of the row goes
+// to thread c mod T, so a warp reads 512 contiguous bytes per load), all loads
+// issued before any arithmetic; many CTAs per SM keep enough loads in flight.
+// The row then stays in registers as packed bf16 y values: one HBM read, one
+// write of the codes.  Group amax = shuffle over the 16 threads that own one
+// 128-wide group; row amax and the RMSNorm sum of squares = warp shuffle + a
+// shared-memory pass over the warps.  Rows of more than 2048 chunks are
+// streamed into shared memory by a bulk-copy ring instead (quant_ring_kernel).
 //
-// Exactness.  Codes and scales are meant to equal the definition bit for bit:
-//   - the scale is an IEEE fp32 division, the codes come from an IEEE fp32
-//     division x/s and the hardware saturating RNE e4m3 conversion;
-//   - y must be the correctly rounded bf16 of the op's real value.  The fast
-//     path computes it in fp32 with a known error bound (a few fp32 ulps); when
-//     that fp32 value lies within the bound of a bf16 rounding midpoint, or is
-//     tiny, the element is recomputed in fp64 and rounded to bf16 once
-//     (round-to-odd to fp32, then nearest-even to bf16).  The RMSNorm sum of
-//     squares and 1/sqrt are fp64.
+// Exactness.  Codes and scales equal the definition bit for bit:
+//   - the scale is fl32(max(amax, 1e-10) / 448) (IEEE division, recovered
+//     from a product and its FMA residual); codes are the saturating RNE e4m3
+//     of fl32(y / s), the IEEE quotient obtained with Markstein's division
+//     step from the correctly rounded reciprocal of s (quant_chunk).
+//   - y must be the correctly rounded bf16 of the op's real value.  RMSNorm:
+//     n = bf16(x r) from a = rz(x r_lo) and b = rz(x r_hi) + 1 ulp, whose
+//     magnitudes bracket |x r| for every x, subnormal results included;
+//     SiLU*mul: the fp32 value and its proven error bound give the bracket.
+//     Equal roundings of both ends are the rounding of the real value; pairs
+//     whose ends differ (or, for SiLU, that are tiny or have a gate below
+//     -85) are recomputed in fp64 and rounded to bf16 once.
+//   - The RMSNorm sum of squares is accumulated in fp64, where squares of
+//     bf16 values are exact; r is rsqrtf refined by one Newton step in fp64.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -30,6 +37,8 @@
 
 namespace fp8q {
 namespace {
+
+using namespace sm100;
 
 enum { OP_PLAIN = 0, OP_RMS = 1, OP_SILU = 2 };
 constexpr int kMaxThreads = 512;  // rows up to 8 * 8 * 512 = 32768 elements
@@ -47,6 +56,9 @@ struct QuantParams {
   int64_t s_sm, s_sg;
 };
 
+// ---------------------------------------------------------------------------
+// Scalar helpers
+
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float(b16 << 16); }
 
 __device__ __forceinline__ uint32_t f32_to_bf16_bits_rn(float f) {
@@ -60,64 +72,6 @@ __device__ __noinline__ uint32_t f64_to_bf16_bits_rn(double v) {
   float f = __double2float_rz(v);
   if (static_cast<double>(f) != v) f = __uint_as_float(__float_as_uint(f) | 1u);
   return f32_to_bf16_bits_rn(f);
-}
-
-// ---------------------------------------------------------------------------
-// Paired fp32 arithmetic (sm_100 .f32x2: two IEEE fp32 operations per
-// instruction).  A pair travels as one 64-bit register: low word = element 0.
-__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void up2(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-// bf16x2 word (element 0 in the low half) <-> fp32 pair.
-__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
-  return pk2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
-__device__ __forceinline__ uint32_t f2_to_bf2_rn(uint64_t v) {
-  float a, b;
-  up2(v, a, b);
-  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-__device__ __forceinline__ uint32_t f2_to_e4m3x2(uint64_t v) {
-  float a, b;
-  up2(v, a, b);
-  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
-}
-
-// Rounding-decision test used by every fast path below.  A fast fp32 value p
-// is within a proven relative error e < delta of the exact value v; the two
-// ends p(1 - delta) and p(1 + delta) (each one more rounding) bracket v.
-// Rounding to nearest is monotone, so if both ends round to the same code, v
-// rounds to it as well; otherwise the element takes the exact slow path.
-constexpr float kBf16Lo = 1.0f - 0x1p-20f, kBf16Hi = 1.0f + 0x1p-20f;   // errors < 2^-21.7
-constexpr float kSiluLo = 1.0f - 0x1p-19f, kSiluHi = 1.0f + 0x1p-19f;   // errors <= 2^-20.6
-constexpr float kE4m3Lo = 1.0f - 0x1p-21f, kE4m3Hi = 1.0f + 0x1p-21f;   // errors <= 2^-22
-constexpr float kTiny = 0x1p-100f;  // below this fp32 products may lose relative precision
-
-// Two fp32 values -> bf16x2 word (element 0 in the low half), nearest even.
-__device__ __forceinline__ uint32_t bf2_rn(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // Hardware approximations with error bounds measured exhaustively (every
@@ -134,56 +88,61 @@ __device__ __forceinline__ float rcp_approx(float s) {
   return r;
 }
 
-// e^x for |x| <= 87 as 2^(x log2 e) with the exponent split exactly
-// (Cody & Waite argument splitting): a = fl(x * L2E) plus the exact FMA
-// residual of that product and x times the error of L2E itself; then
-// 2^a * (1 + lo ln 2).  Relative error <= 2^-22.2 (measured exhaustively
-// over every fp32 x in [-87, 87]).
-__device__ __forceinline__ float exp_fast(float x) {
-  const float L2E = 1.44269502f;           // fl32(log2 e)
-  const float L2E_LO = 1.925963e-8f;       // log2 e - L2E
-  const float a = __fmul_rn(x, L2E);
-  const float lo = __fmaf_rn(x, L2E_LO, __fmaf_rn(x, L2E, -a));
-  const float e = ex2_approx(a);
-  return __fmaf_rn(e, __fmul_rn(lo, 0.693147182f), e);
+// ---------------------------------------------------------------------------
+// Paired fp32 arithmetic (sm_100 .f32x2: two IEEE fp32 operations per
+// instruction).  A pair travels as one 64-bit register: low word = element 0.
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
 }
-
-// The rare exact paths, kept out of line: inlined into every unrolled element
-// position they would overflow the instruction cache.
-// r = 1 / sqrt(mean(x^2) + eps) in fp64 from the fp64 row sum of squares.
-__device__ __forceinline__ double rms_inv_f64(double ss, int64_t L, float eps) {
-  return 1.0 / sqrt(ss / static_cast<double>(L) + static_cast<double>(eps));
+__device__ __forceinline__ void up2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
-
-__device__ __noinline__ uint32_t rms_pair_f64(uint32_t xw, double ss, int64_t L, float eps) {
-  const double r = rms_inv_f64(ss, L, eps);
-  const uint32_t lo = f64_to_bf16_bits_rn(static_cast<double>(bf16_bits_to_f32(xw & 0xFFFFu)) * r);
-  const uint32_t hi = f64_to_bf16_bits_rn(static_cast<double>(bf16_bits_to_f32(xw >> 16)) * r);
-  return lo | (hi << 16);
+__device__ __forceinline__ uint64_t dup2(float v) { return pk2(v, v); }
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
-
-__device__ __noinline__ uint32_t silu_pair_f64(uint32_t gw, uint32_t uw) {
-  uint32_t out = 0;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const double g = bf16_bits_to_f32((gw >> (16 * h)) & 0xFFFFu);
-    const double u = bf16_bits_to_f32((uw >> (16 * h)) & 0xFFFFu);
-    out |= f64_to_bf16_bits_rn(g / (1.0 + exp(-g)) * u) << (16 * h);
-  }
-  return out;
+__device__ __forceinline__ uint64_t mulz2(uint64_t a, uint64_t b) {   // toward zero
+  uint64_t r;
+  asm("mul.rz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// Both elements one unit in the last place further from zero (finite
+// values: the bit patterns are sign-magnitude, and no carry crosses lanes).
+__device__ __forceinline__ uint64_t bump2(uint64_t v) { return v + 0x0000000100000001ull; }
 
-// RMSNorm pair, fast path: n = bf16(x * r) from p = fl(x * r32) with r32 the
-// fp32 rsqrt (relative error < 2^-21.7 in all), bracket +-2^-20.  `unsafe` is set when the
-// bracket does not decide the rounding or |p| is tiny; the caller then
-// recomputes the pair exactly (rms_pair_f64).
-__device__ __forceinline__ uint32_t rms_n_fast(uint32_t xw, float r32, bool& unsafe) {
-  const float p0 = __fmul_rn(__uint_as_float(xw << 16), r32);
-  const float p1 = __fmul_rn(__uint_as_float(xw & 0xFFFF0000u), r32);
-  const uint32_t lo = bf2_rn(__fmul_rn(p0, kBf16Lo), __fmul_rn(p1, kBf16Lo));
-  const uint32_t hi = bf2_rn(__fmul_rn(p0, kBf16Hi), __fmul_rn(p1, kBf16Hi));
-  unsafe = (lo != hi) || fminf(fabsf(p0), fabsf(p1)) < kTiny;
-  return lo;
+// bf16x2 word (element 0 in the low half) <-> fp32 pair.
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
+  return pk2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t f2_to_bf2_rn(uint64_t v) {
+  float a, b;
+  up2(v, a, b);
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t f2_to_e4m3x2(uint64_t v) {
+  float a, b;
+  up2(v, a, b);
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
 }
 
 // y = bf16(n * w): one exactly rounded bf16 multiply per half (the product of
@@ -194,25 +153,20 @@ __device__ __forceinline__ uint32_t bf2_mul(uint32_t n, uint32_t w) {
   return *reinterpret_cast<const uint32_t*>(&y);
 }
 
-// SiLU*mul element, fast: silu(g) * u = g * (1 / (1 + e^-g)) * u with
-// exp_fast (<= 2^-22.2), one rounding of 1 + e, rcp_approx (<= 2^-23.3) and
-// two multiplications: relative error <= 2^-20.6.
-__device__ __forceinline__ float silu_mul_fast(float g, float u) {
-  const float d = __fadd_rn(1.0f, exp_fast(-g));
-  return __fmul_rn(__fmul_rn(g, rcp_approx(d)), u);
+// max |y| of 8 bf16 values, accumulated packed (|.| = sign bits cleared).
+__device__ __forceinline__ uint32_t chunk_absmax2(const uint4& y, uint32_t m) {
+  const uint32_t w[4] = {y.x & 0x7FFF7FFFu, y.y & 0x7FFF7FFFu, y.z & 0x7FFF7FFFu, y.w & 0x7FFF7FFFu};
+  __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&m);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) a = __hmax2(a, *reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+  return *reinterpret_cast<const uint32_t*>(&a);
+}
+__device__ __forceinline__ float absmax2_to_f32(uint32_t m) {
+  return fmaxf(bf16_bits_to_f32(m & 0xFFFFu), bf16_bits_to_f32(m >> 16));
 }
 
-// SiLU*mul pair: bracket +-2^-19; gates below -85 (e^-g beyond the fast
-// exp's range) and tiny results take the exact path.
-__device__ __forceinline__ uint32_t silu_pair_fast(uint32_t gw, uint32_t uw, bool& unsafe) {
-  const float g0 = __uint_as_float(gw << 16), g1 = __uint_as_float(gw & 0xFFFF0000u);
-  const float p0 = silu_mul_fast(g0, __uint_as_float(uw << 16));
-  const float p1 = silu_mul_fast(g1, __uint_as_float(uw & 0xFFFF0000u));
-  const uint32_t lo = bf2_rn(__fmul_rn(p0, kSiluLo), __fmul_rn(p1, kSiluLo));
-  const uint32_t hi = bf2_rn(__fmul_rn(p0, kSiluHi), __fmul_rn(p1, kSiluHi));
-  unsafe = (lo != hi) || fminf(fabsf(p0), fabsf(p1)) < kTiny || fminf(g0, g1) < -85.0f;
-  return lo;
-}
+// ---------------------------------------------------------------------------
+// Scales and codes
 
 // Scale of a group: fl32(max(amax, 1e-10) / 448), UE8M0: rounded up to a
 // power of two.  The quotient is q0 = a * fl(1/448) corrected once by its
@@ -233,46 +187,187 @@ __device__ __forceinline__ float group_scale(float amax, int ue8m0) {
   return s;
 }
 
-// Codes of a chunk by IEEE division, for the rare chunk whose fast codes
-// could differ (out of line).
-__device__ __noinline__ uint2 quantize_chunk_ieee(const uint4 y, float s) {
-  const uint32_t w[4] = {y.x, y.y, y.z, y.w};
-  uint32_t c[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    c[j] = f2_to_e4m3x2(pk2(__fdiv_rn(bf16_bits_to_f32(w[j] & 0xFFFFu), s),
-                            __fdiv_rn(bf16_bits_to_f32(w[j] >> 16), s)));
-  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+// A scale with what the codes need: the correctly rounded reciprocal
+// rcp = RN(1/s) and -s, both duplicated into pairs.
+struct QScale {
+  float s;
+  uint64_t rcp2, neg2;
+};
+__device__ __forceinline__ QScale make_qscale(float amax, int ue8m0) {
+  QScale q;
+  q.s = group_scale(amax, ue8m0);
+  q.rcp2 = dup2(__frcp_rn(q.s));
+  q.neg2 = dup2(-q.s);
+  return q;
 }
 
-// 8 bf16 values (one chunk) -> 8 e4m3 codes of fl32(y / s), fast path:
-// t = y * rcp with rcp within 2^-23.3 of 1/s is within 2^-22 of fl32(y/s);
-// bracket +-2^-21.  `unsafe` asks the caller for quantize_chunk_ieee.
-__device__ __forceinline__ uint2 quantize_chunk_fast(const uint4& y, float rcp, bool& unsafe) {
+// 8 bf16 values (one chunk) -> 8 e4m3 codes of fl32(y / s).  The quotient is
+// the IEEE one, by Markstein's division step (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990): q0 = RN(y rcp) is within an ulp of y/s, so the residual
+// r = y - q0 s is exact under FMA and RN(q0 + r rcp) = RN(y/s) when rcp is
+// the correctly rounded 1/s.  (Quotients too small for that argument, below
+// 2^-12, become code 0 either way.)  Ties of the e4m3 rounding -- frequent:
+// bf16 data over a bf16 amax often gives quotients like 10.5 exactly -- are
+// then decided by the conversion itself, as in the definition.
+__device__ __forceinline__ uint2 quant_chunk(const uint4& y, const QScale& qs) {
   const uint32_t w[4] = {y.x, y.y, y.z, y.w};
   uint32_t c[4];
-  bool slow = false;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float t0 = __fmul_rn(__uint_as_float(w[j] << 16), rcp);
-    const float t1 = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), rcp);
-    c[j] = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
-        make_float2(__fmul_rn(t0, kE4m3Lo), __fmul_rn(t1, kE4m3Lo)), __NV_SATFINITE, __NV_E4M3));
-    const uint32_t chi = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
-        make_float2(__fmul_rn(t0, kE4m3Hi), __fmul_rn(t1, kE4m3Hi)), __NV_SATFINITE, __NV_E4M3));
-    slow |= c[j] != chi;
+  for (int k = 0; k < 4; ++k) {
+    const uint64_t f = bf2_to_f2(w[k]);
+    const uint64_t q0 = mul2(f, qs.rcp2);
+    const uint64_t r = fma2(q0, qs.neg2, f);
+    c[k] = f2_to_e4m3x2(fma2(r, qs.rcp2, q0));
   }
-  unsafe = slow;
-  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+  // The step turns y = -0 into +0; every code takes the sign bit of its y
+  // (bytes 1 and 3 of each bf16x2 word hold the two signs in their bit 7).
+  return make_uint2((c[0] | (c[1] << 16)) | (__byte_perm(w[0], w[1], 0x7531) & 0x80808080u),
+                    (c[2] | (c[3] << 16)) | (__byte_perm(w[2], w[3], 0x7531) & 0x80808080u));
 }
 
-__device__ __forceinline__ float chunk_amax(const uint4& y) {
-  // max |y| of 8 bf16 values with packed bf16 max (|.| = sign bits cleared)
-  const uint32_t w[4] = {y.x & 0x7FFF7FFFu, y.y & 0x7FFF7FFFu, y.z & 0x7FFF7FFFu, y.w & 0x7FFF7FFFu};
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(w);
-  const __nv_bfloat162 m = __hmax2(__hmax2(h[0], h[1]), __hmax2(h[2], h[3]));
-  return fmaxf(__low2float(m), __high2float(m));
+// ---------------------------------------------------------------------------
+// RMSNorm
+
+// r = 1 / sqrt(mean(x^2) + eps) in fp64 from the fp64 row sum of squares.
+__device__ __forceinline__ double rms_inv_f64(double ss, int64_t L, float eps) {
+  return 1.0 / sqrt(ss / static_cast<double>(L) + static_cast<double>(eps));
 }
+
+// Exact bf16(x * r) of a pair (out of line).
+__device__ __noinline__ uint32_t rms_pair_f64(uint32_t xw, double ss, int64_t L, float eps) {
+  const double r = rms_inv_f64(ss, L, eps);
+  const uint32_t lo = f64_to_bf16_bits_rn(static_cast<double>(bf16_bits_to_f32(xw & 0xFFFFu)) * r);
+  const uint32_t hi = f64_to_bf16_bits_rn(static_cast<double>(bf16_bits_to_f32(xw >> 16)) * r);
+  return lo | (hi << 16);
+}
+
+// n = bf16(x * r) of a pair, from the bracket ends a = rz(x r_lo) and
+// b = rz(x r_hi) + 1 ulp (r_lo <= r <= r_hi): |a| <= |x r| <= |b|.  Returns the
+// rounding of a; `d` collects the XOR with the rounding of b.
+__device__ __forceinline__ uint32_t rms_n_pair(uint32_t xw, uint64_t rlo2, uint64_t rhi2, uint32_t& d) {
+  const uint64_t f = bf2_to_f2(xw);
+  const uint32_t na = f2_to_bf2_rn(mulz2(f, rlo2));
+  d |= na ^ f2_to_bf2_rn(bump2(mulz2(f, rhi2)));
+  return na;
+}
+
+// Cold path of a flagged RMSNorm chunk: the pairs whose bracket is open get
+// the exact bf16(x r), then y = bf16(n w).
+__device__ __noinline__ uint4 rms_chunk_fix(const uint4 xv, const uint4 wv, uint4 y, uint64_t rlo2,
+                                           uint64_t rhi2, double ss, int64_t L, float eps) {
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, ww[4] = {wv.x, wv.y, wv.z, wv.w};
+  uint32_t yw[4] = {y.x, y.y, y.z, y.w};
+  for (int k = 0; k < 4; ++k) {
+    uint32_t d = 0;
+    rms_n_pair(xw[k], rlo2, rhi2, d);
+    if (d) yw[k] = bf2_mul(rms_pair_f64(xw[k], ss, L, eps), ww[k]);
+  }
+  return make_uint4(yw[0], yw[1], yw[2], yw[3]);
+}
+
+// Fast bracket of r = 1/sqrt(m): rsqrtf, one Newton step in fp64 (error
+// <= 1.5 e^2 + fp64 roundings, e <= 2^-21 the rsqrtf error: below 2^-40),
+// then the fp32 values just below and above r (1 -+ 2^-30).
+__device__ __forceinline__ void rms_bracket(double m, float& r_lo, float& r_hi) {
+  double r1;
+  if (m >= 0x1p-120 && m <= 0x1p120) {
+    const double r0 = static_cast<double>(rsqrtf(static_cast<float>(m)));
+    const double h = __fma_rn(-m * r0, r0, 1.0);          // 1 - m r0^2
+    r1 = __fma_rn(0.5 * r0, h, r0);
+  } else {
+    r1 = 1.0 / sqrt(m);
+  }
+  r_lo = __double2float_rd(r1 * (1.0 - 0x1p-30));
+  r_hi = __double2float_ru(r1 * (1.0 + 0x1p-30));
+}
+
+// ---------------------------------------------------------------------------
+// SiLU * mul
+
+// Bracket of the fast SiLU*mul value p (relative error <= 2^-20.6, below):
+// p (1 -+ 2^-19), each end one more rounding.
+constexpr float kSiluLo = 1.0f - 0x1p-19f, kSiluHi = 1.0f + 0x1p-19f;
+constexpr float kTiny = 0x1p-100f;  // below this fp32 products may lose relative precision
+
+// e^-g for a pair, |g| <= 85: 2^(-g log2 e) with the exponent split exactly
+// (Cody & Waite argument splitting): a = fl(g L2E) plus the exact FMA
+// residual of that product and g times the error of L2E itself; then
+// 2^-a (1 + lo ln 2).  Relative error <= 2^-22.2 (measured exhaustively for
+// every fp32 argument in [-87, 87] by the tests).
+__device__ __forceinline__ uint64_t exp_neg2(uint64_t g2) {
+  const float L2E = 1.44269502f;           // fl32(log2 e)
+  const float L2E_LO = 1.925963e-8f;       // log2 e - L2E
+  const uint64_t am = mul2(g2, dup2(L2E));                   // fl(g L2E)
+  const uint64_t r = fma2(g2, dup2(-L2E), am);               // -(g L2E - am), exact
+  const uint64_t lo = fma2(g2, dup2(-L2E_LO), r);
+  float a0, a1;
+  up2(am, a0, a1);
+  const uint64_t e = pk2(ex2_approx(-a0), ex2_approx(-a1));
+  return fma2(e, mul2(lo, dup2(0.693147182f)), e);
+}
+
+// Fast silu(g) * u of a pair: g * (1 / (1 + e^-g)) * u with exp_neg2
+// (<= 2^-22.2), one rounding of 1 + e, rcp.approx (<= 2^-23.3) and two
+// multiplications: relative error <= 2^-20.6 while nothing is tiny and the
+// gate is >= -85 (within the fast exp's range).
+__device__ __forceinline__ uint64_t silu_p2(uint64_t g2, uint64_t u2) {
+  const uint64_t dd = add2(dup2(1.0f), exp_neg2(g2));
+  float d0, d1;
+  up2(dd, d0, d1);
+  return mul2(mul2(g2, pk2(rcp_approx(d0), rcp_approx(d1))), u2);
+}
+
+// bf16 rounding of the low bracket end of a pair; `d` collects its XOR with
+// the high end; `bad` is set for tiny values and gates below -85.
+__device__ __forceinline__ uint32_t silu_pair(uint32_t gw, uint32_t uw, uint32_t& d, bool& bad) {
+  const uint64_t g2 = bf2_to_f2(gw);
+  const uint64_t p = silu_p2(g2, bf2_to_f2(uw));
+  const uint32_t na = f2_to_bf2_rn(mul2(p, dup2(kSiluLo)));
+  d |= na ^ f2_to_bf2_rn(mul2(p, dup2(kSiluHi)));
+  float p0, p1, g0, g1;
+  up2(p, p0, p1);
+  up2(g2, g0, g1);
+  bad |= fminf(fabsf(p0), fabsf(p1)) < kTiny || fminf(g0, g1) < -85.0f;
+  return na;
+}
+
+// Exact bf16(silu(g) * u) of a pair (out of line).
+__device__ __noinline__ uint32_t silu_pair_f64(uint32_t gw, uint32_t uw) {
+  uint32_t out = 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const double g = bf16_bits_to_f32((gw >> (16 * h)) & 0xFFFFu);
+    const double u = bf16_bits_to_f32((uw >> (16 * h)) & 0xFFFFu);
+    out |= f64_to_bf16_bits_rn(g / (1.0 + exp(-g)) * u) << (16 * h);
+  }
+  return out;
+}
+
+// Cold path of a flagged SiLU chunk: each element whose fast value is not
+// proven is recomputed exactly.  A zero gate or up value makes the fast
+// value an exact (signed) zero, so those tiny results are kept.
+__device__ __noinline__ uint4 silu_chunk_fix(const uint4 g, const uint4 u, uint4 y) {
+  const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, uw[4] = {u.x, u.y, u.z, u.w};
+  uint32_t yw[4] = {y.x, y.y, y.z, y.w};
+  for (int k = 0; k < 4; ++k) {
+    const uint64_t g2 = bf2_to_f2(gw[k]), u2 = bf2_to_f2(uw[k]);
+    const uint64_t p = silu_p2(g2, u2);
+    const uint32_t open = f2_to_bf2_rn(mul2(p, dup2(kSiluLo))) ^ f2_to_bf2_rn(mul2(p, dup2(kSiluHi)));
+    float pf[2], gf[2], uf[2];
+    up2(p, pf[0], pf[1]);
+    up2(g2, gf[0], gf[1]);
+    up2(u2, uf[0], uf[1]);
+    bool need = open != 0;
+    for (int h = 0; h < 2; ++h)
+      need |= gf[h] < -85.0f || (fabsf(pf[h]) < kTiny && gf[h] != 0.0f && uf[h] != 0.0f);
+    if (need) yw[k] = silu_pair_f64(gw[k], uw[k]);
+  }
+  return make_uint4(yw[0], yw[1], yw[2], yw[3]);
+}
+
+// ---------------------------------------------------------------------------
+// Kernels
 
 __device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
   uint4 v;
@@ -320,13 +415,13 @@ struct SmemRow {
 };
 
 // Quantize one row with a team of T threads (T a multiple of 32, CH chunks
-// of 8 elements per thread).  `release()` is called once the row's input has
-// been read into registers.
+// of 8 elements per thread; chunk c of the row belongs to thread c mod T, so
+// every warp access is 512 contiguous bytes).  `release()` is called once the
+// row's input has been read into registers.
 template <int OP, bool PER_TOKEN, int CH, typename Src, typename Release>
 __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, const Src& src,
                                             int tid, int T, int bar_id, double* red_d,
                                             float* red_f, Release release) {
-  static_assert(CH * 4 <= 32, "one mask bit per bf16 pair");
   const int64_t nchunks = p.L >> 3;
   uint4 y[CH];
   bool valid[CH];
@@ -335,13 +430,12 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
   auto off = [&](int i) { return (tid + static_cast<int64_t>(i) * T) * 8; };
 
   // Hot loops compute every value on the fast path and only flag the rare
-  // pairs / chunks whose rounding the fast path cannot decide; the exact
+  // chunks with a pair whose rounding the fast path cannot decide; the exact
   // recomputation of those runs afterwards, outside the hot loops.
-  uint32_t fix = 0;  // bit 4i + j: pair j of chunk i needs the exact path
+  uint32_t fix = 0;  // bit i: chunk i has a pair to recompute exactly
   if constexpr (OP == OP_PLAIN) {
 #pragma unroll
-    for (int i = 0; i < CH; ++i)
-      if (valid[i]) y[i] = src.ld(off(i));
+    for (int i = 0; i < CH; ++i) y[i] = valid[i] ? src.ld(off(i)) : make_uint4(0, 0, 0, 0);
     release();
   } else if constexpr (OP == OP_SILU) {
     // gate and up chunks are read in batches of SB chunks to bound registers.
@@ -359,148 +453,93 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
 #pragma unroll
       for (int i = 0; i < SB; ++i) {
         if (valid[i0 + i]) {
-          const uint32_t gw[4] = {g[i].x, g[i].y, g[i].z, g[i].w};
-          const uint32_t uw[4] = {u[i].x, u[i].y, u[i].z, u[i].w};
-          uint32_t o[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            bool bad;
-            o[j] = silu_pair_fast(gw[j], uw[j], bad);
-            fix |= static_cast<uint32_t>(bad) << (4 * (i0 + i) + j);
-          }
-          y[i0 + i] = make_uint4(o[0], o[1], o[2], o[3]);
+          uint32_t d = 0;
+          bool bad = false;
+          y[i0 + i].x = silu_pair(g[i].x, u[i].x, d, bad);
+          y[i0 + i].y = silu_pair(g[i].y, u[i].y, d, bad);
+          y[i0 + i].z = silu_pair(g[i].z, u[i].z, d, bad);
+          y[i0 + i].w = silu_pair(g[i].w, u[i].w, d, bad);
+          fix |= static_cast<uint32_t>(d != 0 || bad) << (i0 + i);
+        } else {
+          y[i0 + i] = make_uint4(0, 0, 0, 0);
         }
       }
     }
-    if (fix) {  // rare: re-read the flagged chunks and recompute their pairs exactly
+    if (fix) {  // rare: re-read the flagged chunks and recompute them exactly
 #pragma unroll
-      for (int i = 0; i < CH; ++i) {
-        if ((fix >> (4 * i)) & 0xFu) {
-          const uint4 g = src.ld(off(i)), u = src.ld(p.L + off(i));
-          uint32_t* yw = reinterpret_cast<uint32_t*>(&y[i]);
-          const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
-          const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if ((fix >> (4 * i + j)) & 1u) yw[j] = silu_pair_f64(gw[j], uw[j]);
-        }
-      }
+      for (int i = 0; i < CH; ++i)
+        if ((fix >> i) & 1u) y[i] = silu_chunk_fix(src.ld(off(i)), src.ld(p.L + off(i)), y[i]);
     }
     release();
   } else {  // OP_RMS
     uint4 xv[CH];
 #pragma unroll
-    for (int i = 0; i < CH; ++i)
-      if (valid[i]) xv[i] = src.ld(off(i));
+    for (int i = 0; i < CH; ++i) xv[i] = valid[i] ? src.ld(off(i)) : make_uint4(0, 0, 0, 0);
     release();
-    // Sum of squares: squares of bf16 values are exact in fp32; they are
-    // accumulated with paired TwoSum (Knuth, TAOCP vol. 2, 4.2.2), a running
-    // sum plus the exact error of every addition, then combined in fp64.
-    uint64_t sum = pk2(0.0f, 0.0f), comp = pk2(0.0f, 0.0f);
+    // Sum of squares in fp64: squares of bf16 values are exact there (16
+    // significant bits, exponents far inside the range).
+    double a0 = 0.0, a1 = 0.0;
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
-      if (valid[i]) {
-        const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+      const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint64_t x2 = bf2_to_f2(xw[j]);
-          const uint64_t v = mul2(x2, x2);
-          const uint64_t s1 = add2(sum, v);
-          const uint64_t bp = sub2(s1, sum);
-          comp = add2(comp, add2(sub2(sum, sub2(s1, bp)), sub2(v, bp)));
-          sum = s1;
-        }
+      for (int k = 0; k < 4; ++k) {
+        const double lo = __uint_as_float(xw[k] << 16), hi = __uint_as_float(xw[k] & 0xFFFF0000u);
+        a0 = __fma_rn(lo, lo, a0);
+        a1 = __fma_rn(hi, hi, a1);
       }
     }
-    float s0, s1f, c0, c1;
-    up2(sum, s0, s1f);
-    up2(comp, c0, c1);
-    double ss = (static_cast<double>(s0) + static_cast<double>(s1f)) +
-                (static_cast<double>(c0) + static_cast<double>(c1));
-    ss = team_reduce(ss, SumOp(), red_d, tid, T, bar_id);
-    // Fast path: r32 = rsqrtf(fl32(mean + eps)): <= 2 ulp + half an ulp from
-    // the conversion, < 2^-21.9 relative; the fp64 r is computed only by the
-    // exact path.
-    const float r32 = rsqrtf(static_cast<float>(ss / static_cast<double>(p.L) + static_cast<double>(p.eps)));
+    const double ss = team_reduce(a0 + a1, SumOp(), red_d, tid, T, bar_id);
+    float r_lo, r_hi;
+    rms_bracket(__fma_rn(ss, 1.0 / static_cast<double>(p.L), static_cast<double>(p.eps)), r_lo, r_hi);
+    const uint64_t rlo2 = dup2(r_lo), rhi2 = dup2(r_hi);
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
       if (valid[i]) {
-        const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
         const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.w + off(i)));
-        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          bool bad;
-          o[j] = bf2_mul(rms_n_fast(xw[j], r32, bad), ww[j]);
-          fix |= static_cast<uint32_t>(bad) << (4 * i + j);
-        }
-        y[i] = make_uint4(o[0], o[1], o[2], o[3]);
+        uint32_t d = 0;
+        y[i].x = bf2_mul(rms_n_pair(xv[i].x, rlo2, rhi2, d), wv.x);
+        y[i].y = bf2_mul(rms_n_pair(xv[i].y, rlo2, rhi2, d), wv.y);
+        y[i].z = bf2_mul(rms_n_pair(xv[i].z, rlo2, rhi2, d), wv.z);
+        y[i].w = bf2_mul(rms_n_pair(xv[i].w, rlo2, rhi2, d), wv.w);
+        fix |= static_cast<uint32_t>(d != 0) << i;
+      } else {
+        y[i] = make_uint4(0, 0, 0, 0);
       }
     }
-    if (fix) {  // rare: exact bf16(x * r) for the flagged pairs, then y again
+    if (fix) {  // rare: exact bf16(x r) for the pairs whose bracket is open
 #pragma unroll
-      for (int i = 0; i < CH; ++i) {
-        if ((fix >> (4 * i)) & 0xFu) {
-          const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
-          const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.w + off(i)));
-          const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-          uint32_t* yw = reinterpret_cast<uint32_t*>(&y[i]);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if ((fix >> (4 * i + j)) & 1u) yw[j] = bf2_mul(rms_pair_f64(xw[j], ss, p.L, p.eps), ww[j]);
-        }
-      }
+      for (int i = 0; i < CH; ++i)
+        if ((fix >> i) & 1u)
+          y[i] = rms_chunk_fix(xv[i], __ldg(reinterpret_cast<const uint4*>(p.w + off(i))), y[i], rlo2,
+                               rhi2, ss, p.L, p.eps);
     }
   }
 
-  // Codes are stored as soon as they are made; a flagged chunk is stored
-  // again, from IEEE division, after the loop.
   uint8_t* qr = p.q + row * p.ldq;
-  uint32_t qfix = 0;  // bit i: chunk i needs IEEE division
   if constexpr (PER_TOKEN) {
-    float amax = 0.0f;
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int i = 0; i < CH; ++i) m2 = chunk_absmax2(y[i], m2);
+    const float amax = team_reduce(absmax2_to_f32(m2), MaxOp(), red_f, tid, T, bar_id);
+    const QScale qs = make_qscale(amax, p.ue8m0);
 #pragma unroll
     for (int i = 0; i < CH; ++i)
-      if (valid[i]) amax = fmaxf(amax, chunk_amax(y[i]));
-    amax = team_reduce(amax, MaxOp(), red_f, tid, T, bar_id);
-    const float s = group_scale(amax, p.ue8m0);
-    const float rcp = rcp_approx(s);
-#pragma unroll
-    for (int i = 0; i < CH; ++i) {
-      if (valid[i]) {
-        bool bad;
-        *reinterpret_cast<uint2*>(qr + off(i)) = quantize_chunk_fast(y[i], rcp, bad);
-        qfix |= static_cast<uint32_t>(bad) << i;
-      }
-    }
-    if (tid == 0) p.s[row * p.s_sm] = s;
-    if (qfix) {
-#pragma unroll
-      for (int i = 0; i < CH; ++i)
-        if ((qfix >> i) & 1u) *reinterpret_cast<uint2*>(qr + off(i)) = quantize_chunk_ieee(y[i], s);
-    }
+      if (valid[i]) *reinterpret_cast<uint2*>(qr + off(i)) = quant_chunk(y[i], qs);
+    if (tid == 0) p.s[row * p.s_sm] = qs.s;
   } else {
     // 128-wide groups: the 16 threads tid & ~15 .. +15 own one group per i
     // (T is a multiple of 32 and L of 128, so whole half-warps are valid or not).
-    float sc[CH];
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
-      float a = valid[i] ? chunk_amax(y[i]) : 0.0f;
+      float a = absmax2_to_f32(chunk_absmax2(y[i], 0u));
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
-      sc[i] = group_scale(a, p.ue8m0);
       if (valid[i]) {
-        bool bad;
-        *reinterpret_cast<uint2*>(qr + off(i)) = quantize_chunk_fast(y[i], rcp_approx(sc[i]), bad);
-        qfix |= static_cast<uint32_t>(bad) << i;
-        if ((tid & 15) == 0) p.s[row * p.s_sm + (off(i) >> 7) * p.s_sg] = sc[i];
+        const QScale qs = make_qscale(a, p.ue8m0);
+        *reinterpret_cast<uint2*>(qr + off(i)) = quant_chunk(y[i], qs);
+        if ((tid & 15) == 0) p.s[row * p.s_sm + (off(i) >> 7) * p.s_sg] = qs.s;
       }
-    }
-    if (qfix) {
-#pragma unroll
-      for (int i = 0; i < CH; ++i)
-        if ((qfix >> i) & 1u) *reinterpret_cast<uint2*>(qr + off(i)) = quantize_chunk_ieee(y[i], sc[i]);
     }
   }
 }

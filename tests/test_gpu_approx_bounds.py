@@ -1,11 +1,13 @@
-"""The error bounds the quant kernels' fast paths rest on, measured on this GPU.
+"""The arithmetic facts the quant kernels' fast paths rest on, measured on this GPU.
 
-The SiLU fast path uses ex2.approx / rcp.approx and the RMSNorm fast path
-rsqrtf; their rounding brackets (+-2^-19, +-2^-20) are sized from these
-worst-case relative errors: if a bound grew, a fast result could round
-differently from the exact value unnoticed.
-tests/cuda/approx_bounds.cu checks every fp32 input of the ranges used
-against fp64 and reports the maxima.
+The SiLU fast path uses ex2.approx / rcp.approx, its rounding bracket
+(+-2^-19) sized from their worst-case relative errors; the RMSNorm path
+refines rsqrtf by one Newton step, whose error (1.5 e^2) must stay far below
+the 2^-30 margin of its bracket.  tests/cuda/approx_bounds.cu checks every
+fp32 input of the ranges used against fp64 and reports the maxima.
+The codes come from the IEEE quotient y / s obtained by Markstein's division
+step; tests/cuda/quotient_exact.cu checks that against IEEE division for
+every bf16 amax and every bf16 y the kernels can meet.
 """
 import os
 import shutil
@@ -31,6 +33,17 @@ def test_hardware_approximation_bounds(tmp_path):
     # the SiLU fast value's total relative error must stay inside its bracket
     total = expf + 2.0 ** -24 + rcp + 2 * 2.0 ** -24
     assert total + 2.0 ** -24 < 2.0 ** -19
-    # the RMSNorm fast value: rsqrtf + half an ulp (fp32 argument) + one product,
-    # inside its +-2^-20 bracket
-    assert rsq + 2.0 ** -25 + 2.0 ** -24 + 2.0 ** -24 < 2.0 ** -20
+    # the RMSNorm r: rsqrtf of the fp32-rounded argument (half an ulp more),
+    # one Newton step in fp64 squares the error: far inside the 2^-30 margin
+    e = rsq + 2.0 ** -25
+    assert 1.5 * e * e + 2.0 ** -50 < 2.0 ** -30
+
+
+def test_markstein_quotient_equals_ieee_division(tmp_path):
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    exe = str(tmp_path / "quotient_exact")
+    subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-o", exe,
+                    os.path.join(HERE, "cuda", "quotient_exact.cu")], check=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True, timeout=300).stdout
+    bad_q, bad_c = (int(v) for v in out.split())
+    assert (bad_q, bad_c) == (0, 0)
