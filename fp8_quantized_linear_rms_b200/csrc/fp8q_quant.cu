@@ -285,9 +285,9 @@ __device__ __forceinline__ void rms_bracket(double m, float& r_lo, float& r_hi) 
 // ---------------------------------------------------------------------------
 // SiLU * mul
 
-// Bracket of the fast SiLU*mul value p (relative error <= 2^-20.6, below):
-// p (1 -+ 2^-19), each end one more rounding.
-constexpr float kSiluLo = 1.0f - 0x1p-19f, kSiluHi = 1.0f + 0x1p-19f;
+// Bracket of the fast SiLU*mul value p (relative error <= 2^-21.0, below):
+// p (1 -+ 2^-20.5), each end one more rounding.
+constexpr float kSiluLo = 1.0f - 0x1.6a09e6p-21f, kSiluHi = 1.0f + 0x1.6a09e6p-21f;
 constexpr float kTiny = 0x1p-100f;  // below this fp32 products may lose relative precision
 
 // e^-g for a pair, |g| <= 85: 2^(-g log2 e) with the exponent split exactly
@@ -308,14 +308,20 @@ __device__ __forceinline__ uint64_t exp_neg2(uint64_t g2) {
 }
 
 // Fast silu(g) * u of a pair: g * (1 / (1 + e^-g)) * u with exp_neg2
-// (<= 2^-22.2), one rounding of 1 + e, rcp.approx (<= 2^-23.3) and two
-// multiplications: relative error <= 2^-20.6 while nothing is tiny and the
-// gate is >= -85 (within the fast exp's range).
+// (<= 2^-22.2), one rounding of 1 + e, the Newton-refined reciprocal
+// (<= 2^-23.9) and two multiplications: relative error <= 2^-21.0 while
+// nothing is tiny and the gate is >= -85 (within the fast exp's range).
 __device__ __forceinline__ uint64_t silu_p2(uint64_t g2, uint64_t u2) {
   const uint64_t dd = add2(dup2(1.0f), exp_neg2(g2));
   float d0, d1;
   up2(dd, d0, d1);
-  return mul2(mul2(g2, pk2(rcp_approx(d0), rcp_approx(d1))), u2);
+  // -1/d by rcp.approx of -d, then one Newton step: h = 1 - d r0,
+  // -r1 = -r0 (1 + h); the result is within 2^-23.9 of 1/d.
+  const uint64_t nr0 = pk2(rcp_approx(-d0), rcp_approx(-d1));
+  const uint64_t h = fma2(dd, nr0, dup2(1.0f));
+  const uint64_t nr1 = fma2(nr0, h, nr0);
+  // (-g)(-r1) u: negate g by its sign bits
+  return mul2(mul2(g2 ^ 0x8000000080000000ull, nr1), u2);
 }
 
 // bf16 rounding of the low bracket end of a pair; `d` collects its XOR with
@@ -546,8 +552,11 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
 
 // Register kernel: one CTA per row, the row loaded straight into registers.
 // Used for rows too long for the shared-memory ring below.
-template <int OP, bool PER_TOKEN, int CH>
-__global__ void __launch_bounds__(kMaxThreads, (CH <= 4 ? 2 : 1)) quant_rows_kernel(const QuantParams p) {
+// MAXT/MINB set the register budget (measured): 64 registers for 4 chunks
+// per thread (plain and RMSNorm: the occupancy beats the few spills), 80 for
+// SiLU rows of up to 384 threads, 128 for 8 chunks per thread.
+template <int OP, bool PER_TOKEN, int CH, int MAXT, int MINB>
+__global__ void __launch_bounds__(MAXT, MINB) quant_rows_kernel(const QuantParams p) {
   __shared__ double red_d[32];
   __shared__ float red_f[32];
   for (int64_t row = blockIdx.x; row < p.M; row += gridDim.x)
@@ -702,11 +711,17 @@ fp8q_status launch_quant(const QuantParams& p, cudaStream_t stream) {
   const int64_t grid = p.M < (1LL << 30) ? p.M : (1LL << 30);
   const dim3 g(static_cast<unsigned>(grid)), b(T);
   if (ch == 8) {
-    if (per_token) quant_rows_kernel<OP, true, 8><<<g, b, 0, stream>>>(p);
-    else quant_rows_kernel<OP, false, 8><<<g, b, 0, stream>>>(p);
+    if (per_token) quant_rows_kernel<OP, true, 8, 512, 1><<<g, b, 0, stream>>>(p);
+    else quant_rows_kernel<OP, false, 8, 512, 1><<<g, b, 0, stream>>>(p);
+  } else if (OP == OP_SILU && T <= 256) {
+    if (per_token) quant_rows_kernel<OP, true, 4, 256, 3><<<g, b, 0, stream>>>(p);
+    else quant_rows_kernel<OP, false, 4, 256, 3><<<g, b, 0, stream>>>(p);
+  } else if (OP == OP_SILU && T <= 384) {
+    if (per_token) quant_rows_kernel<OP, true, 4, 384, 2><<<g, b, 0, stream>>>(p);
+    else quant_rows_kernel<OP, false, 4, 384, 2><<<g, b, 0, stream>>>(p);
   } else {
-    if (per_token) quant_rows_kernel<OP, true, 4><<<g, b, 0, stream>>>(p);
-    else quant_rows_kernel<OP, false, 4><<<g, b, 0, stream>>>(p);
+    if (per_token) quant_rows_kernel<OP, true, 4, 512, 2><<<g, b, 0, stream>>>(p);
+    else quant_rows_kernel<OP, false, 4, 512, 2><<<g, b, 0, stream>>>(p);
   }
   return launch_status();
 }

@@ -13,6 +13,7 @@ import os
 import shutil
 import subprocess
 
+import numpy as np
 import pytest
 
 pytestmark = pytest.mark.gpu
@@ -25,14 +26,21 @@ def test_hardware_approximation_bounds(tmp_path):
     subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-o", exe,
                     os.path.join(HERE, "cuda", "approx_bounds.cu")], check=True)
     out = subprocess.run([exe], check=True, capture_output=True, text=True, timeout=300).stdout
-    ex2, rcp, expf, rsq = (float(v) for v in out.split())
-    print(f"ex2.approx {ex2:.3e}, rcp.approx {rcp:.3e}, exp_fast {expf:.3e}, rsqrtf {rsq:.3e}")
+    ex2, rcp, expf, rsq, rcp_n = (float(v) for v in out.split())
+    print(f"ex2.approx {ex2:.3e}, rcp.approx {rcp:.3e}, exp_fast {expf:.3e}, rsqrtf {rsq:.3e}, "
+          f"Newton reciprocal {rcp_n:.3e}")
     assert ex2 <= 2.0 ** -22.5
     assert rcp <= 2.0 ** -23.0
     assert expf <= 2.0 ** -22.0
-    # the SiLU fast value's total relative error must stay inside its bracket
-    total = expf + 2.0 ** -24 + rcp + 2 * 2.0 ** -24
-    assert total + 2.0 ** -24 < 2.0 ** -19
+    assert rcp_n <= 2.0 ** -23.9
+    # the SiLU fast value p: exp, the rounding of 1 + e, the reciprocal and two
+    # products; its bracket ends p (1 -+ 2^-20.5), each rounded once more to
+    # fp32, must still enclose the real value
+    total = expf + 2.0 ** -24 + rcp_n + 2 * 2.0 ** -24
+    lo = float(np.float32(1.0 - 2.0 ** -20.5))
+    hi = float(np.float32(1.0 + 2.0 ** -20.5))
+    assert lo * (1 + total) * (1 + 2.0 ** -24) < 1.0
+    assert hi * (1 - total) * (1 - 2.0 ** -24) > 1.0
     # the RMSNorm r: rsqrtf of the fp32-rounded argument (half an ulp more),
     # one Newton step in fp64 squares the error: far inside the 2^-30 margin
     e = rsq + 2.0 ** -25
