@@ -39,11 +39,13 @@ _INT = ctypes.c_int
 
 
 class GemmVariant(ctypes.Structure):
-    """fp8q_gemm_variant: swap_ab, split_k, block_n."""
-    _fields_ = [("swap_ab", ctypes.c_int), ("split_k", ctypes.c_int), ("block_n", ctypes.c_int)]
+    """fp8q_gemm_variant: swap_ab, split_k, block_n, cta_pair."""
+    _fields_ = [("swap_ab", ctypes.c_int), ("split_k", ctypes.c_int), ("block_n", ctypes.c_int),
+                ("cta_pair", ctypes.c_int)]
 
     def as_dict(self):
-        return {"swap_ab": self.swap_ab, "split_k": self.split_k, "block_n": self.block_n}
+        return {"swap_ab": self.swap_ab, "split_k": self.split_k, "block_n": self.block_n,
+                "cta_pair": self.cta_pair}
 
 
 _SIGS = {
@@ -285,12 +287,13 @@ def fp8q_select_gemm_variant(M: int, N: int, K: int, blockwise: bool) -> dict:
     return v.as_dict()
 
 
-def fp8q_force_gemm_variant(swap_ab: int | None = None, split_k: int = 1, block_n: int = 128):
+def fp8q_force_gemm_variant(swap_ab: int | None = None, split_k: int = 1, block_n: int = 128,
+                            cta_pair: int = 0):
     """Force a GEMM variant for the following calls (testing/tuning); no args = automatic."""
     if swap_ab is None:
         _check("fp8q_force_gemm_variant", lib.fp8q_force_gemm_variant(None))
         return
-    v = GemmVariant(int(swap_ab), int(split_k), int(block_n))
+    v = GemmVariant(int(swap_ab), int(split_k), int(block_n), int(cta_pair))
     _check("fp8q_force_gemm_variant", lib.fp8q_force_gemm_variant(ctypes.byref(v)))
 
 

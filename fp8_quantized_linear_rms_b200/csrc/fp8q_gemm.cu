@@ -75,7 +75,9 @@ struct Cfg {
   static constexpr int EPI_WARPS = (BW && BN >= 256) ? 16 : ((BW && BN >= 128) ? 8 : 4);
   static constexpr int COL_GROUPS = EPI_WARPS / 4;        // column slices per TMEM lane quadrant
   static constexpr int CPT = BN / COL_GROUPS;              // columns per epilogue thread
-  static constexpr int CHUNK = (EPI_WARPS == 16 || CPT < 32) ? 16 : 32;  // columns per tcgen05.ld
+  // Columns per tcgen05.ld.  The 16-warp variant holds 64 fp32 accumulators
+  // per thread in a 96-register budget, so it reads 8 columns at a time.
+  static constexpr int CHUNK = EPI_WARPS == 16 ? 8 : (CPT < 32 ? 16 : 32);
   static constexpr int NBUF = (BW && BN < 256) ? 4 : 2;    // TMEM accumulator buffers
   static constexpr int TMEM_NEED = NBUF * BN;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
@@ -85,7 +87,7 @@ struct Cfg {
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
   static_assert(STAGES >= 2, "pipeline too shallow");
   static_assert(TMEM_NEED <= 512, "accumulators exceed TMEM");
-  static_assert(CPT % CHUNK == 0 && (CHUNK == 16 || CHUNK == 32), "chunking");
+  static_assert(CPT % CHUNK == 0 && (CHUNK == 8 || CHUNK == 16 || CHUNK == 32), "chunking");
   static_assert(B_BYTES % 1024 == 0, "B tiles must stay 1024-byte aligned");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
@@ -439,14 +441,12 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
 #pragma unroll
         for (int j = 0; j < NCH; ++j) {
           const int c = col0 + j * C::CHUNK;
+          uint32_t r[C::CHUNK];
+          tmem_ld_waited<C::CHUNK>(tmem_base + lane_addr + buf * BN + c, r);
           float v[C::CHUNK];
-          const uint32_t taddr = tmem_base + lane_addr + buf * BN + c;
-          if (C::CHUNK == 32) tmem_ld_32x32b_x32(taddr, v);
-          else tmem_ld_32x32b_x16(taddr, v);
-          tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < C::CHUNK; ++i)
-            v[i] = v[i] * (srow * __shfl_sync(0xFFFFFFFFu, colsc[j], i));
+            v[i] = __uint_as_float(r[i]) * (srow * __shfl_sync(0xFFFFFFFFu, colsc[j], i));
           if (g.ncontrib == 1) emit(c, v);
           else stash(c, v);
         }
@@ -457,75 +457,90 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
         if (g.ncontrib > 1) finish_split();
       } else {
         // -------- blockwise scales: promote each K-block partial into registers.
-        // The scales of K block kb+1 are loaded while block kb is processed, so
-        // their latency stays off the per-block critical path.  Swap-AB: the
-        // scale varies per column (token); lane l holds that of column c + l.
+        // The scales of the next SD K blocks are kept in flight in a register
+        // ring (stage 0 = the block being promoted), so the global-load
+        // latency of a block's scales overlaps the promotion of the blocks
+        // before it.  Swap-AB: the scale varies per column (token); lane l
+        // holds that of column c + l of every chunk.
         constexpr int NCH = C::CPT / C::CHUNK;
+        constexpr int SD = C::EPI_WARPS == 16 ? 1 : 4;
         uint64_t acc[C::CPT / 2];                      // fp32 pairs, columns 2i, 2i+1
 #pragma unroll
         for (int i = 0; i < C::CPT / 2; ++i) acc[i] = 0ull;
-        // Weight block row of this thread's columns: the whole tile (Swap-AB) or
-        // this warp's 128-column slice (a slice never straddles a block row).
+        // Scale offsets (elements; every scale array is far below 2^31 of
+        // them) advance one K block per load.  A row or column outside the
+        // problem reads the scales of row/column 0 instead: its output is never
+        // written.  Weight block row: the whole tile (Swap-AB) or this warp's
+        // 128-column slice (a slice never straddles a block row).
         const int nb = SWAP ? ta : (tb * BN + col0) / 128;
         const bool slice_valid = SWAP || (tb * BN + col0) < p.N;
-        // Scales of the next SD K blocks are kept in flight in a register ring
-        // (stage 0 = the block being promoted), so the global-load latency of
-        // a block's scales overlaps the promotion of the SD-1 blocks before it.
-        constexpr int SD = 4;
-        float srow_q[SD], colsc_q[SD][NCH];
-        auto load_scales = [&](int kb, float& srow_o, float* colsc_o) {
-          const bool in = kb < kb1;
-          const float sbk = (in && slice_valid) ? __ldg(p.sb + nb * p.sb_snb + kb * p.sb_skb) : 0.0f;
-          if (!SWAP) {
-            srow_o = (in && a_valid && slice_valid) ? __ldg(p.sa + a_idx * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
-          } else {
-            srow_o = 0.0f;
+        int sb_o = static_cast<int>((slice_valid ? nb : 0) * p.sb_snb + kb0 * p.sb_skb);
+        int sa_o[SWAP ? NCH : 1];
+        if (!SWAP) {
+          sa_o[0] = static_cast<int>((a_valid ? a_idx : 0) * p.sa_sm + kb0 * p.sa_skb);
+        } else {
 #pragma unroll
-            for (int j = 0; j < NCH; ++j) {
-              const int m = b_base + col0 + j * C::CHUNK + lane;
-              colsc_o[j] = (in && lane < C::CHUNK && m < p.M)
-                               ? __ldg(p.sa + m * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
-            }
+          for (int j = 0; j < NCH; ++j) {
+            const int m = b_base + col0 + j * C::CHUNK + lane;
+            sa_o[j] = static_cast<int>((m < p.M ? m : 0) * p.sa_sm + kb0 * p.sa_skb);
           }
+        }
+        float sq[SD][SWAP ? NCH : 1];                  // non-swap: sa * sb of the row
+        int kl = kb0;                                  // next K block to load scales of
+        auto load_scales = [&](float* out) {
+          const bool in = kl < kb1;
+          const float sbk = in ? __ldg(p.sb + sb_o) : 0.0f;
+#pragma unroll
+          for (int j = 0; j < (SWAP ? NCH : 1); ++j) {
+            out[j] = in ? __ldg(p.sa + sa_o[j]) * sbk : 0.0f;
+            sa_o[j] += static_cast<int>(p.sa_skb);
+          }
+          sb_o += static_cast<int>(p.sb_skb);
+          ++kl;
         };
 #pragma unroll
-        for (int q = 0; q < SD; ++q) load_scales(kb0 + q, srow_q[q], colsc_q[q]);
+        for (int q = 0; q < SD; ++q) load_scales(sq[q]);
+        int pb = pc % NB;
+        uint32_t ph = (pc / NB) & 1;
         for (int kb = kb0; kb < kb1; ++kb) {
-          const int pb = pc % NB;
-          const uint64_t srow2 = pair_f32(srow_q[0], srow_q[0]);
-          float colsc[NCH];
+          float sc0[SWAP ? NCH : 1];
 #pragma unroll
-          for (int j = 0; j < NCH; ++j) colsc[j] = SWAP ? colsc_q[0][j] : 0.0f;
+          for (int j = 0; j < (SWAP ? NCH : 1); ++j) sc0[j] = sq[0][j];
 #pragma unroll
-          for (int q = 0; q + 1 < SD; ++q) {
-            srow_q[q] = srow_q[q + 1];
+          for (int q = 0; q + 1 < SD; ++q)
 #pragma unroll
-            for (int j = 0; j < NCH; ++j) colsc_q[q][j] = colsc_q[q + 1][j];
-          }
-          load_scales(kb + SD, srow_q[SD - 1], colsc_q[SD - 1]);
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[pb], (pc / NB) & 1, abort_flag, p.status))) {
+            for (int j = 0; j < (SWAP ? NCH : 1); ++j) sq[q][j] = sq[q + 1][j];
+          load_scales(sq[SD - 1]);
+          const uint64_t srow2 = pair_f32(sc0[0], sc0[0]);
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[pb], ph, abort_flag, p.status))) {
             ok = false;
             break;
           }
           tc_fence_after();
+          // One chunk per load+wait; the buffer is handed back to the MMA as
+          // soon as the last chunk has landed, before its FMAs.
+          const uint32_t tbuf = tmem_base + lane_addr + pb * BN + col0;
 #pragma unroll
           for (int j = 0; j < NCH; ++j) {
             uint32_t r[C::CHUNK];
-            const uint32_t taddr = tmem_base + lane_addr + pb * BN + col0 + j * C::CHUNK;
-            if (C::CHUNK == 32) tmem_ld_32x32b_x32_raw(taddr, r);
-            else tmem_ld_32x32b_x16_raw(taddr, r);
-            tmem_ld_wait();
+            tmem_ld_waited<C::CHUNK>(tbuf + j * C::CHUNK, r);
+            if (j == NCH - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[pb]);
+            }
 #pragma unroll
             for (int i = 0; i < C::CHUNK; i += 2) {
-              const uint64_t sc = SWAP ? pair_f32(__shfl_sync(0xFFFFFFFFu, colsc[j], i),
-                                                  __shfl_sync(0xFFFFFFFFu, colsc[j], i + 1))
+              const uint64_t sc = SWAP ? pair_f32(__shfl_sync(0xFFFFFFFFu, sc0[SWAP ? j : 0], i),
+                                                  __shfl_sync(0xFFFFFFFFu, sc0[SWAP ? j : 0], i + 1))
                                        : srow2;
               ffma2_acc(acc[(j * C::CHUNK + i) / 2], r[i], r[i + 1], sc);
             }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[pb]);
+          if (++pb == NB) {
+            pb = 0;
+            ph ^= 1u;
+          }
           ++pc;
         }
         if (!ok) break;
@@ -546,6 +561,295 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ CTA pairs
+// Pair kernel: a cluster of two CTAs (on two SMs) computes one 256 x BN tile
+// with tcgen05 .cta_group::2 MMAs.  CTA rank r loads rows [128 r, 128 r + 128)
+// of the A tile and rows [BN/2 r, BN/2 r + BN/2) of the B tile into its own
+// shared memory, and its TMEM receives rows [128 r, 128 r + 128) of the
+// accumulator; the even CTA issues the MMAs (M = 256, N = BN) and every
+// completion is multicast to both CTAs' mbarriers.  Each SM thus stages half
+// a B tile per K block: a 128-column tile costs it the shared-memory traffic
+// of a 256-column single-CTA tile while TMEM keeps room for four 128-column
+// accumulator buffers -- for the blockwise scheme three K blocks of slack
+// between the MMA and the promotion epilogue instead of one.
+// Both CTAs' TMA loads count their bytes on the even CTA's full barrier (no
+// multicast loads); the epilogue warps of both CTAs release an accumulator
+// buffer on the even CTA's tempty barrier.  A cluster barrier precedes any
+// cross-CTA use of the barriers and the TMEM release.
+template <int BN, bool BW>
+struct Cfg2 {
+  static constexpr int HB = BN / 2;                        // B rows per CTA
+  static constexpr int B_BYTES = HB * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // per CTA
+  static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int NBUF = (512 / BN) > 4 ? 4 : (512 / BN);
+  static constexpr int EPI_WARPS = BW ? (BN >= 256 ? 16 : 8) : 4;
+  static constexpr int COL_GROUPS = EPI_WARPS / 4;
+  static constexpr int CPT = BN / COL_GROUPS;
+  static constexpr int CHUNK = 32;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * NBUF + 1) + 16;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static_assert(NBUF * BN <= 512, "accumulators exceed TMEM");
+  static_assert(CPT % CHUNK == 0, "chunking");
+  static_assert(B_BYTES % 1024 == 0, "B tiles must stay 1024-byte aligned");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+template <int BN, bool BW>
+__global__ void __launch_bounds__(Cfg2<BN, BW>::THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const GemmArgs p) {
+  using C = Cfg2<BN, BW>;
+  constexpr int S = C::STAGES;
+  constexpr int NB = C::NBUF;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * C::B_BYTES);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + NB;
+  uint64_t* drain = tempty + NB;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < NB; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 2 * C::EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int npairs = static_cast<int>(gridDim.x >> 1);
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int u = pair; ok && u < p.units; u += npairs) {
+        const int ta = u % p.tiles_a, tb = u / p.tiles_a;
+        for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+          const int st = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&full[st], 2 * C::STAGE_BYTES);
+          const uint32_t fb = mapa_shared(smem_u32(&full[st]), 0);
+          tma_load_2d_pair(sA + st * A_BYTES, &tmA, fb, kb * BK, ta * (2 * BM) + static_cast<int>(rank) * BM);
+          tma_load_2d_pair(sB + st * C::B_BYTES, &tmB, fb, kb * BK, tb * BN + static_cast<int>(rank) * C::HB);
+        }
+      }
+      if (leader) {
+        // Let the copies of both CTAs land (they count on these barriers)
+        // before the pair can leave (immediate when everything was consumed).
+        const int first = it - S > 0 ? it - S : 0;
+        for (int j = first; j < it; ++j) drain_wait(&full[j % S], (j / S) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(2 * BM, BN);
+      int it = 0, t = 0, pc = 0;
+      bool ok = true;
+      for (int u = pair; ok && u < p.units; u += npairs) {
+        uint32_t d = tmem_base;
+        int buf = 0;
+        if (!BW) {
+          buf = t % NB;
+          if (!mbar_wait(&tempty[buf], ((t / NB) & 1) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          d = tmem_base + buf * BN;
+        }
+        for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+          const int st = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!mbar_wait(&full[st], ph, abort_flag, p.status)) { ok = false; break; }
+          int pb = 0;
+          if (BW) {
+            pb = pc % NB;
+            if (!mbar_wait(&tempty[pb], ((pc / NB) & 1) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+            d = tmem_base + pb * BN;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_kmajor_sw128(sA + st * A_BYTES);
+          const uint64_t bdesc = smem_desc_kmajor_sw128(sB + st * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            const uint32_t acc = BW ? (k > 0) : (kb > 0 || k > 0);
+            mma_f8f6f4_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
+          }
+          mma_commit_pair(&empty[st], 0x3);
+          if (BW) {
+            mma_commit_pair(&tfull[pb], 0x3);
+            ++pc;
+          }
+        }
+        if (!ok) break;
+        if (!BW) {
+          mma_commit_pair(&tfull[buf], 0x3);
+          ++t;
+        }
+      }
+      // Every MMA issued so far, which reads both CTAs' shared memory, has
+      // completed once `drain` flips in both CTAs.
+      mma_commit_pair(drain, 0x3);
+    }
+    if (lane == 0) drain_wait(drain, 0);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int e = warp - 2;
+    const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
+    const int cg = e >> 2;                     // column slice
+    const int row = quad * 32 + lane;          // accumulator row within this CTA's half
+    const int col0 = cg * C::CPT;
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    constexpr int NCH = C::CPT / C::CHUNK;
+    int t = 0, pc = 0;
+    bool ok = true;
+    for (int u = pair; ok && u < p.units; u += npairs) {
+      const int ta = u % p.tiles_a, tb = u / p.tiles_a;
+      const int m = ta * (2 * BM) + static_cast<int>(rank) * BM + row;
+      const bool m_valid = m < p.M;
+      uint16_t* yr = p.y + static_cast<int64_t>(m_valid ? m : 0) * p.ldy;
+      auto emit = [&](int col, const float* v) {
+        if (!m_valid) return;
+#pragma unroll
+        for (int g8 = 0; g8 < C::CHUNK; g8 += 8) {
+          const int n = tb * BN + col + g8;
+          if (n < p.N) {
+            uint4 o;
+            o.x = pack_bf16x2(v[g8 + 0], v[g8 + 1]);
+            o.y = pack_bf16x2(v[g8 + 2], v[g8 + 3]);
+            o.z = pack_bf16x2(v[g8 + 4], v[g8 + 5]);
+            o.w = pack_bf16x2(v[g8 + 6], v[g8 + 7]);
+            *reinterpret_cast<uint4*>(yr + n) = o;
+          }
+        }
+      };
+      if (!BW) {
+        // -------- per-token / per-channel scales: one accumulator per tile
+        const int buf = t % NB;
+        const float srow = m_valid ? __ldg(p.sa + m * p.sa_sm) : 0.0f;
+        float colsc[NCH];
+#pragma unroll
+        for (int j = 0; j < NCH; ++j) {
+          const int n = tb * BN + col0 + j * C::CHUNK + lane;
+          colsc[j] = n < p.N ? __ldg(p.sb + n * p.sb_sn) : 0.0f;
+        }
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[buf], (t / NB) & 1, abort_flag, p.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < NCH; ++j) {
+          uint32_t r[C::CHUNK];
+          tmem_ld_waited<C::CHUNK>(tmem_base + lane_addr + buf * BN + col0 + j * C::CHUNK, r);
+          float v[C::CHUNK];
+#pragma unroll
+          for (int i = 0; i < C::CHUNK; ++i)
+            v[i] = __uint_as_float(r[i]) * (srow * __shfl_sync(0xFFFFFFFFu, colsc[j], i));
+          emit(col0 + j * C::CHUNK, v);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * buf);
+        ++t;
+      } else {
+        // -------- blockwise scales: promote each K-block partial into registers
+        uint64_t acc[C::CPT / 2];
+#pragma unroll
+        for (int i = 0; i < C::CPT / 2; ++i) acc[i] = 0ull;
+        const int nb = (tb * BN + col0) / 128;
+        const bool slice_valid = (tb * BN + col0) < p.N;
+        constexpr int SD = 4;
+        float srow_q[SD];
+        auto load_scale = [&](int kb) {
+          if (kb >= p.kblocks || !slice_valid || !m_valid) return 0.0f;
+          return __ldg(p.sa + m * p.sa_sm + kb * p.sa_skb) * __ldg(p.sb + nb * p.sb_snb + kb * p.sb_skb);
+        };
+#pragma unroll
+        for (int q = 0; q < SD; ++q) srow_q[q] = load_scale(q);
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          const int pb = pc % NB;
+          const uint64_t srow2 = pair_f32(srow_q[0], srow_q[0]);
+#pragma unroll
+          for (int q = 0; q + 1 < SD; ++q) srow_q[q] = srow_q[q + 1];
+          srow_q[SD - 1] = load_scale(kb + SD);
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[pb], (pc / NB) & 1, abort_flag, p.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // All of this warp's columns are read with one wait, the buffer is
+          // handed back, then the partial is scaled into the accumulators.
+          uint32_t r[NCH][C::CHUNK];
+#pragma unroll
+          for (int j = 0; j < NCH; ++j)
+            tmem_ld_32x32b_x32_raw(tmem_base + lane_addr + pb * BN + col0 + j * C::CHUNK, r[j]);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * pb);
+#pragma unroll
+          for (int j = 0; j < NCH; ++j)
+#pragma unroll
+            for (int i = 0; i < C::CHUNK; i += 2)
+              ffma2_acc(acc[(j * C::CHUNK + i) / 2], r[j][i], r[j][i + 1], srow2);
+          ++pc;
+        }
+        if (!ok) break;
+#pragma unroll
+        for (int c = 0; c < C::CPT; c += C::CHUNK) {
+          float v[C::CHUNK];
+#pragma unroll
+          for (int i = 0; i < C::CHUNK; i += 2) unpair_f32(acc[(c + i) / 2], v[i], v[i + 1]);
+          emit(col0 + c, v);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------ host side
@@ -646,13 +950,79 @@ fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
   return launch_status();
 }
 
+// Clusters of two CTAs that can be resident at once (cached per kernel and
+// device); the pair kernel is persistent over that many pairs.
+template <int BN, bool BW>
+int pair_clusters() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    using C = Cfg2<BN, BW>;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * static_cast<unsigned>(num_sms()));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<BN, BW>, &cfg) != cudaSuccess) n = 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+template <int BN, bool BW>
+fp8q_status launch_pair(const void* a_op, const void* b_op, const GemmArgs& p, cudaStream_t stream) {
+  using C = Cfg2<BN, BW>;
+  CUtensorMap ma, mb;
+  if (!tensor_map(a_op, p.rows_a, p.K, BM, &ma) || !tensor_map(b_op, p.rows_b, p.K, C::HB, &mb))
+    return FP8Q_ERR_CUDA;
+  static int attr_done[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(gemm_pair_kernel<BN, BW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return FP8Q_ERR_CUDA;
+    attr_done[dev] = 1;
+  }
+  const int nc = pair_clusters<BN, BW>();
+  if (nc < 1) return FP8Q_ERR_UNSUPPORTED;
+  const int npairs = p.units < nc ? p.units : nc;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * static_cast<unsigned>(npairs));
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, BW>, ma, mb, p) != cudaSuccess) return FP8Q_ERR_CUDA;
+  return launch_status();
+}
+
 // ---------------------------------------------------------------- dispatch
 
 std::mutex g_force_mu;
 bool g_forced = false;
-fp8q_gemm_variant g_force{0, 1, 128};
+fp8q_gemm_variant g_force{0, 1, 128, 0};
 
 bool variant_supported(const fp8q_gemm_variant& v, int blockwise) {
+  if (v.cta_pair != 0 && v.cta_pair != 1) return false;
+  // (pairs: blockwise with 128-column tiles -- four accumulator buffers --,
+  // per token with 128 or 256)
+  if (v.cta_pair) return !v.swap_ab && v.split_k == 1 && (v.block_n == 128 || (!blockwise && v.block_n == 256));
   if (v.split_k < 0 || v.split_k > 64) return false;   // 0: stream-K
   if (v.swap_ab) return v.block_n == 16 || v.block_n == 32 || v.block_n == 64 || v.block_n == 128;
   if (blockwise) return v.block_n == 128 || v.block_n == 256;
@@ -671,11 +1041,11 @@ int epi_warps(const fp8q_gemm_variant& v, int blockwise) {
 struct TunedVariant {
   int blockwise;
   int64_t m_max, n, k;
-  int swap_ab, split_k, block_n;
+  int swap_ab, split_k, block_n, cta_pair;
 };
 constexpr TunedVariant kTuned[] = {
 #include "fp8q_variant_table.inc"
-    {-1, 0, 0, 0, 0, 0, 0},   // end marker
+    {-1, 0, 0, 0, 0, 0, 0, 0},   // end marker
 };
 
 bool tuned_variant(int64_t M, int64_t N, int64_t K, int blockwise, fp8q_gemm_variant* out) {
@@ -691,12 +1061,14 @@ bool tuned_variant(int64_t M, int64_t N, int64_t K, int blockwise, fp8q_gemm_var
   out->swap_ab = best->swap_ab;
   out->split_k = best->split_k;
   out->block_n = best->block_n;
+  out->cta_pair = best->cta_pair;
   return variant_supported(*out, blockwise);
 }
 
 // Shapes outside the table: rules drawn from the same measurements.
 fp8q_gemm_variant heuristic_variant(int64_t M, int64_t N, int64_t K, int blockwise) {
   fp8q_gemm_variant v;
+  v.cta_pair = 0;
   if (M <= 128) {
     // Swap-AB: the weight rows fill the 128-row MMA slot, the tokens its N.
     v.swap_ab = 1;
@@ -752,14 +1124,21 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int blockwise, const fp8q_gemm_v
   Plan pl;
   pl.v = v;
   const int64_t rows_a = v.swap_ab ? N : M, rows_b = v.swap_ab ? M : N;
-  pl.tiles_a = static_cast<int>((rows_a + BM - 1) / BM);
+  const int tile_rows = v.cta_pair ? 2 * BM : BM;      // CTA pairs: 256-row tiles
+  pl.tiles_a = static_cast<int>((rows_a + tile_rows - 1) / tile_rows);
   pl.tiles_b = static_cast<int>((rows_b + v.block_n - 1) / v.block_n);
   pl.kblocks = static_cast<int>((K + BK - 1) / BK);
   const int64_t tiles = static_cast<int64_t>(pl.tiles_a) * pl.tiles_b;
   pl.streamk = 0;
   pl.seg_len = 0;
   pl.total_iters = 0;
-  if (v.split_k == 0) {
+  if (v.cta_pair) {
+    pl.split = 1;
+    pl.kb_per_split = pl.kblocks;
+    pl.units = static_cast<int>(tiles);
+    pl.grid = 0;
+    pl.max_contrib = 1;
+  } else if (v.split_k == 0) {
     // stream-K: equal K-block ranges over at most one CTA per SM
     const int64_t total = tiles * pl.kblocks;
     int64_t grid = num_sms();
@@ -809,6 +1188,15 @@ fp8q_status run_gemm(const void* a_q, const void* b_q, GemmArgs& p, const Plan& 
   p.ws = pl.max_contrib > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.counter_bytes) : nullptr;
   p.status = device_status_ptr();
   const int bn = pl.v.block_n;
+  if (pl.v.cta_pair) {
+    p.rows_a = p.M;
+    p.rows_b = p.N;
+    if (bn == 128) return launch_pair<128, BW>(a_q, b_q, p, stream);
+    if constexpr (!BW) {
+      if (bn == 256) return launch_pair<256, false>(a_q, b_q, p, stream);
+    }
+    return FP8Q_ERR_UNSUPPORTED;
+  }
   if (pl.v.swap_ab) {
     p.rows_a = p.N;
     p.rows_b = p.M;

@@ -5,7 +5,7 @@
 For each scheme (per-token/per-channel scales, 1x128/128x128 block scales),
 each linear-layer shape (N, K) of the Qwen3-8B and Qwen3-32B models and each
 bucket of M, every candidate variant -- Swap-AB or not, tile width, whole-K
-tiles, split-K factors, stream-K -- is timed on the device, and the fastest
+tiles, split-K factors, stream-K, CTA pairs -- is timed on the device, and the fastest
 goes into ``csrc/fp8q_variant_table.inc``, which ``fp8q_gemm.cu`` compiles in.
 Rebuild the library afterwards (``python fp8_quantized_linear_rms_b200/build.py``).
 
@@ -63,16 +63,20 @@ def _splits(tiles: int, kblocks: int, sms: int) -> list[int]:
     return out
 
 
-def candidates(M: int, N: int, K: int, sms: int) -> list[tuple[int, int, int]]:
+def candidates(M: int, N: int, K: int, sms: int, blockwise: bool) -> list[tuple[int, int, int, int]]:
+    """(swap_ab, split_k, block_n, cta_pair) variants worth timing for this shape."""
     kb = K // 128
     out = []
     if M <= 128:
         bn = next(b for b in (16, 32, 64, 128) if b >= M)
         for b in sorted({bn, min(128, 2 * bn)}):
-            out += [(1, s, b) for s in _splits(_tiles(N, M, b), kb, sms)]
+            out += [(1, s, b, 0) for s in _splits(_tiles(N, M, b), kb, sms)]
     if M >= 32:
         for b in (128, 256):
-            out += [(0, s, b) for s in _splits(_tiles(M, N, b), kb, sms)]
+            out += [(0, s, b, 0) for s in _splits(_tiles(M, N, b), kb, sms)]
+    if M >= 256:
+        # CTA pairs: 256-row tiles on two SMs
+        out += [(0, 1, 128, 1)] + ([] if blockwise else [(0, 1, 256, 1)])
     return out
 
 
@@ -121,7 +125,7 @@ def tune(reps: int = 5, shapes=SHAPES, buckets=M_BUCKETS, log=print):
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             for bw in (0, 1):
                 times = {}
-                for v in candidates(M, N, K, sms):
+                for v in candidates(M, N, K, sms, bool(bw)):
                     fq.fp8q_force_gemm_variant(*v)
                     try:
                         ws = fq.make_workspace(M, N, K, bool(bw), dev)
@@ -141,7 +145,7 @@ def tune(reps: int = 5, shapes=SHAPES, buckets=M_BUCKETS, log=print):
                 row = {"shape": name, "blockwise": bw, "m_max": M, "N": N, "K": K,
                        "variant": list(best), "us": round(times[best], 2),
                        "tflops": round(2.0 * M * N * K / times[best] / 1e6, 1),
-                       "all": {f"{v[0]},{v[1]},{v[2]}": round(t, 2) for v, t in times.items()}}
+                       "all": {",".join(map(str, v)): round(t, 2) for v, t in times.items()}}
                 rows.append(row)
                 log(json.dumps(row))
             del a, y
@@ -155,10 +159,10 @@ def write_table(rows, path: str) -> None:
         f.write(f"// Measured GEMM variant table, written by tune.py on {dev}\n")
         f.write(f"// ({datetime.date.today().isoformat()}): the fastest variant per scheme, (N, K)\n")
         f.write("// and bucket of M (mean microseconds per call, weights read from HBM).\n")
-        f.write("// {blockwise, m_max, N, K, swap_ab, split_k (0 = stream-K), block_n}\n")
+        f.write("// {blockwise, m_max, N, K, swap_ab, split_k (0 = stream-K), block_n, cta_pair}\n")
         for r in rows:
-            s, k, n = r["variant"]
-            f.write(f"{{{r['blockwise']}, {r['m_max']}, {r['N']}, {r['K']}, {s}, {k}, {n}}},"
+            s, k, n, c = r["variant"]
+            f.write(f"{{{r['blockwise']}, {r['m_max']}, {r['N']}, {r['K']}, {s}, {k}, {n}, {c}}},"
                     f"  // {r['shape']}: {r['us']} us\n")
 
 

@@ -215,11 +215,16 @@ FP8Q_API size_t fp8q_workspace_bytes(int64_t M, int64_t N, int64_t K, int blockw
  * loop of every output tile among that many CTAs; split_k = 0 selects
  * stream-K: every CTA (at most one per SM) takes an equal contiguous range of
  * (tile, K block) iterations and tiles cut by range boundaries are summed
- * from their pieces in a fixed order; block_n is the MMA N extent. */
+ * from their pieces in a fixed order; block_n is the MMA N extent;
+ * cta_pair = 1 runs each 256-row tile on a cluster of two CTAs (two SMs)
+ * sharing one tcgen05 .cta_group::2 MMA, each SM staging half of the B tile
+ * (only with swap_ab = 0 and split_k = 1; block_n 128, or 256 for the
+ * per-token scheme). */
 typedef struct {
     int swap_ab;
     int split_k;
     int block_n;
+    int cta_pair;
 } fp8q_gemm_variant;
 
 /* The variant the library would run for this shape: the row of its built-in
@@ -234,7 +239,8 @@ FP8Q_API fp8q_status fp8q_select_gemm_variant(int64_t M, int64_t N, int64_t K, i
 /* Force a variant for every following GEMM call in this process (testing and
  * tuning only; not thread-safe).  NULL restores automatic selection.  Returns
  * FP8Q_ERR_INVALID_ARG if the variant is malformed (block_n not one of
- * 16, 32, 64, 128, 256; split_k < 0 or > 64). */
+ * 16, 32, 64, 128, 256; split_k < 0 or > 64; cta_pair not 0 or 1, or set
+ * with another combination than the one above). */
 FP8Q_API fp8q_status fp8q_force_gemm_variant(const fp8q_gemm_variant* v);
 
 /* ------------------------------------------------------------------------ */

@@ -66,7 +66,7 @@ def _variant_table():
     path = os.path.join(ROOT, "fp8_quantized_linear_rms_b200", "csrc", "fp8q_variant_table.inc")
     rows = []
     for line in open(path):
-        m = re.match(r"\{(-?\d+), (\d+), (\d+), (\d+), (\d+), (\d+), (\d+)\},", line)
+        m = re.match(r"\{(-?\d+), (\d+), (\d+), (\d+), (\d+), (\d+), (\d+), (\d+)\},", line)
         if m:
             rows.append(tuple(int(x) for x in m.groups()))
     return rows
@@ -76,9 +76,9 @@ def test_variant_table_lookup():
     rows = _variant_table()
     assert len(rows) >= 100
     keys = {}
-    for bw, m_max, n, k, swap, split, bn in rows:
+    for bw, m_max, n, k, swap, split, bn, pair in rows:
         keys.setdefault((bw, n, k), []).append(m_max)
-        want = {"swap_ab": swap, "split_k": split, "block_n": bn}
+        want = {"swap_ab": swap, "split_k": split, "block_n": bn, "cta_pair": pair}
         assert fq.fp8q_select_gemm_variant(m_max, n, k, bool(bw)) == want
     # an M between buckets takes the next larger bucket; above all, the largest
     for (bw, n, k), ms in keys.items():
@@ -88,10 +88,10 @@ def test_variant_table_lookup():
             if hi - lo > 1:
                 r = by_m[hi]
                 assert fq.fp8q_select_gemm_variant(lo + 1, n, k, bool(bw)) == \
-                    {"swap_ab": r[4], "split_k": r[5], "block_n": r[6]}
+                    {"swap_ab": r[4], "split_k": r[5], "block_n": r[6], "cta_pair": r[7]}
         r = by_m[ms[-1]]
         assert fq.fp8q_select_gemm_variant(ms[-1] * 4, n, k, bool(bw)) == \
-            {"swap_ab": r[4], "split_k": r[5], "block_n": r[6]}
+            {"swap_ab": r[4], "split_k": r[5], "block_n": r[6], "cta_pair": r[7]}
 
 
 def test_variant_selection_host_logic():
@@ -103,7 +103,7 @@ def test_variant_selection_host_logic():
     assert fq.fp8q_select_gemm_variant(33, N, K, True)["block_n"] == 64
     assert fq.fp8q_select_gemm_variant(100, N, K, False)["block_n"] == 128
     v = fq.fp8q_select_gemm_variant(8192, N, K, False)
-    assert v == {"swap_ab": 0, "split_k": 1, "block_n": 256}
+    assert v == {"swap_ab": 0, "split_k": 1, "block_n": 256, "cta_pair": 0}
     # 24 tiles: whole-K ranges split so that the tiles fill the SMs, each
     # range at least 8 K blocks; blockwise with M > 16 takes stream-K
     assert fq.fp8q_select_gemm_variant(16, N, K, False)["split_k"] == 2
@@ -113,7 +113,12 @@ def test_variant_selection_host_logic():
     assert fq.fp8q_workspace_bytes(8192, 51200, 5120, False) == 0
     # forcing
     fq.fp8q_force_gemm_variant(0, 2, 256)
-    assert fq.fp8q_select_gemm_variant(8192, 51200, 5120, False) == {"swap_ab": 0, "split_k": 2, "block_n": 256}
+    assert fq.fp8q_select_gemm_variant(8192, 51200, 5120, False) == \
+        {"swap_ab": 0, "split_k": 2, "block_n": 256, "cta_pair": 0}
+    fq.fp8q_force_gemm_variant(0, 1, 128, cta_pair=1)
+    assert fq.fp8q_select_gemm_variant(8192, 51200, 5120, True) == \
+        {"swap_ab": 0, "split_k": 1, "block_n": 128, "cta_pair": 1}
+    assert fq.fp8q_workspace_bytes(8192, 51200, 5120, True) == 0
     fq.fp8q_force_gemm_variant()
     with pytest.raises(fq.Fp8qError):
         fq.fp8q_force_gemm_variant(0, 1, 48)

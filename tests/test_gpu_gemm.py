@@ -80,6 +80,55 @@ def test_scaled_mm_blockwise_variants(M, N, K, swap, bn, split):
     gemm_tolerance_check(y, y_ref, ad, f"bw swap={swap} bn={bn} split={split}")
 
 
+# CTA pairs (cta_group::2): 256-row tiles on two SMs; tiny M leaves the odd
+# CTA's rows outside the matrix, K tails and many tiles per pair included.
+PAIR_SHAPES = [(1, 256, 384), (100, 384, 512), (260, 256, 1024), (600, 640, 768), (1024, 2048, 512)]
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("M,N,K", PAIR_SHAPES + [(100, 272, 400)])
+def test_scaled_mm_cta_pair(M, N, K, bn):
+    a = inp.random_e4m3_codes(M * 3 + K, (M, K))
+    b = inp.random_e4m3_codes(N * 7 + K, (N, K))
+    sa = inp.random_scales(M + 5, (M,))
+    sb = inp.random_scales(N + 6, (N,))
+    fq.fp8q_force_gemm_variant(0, 1, bn, cta_pair=1)
+    y = _run_pt(a, b, sa, sb, M, N, K)
+    y_ref, ad = oracle.scaled_mm(a, b, sa, sb)
+    gemm_tolerance_check(y, y_ref, ad, f"pt pair bn={bn}")
+
+
+@pytest.mark.parametrize("layout", ["row_major", "group_major"])
+@pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
+def test_scaled_mm_blockwise_cta_pair(M, N, K, layout):
+    a = inp.random_e4m3_codes(M * 5 + K, (M, K))
+    b = inp.random_e4m3_codes(N * 9 + K, (N, K))
+    sa = inp.random_scales(M + 7, (M, K // 128))
+    sb = inp.random_scales(N + 8, (N // 128, K // 128))
+    fq.fp8q_force_gemm_variant(0, 1, 128, cta_pair=1)
+    y = _run_bw(a, b, sa, sb, M, N, K, layout)
+    y_ref, ad = oracle.scaled_mm_blockwise(a, b, sa, sb)
+    gemm_tolerance_check(y, y_ref, ad, f"bw pair {layout}")
+
+
+def test_cta_pair_determinism_and_canaries():
+    # the same output bits on reruns; nothing written outside y's rows
+    M, N, K = 300, 512, 1024
+    a = to_dev_codes(inp.random_e4m3_codes(91, (M, K)))
+    b = to_dev_codes(inp.random_e4m3_codes(92, (N, K)))
+    sa = torch.from_numpy(inp.random_scales(93, (M, K // 128))).cuda()
+    sb = torch.from_numpy(inp.random_scales(94, (N // 128, K // 128))).cuda()
+    fq.fp8q_force_gemm_variant(0, 1, 128, cta_pair=1)
+    ys = []
+    for _ in range(2):
+        big = torch.full((M + 2, N), 12345.0, dtype=torch.bfloat16, device="cuda")
+        fq.fp8q_scaled_mm_blockwise(a, b, sa, sb, y=big[1:M + 1])
+        torch.cuda.synchronize()
+        assert torch.all(big[0] == 12345.0) and torch.all(big[M + 1] == 12345.0)
+        ys.append(big[1:M + 1].clone())
+    assert torch.equal(ys[0], ys[1])
+
+
 def test_blockwise_group_major_scales_and_ue8m0():
     M, N, K = 70, 256, 640
     a = inp.random_e4m3_codes(21, (M, K))
