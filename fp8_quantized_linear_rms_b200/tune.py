@@ -74,9 +74,11 @@ def candidates(M: int, N: int, K: int, sms: int, blockwise: bool) -> list[tuple[
     if M >= 32:
         for b in (128, 256):
             out += [(0, s, b, 0) for s in _splits(_tiles(M, N, b), kb, sms)]
-    if M >= 256:
-        # CTA pairs: 256-row tiles on two SMs
-        out += [(0, 1, 128, 1)] + ([] if blockwise else [(0, 1, 256, 1)])
+    if M >= 256 and not blockwise:
+        # CTA pairs: 256x256 tiles on two SMs.  (The blockwise pair kernel,
+        # whose two CTAs hand every K block's partial back and forth, and
+        # 128-wide pairs never come near the single-CTA variants.)
+        out += [(0, 1, 256, 1)]
     return out
 
 
