@@ -17,8 +17,10 @@ W ~ N(0, 0.02), quantized once per output channel / per 128x128 block.
 `value` is whole-job TFLOP/s (GEMM FLOPs of all ranks / max-over-ranks device
 time), inputs resident in HBM; each timed step is bracketed by CUDA events and
 followed by an untimed L2 flush.  `e2e` is the same metric through the public
-API with the activations copied from pinned host memory and both outputs copied
-back inside the timed region.  `--impl reference` times the CPU oracle on a
+API with each step's activations copied from pinned host memory and both of its
+outputs copied back inside the timed region, the copies on their own streams
+overlapping the neighbouring steps' kernels (double-buffered, as a serving loop
+runs); there the L2 flush before each step is inside the timed region.  `--impl reference` times the CPU oracle on a
 bounded sample of the same workload.
 """
 from __future__ import annotations
@@ -35,6 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 H, I = 4096, 12288
+METRIC = "FP8 quant+scaled_mm TFLOP/s (Qwen3-8B MLP block, per-token + blockwise)"
 EPS = 1e-6
 
 # DRAM bytes (read + write) of one launch of each gate_up GEMM, from one ncu
@@ -53,7 +56,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--sweep", default=None,
                     help="per-op timing instead of the step: quant, gemm8b, decode32b, prefill32b, all")
-    ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--reps", type=int, default=50)
     return ap.parse_args()
 
 
@@ -201,8 +204,9 @@ def run_native(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     ev_gu = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
 
-    def step(xin, ev=None):
-        # ev: [pt_start, pt_end, bw_start, bw_end] events around the two gate_up GEMMs
+    def step(xin, ev=None, y_pt=None, y_b=None):
+        # ev: [pt_start, pt_end, bw_start, bw_end] events around the two gate_up GEMMs;
+        # y_pt, y_b: the block outputs of the two chains (default out_pt, out_b)
         fq.fp8q_group_quant(xin, H, q=q_tok, scales=s_tok)
         fq.fp8q_group_quant(xin, 128, q=q_grp, scales=s_grp)
         fq.fp8q_rmsnorm_quant(xin, w_norm, EPS, H, q=qa, scales=sa)
@@ -212,7 +216,8 @@ def run_native(args, rank, world, local_rank):
         if ev:
             ev[1].record(stream)
         fq.fp8q_silu_mul_quant(h, I, q=qh, scales=sh)
-        fq.fp8q_scaled_mm(qh, d_pt, sh.view(-1), sd_pt, y=out_pt, workspace=ws["d"])
+        fq.fp8q_scaled_mm(qh, d_pt, sh.view(-1), sd_pt, y=out_pt if y_pt is None else y_pt,
+                          workspace=ws["d"])
         fq.fp8q_rmsnorm_quant(xin, w_norm, EPS, 128, q=qa_b, scales=sa_b, scale_layout="group_major")
         if ev:
             ev[2].record(stream)
@@ -221,8 +226,8 @@ def run_native(args, rank, world, local_rank):
         if ev:
             ev[3].record(stream)
         fq.fp8q_silu_mul_quant(h_b, 128, q=qh_b, scales=sh_b, scale_layout="group_major")
-        fq.fp8q_scaled_mm_blockwise(qh_b, d_bw, sh_b, sd_bw, a_scale_layout="group_major", y=out_b,
-                                    workspace=ws["db"])
+        fq.fp8q_scaled_mm_blockwise(qh_b, d_bw, sh_b, sd_bw, a_scale_layout="group_major",
+                                    y=out_b if y_b is None else y_b, workspace=ws["db"])
 
     LAUNCHES_PER_STEP = 10
 
@@ -259,24 +264,50 @@ def run_native(args, rank, world, local_rank):
     gub_ms = [e[2].elapsed_time(e[3]) for e in gu_ev]
     total_ms = sum(step_ms)
 
-    # ---- timed: end to end through host buffers
-    out_pinned = torch.empty((2, M, H), dtype=torch.bfloat16).pin_memory()
-    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    xd = torch.empty_like(x)
+    # ---- timed: end to end through host buffers.  Every step copies its input
+    # from pinned host memory and both block outputs back to pinned host memory;
+    # as in a serving loop the copies run on their own streams, double-buffered,
+    # so step i+1's upload and step i-1's download overlap step i's kernels.
+    # The L2 flush before each step's kernels stays inside this timed region.
+    NBUF = 2
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    xd = [torch.empty_like(x) for _ in range(NBUF)]
+    yd = [(torch.empty_like(out_pt), torch.empty_like(out_b)) for _ in range(NBUF)]
+    out_pinned = [torch.empty((2, M, H), dtype=torch.bfloat16).pin_memory() for _ in range(NBUF)]
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    in_done = [ev() for _ in range(args.steps)]
+    comp_done = [ev() for _ in range(args.steps)]
+    out_done = [ev() for _ in range(args.steps)]
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
+    e_start.record(stream)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
     for i in range(args.steps):
+        b = i % NBUF
+        with torch.cuda.stream(s_in):
+            if i >= NBUF:
+                s_in.wait_event(comp_done[i - NBUF])       # step i-2 has read xd[b]
+            xd[b].copy_(x_pinned, non_blocking=True)
+            in_done[i].record(s_in)
+        stream.wait_event(in_done[i])
+        if i >= NBUF:
+            stream.wait_event(out_done[i - NBUF])          # yd[b] has reached the host
         flush.zero_()
-        e_starts[i].record(stream)
-        xd.copy_(x_pinned, non_blocking=True)
-        step(xd)
-        out_pinned[0].copy_(out_pt, non_blocking=True)
-        out_pinned[1].copy_(out_b, non_blocking=True)
-        e_ends[i].record(stream)
+        step(xd[b], y_pt=yd[b][0], y_b=yd[b][1])
+        comp_done[i].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[i])
+            out_pinned[b][0].copy_(yd[b][0], non_blocking=True)
+            out_pinned[b][1].copy_(yd[b][1], non_blocking=True)
+            out_done[i].record(s_out)
+    stream.wait_event(out_done[args.steps - 1])
+    e_end.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends))
+    e2e_ms = e_start.elapsed_time(e_end)
     st = fq.fp8q_last_device_status()
     if st != fq.OK:
         raise RuntimeError(f"device status after timing: {fq.fp8q_status_string(st)}")
@@ -307,7 +338,7 @@ def run_native(args, rank, world, local_rank):
     achieved_bw = gu_flops / (statistics.mean(gub_ms) * 1e-3) / 1e12
     qb = quant_bytes(M)
     line = {
-        "metric": "FP8 quant+scaled_mm TFLOP/s (Qwen3-8B MLP block, per-token + blockwise)",
+        "metric": METRIC,
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
@@ -316,7 +347,10 @@ def run_native(args, rank, world, local_rank):
         "quant_hbm_gbs": round(qb * args.steps / (total_ms * 1e-3) / 1e9, 1),
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": M * H * 2, "d2h_bytes_per_step": 2 * M * H * 2},
+                "h2d_bytes_per_step": M * H * 2, "d2h_bytes_per_step": 2 * M * H * 2,
+                "ms_per_step": round(e2e_ms / args.steps, 4),
+                "copies": "pinned host buffers, own streams, double-buffered against the "
+                          "neighbouring steps' kernels; L2 flush inside the timed region"},
         # The dominant kernel of the step (largest share of the ncu launch list):
         # the blockwise gate_up GEMM.  traffic = ncu dram read + write bytes of one
         # launch of the same kernel build (profiles/gemm_kernel_qwen3_8b_mlp_m2048.md).
@@ -390,7 +424,7 @@ def run_reference(args):
     sample = (f"{rows} of {M} tokens per step (all ops of the step on those tokens; "
               f"value = their GEMM FLOPs / oracle time)")
     return {
-        "metric": "FP8 quant+scaled_mm TFLOP/s (Qwen3-8B MLP block, per-token + blockwise)",
+        "metric": METRIC,
         "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -415,7 +449,9 @@ def cpu_baseline_leg(args):
 def run_sweep(args):
     """Time every op of the path on the config shapes, one JSON line per case:
     device time per launch (CUDA events, median of --reps, L2 flushed before each
-    rep), achieved GB/s or TFLOP/s and the fraction of the measured peak."""
+    rep), achieved GB/s or TFLOP/s and the fraction of the measured peak.  Small
+    batches (quant M <= 128, GEMM M <= 64) are also replayed from a CUDA graph and
+    their per-call time reported (GEMM weights rotated across copies > L2)."""
     import numpy as np
     import torch
 
@@ -454,6 +490,35 @@ def run_sweep(args):
         assert fq.fp8q_last_device_status() == fq.OK
         return float(np.median(ts))
 
+    def graph_time(fns):
+        """Per-call device time of fns[0], fns[1], ... replayed back to back
+        from one CUDA graph (median over --reps replays)."""
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for f in fns:
+                f()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for f in fns:
+                f()
+        g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e-3 / len(fns))
+        assert fq.fp8q_last_device_status() == fq.OK
+        del g
+        return float(np.median(ts))
+
     def emit(d):
         print(json.dumps(d), flush=True)
 
@@ -485,9 +550,13 @@ def run_sweep(args):
                         fn = lambda: fq.fp8q_group_quant(x, g)
                         nbytes = M * (2 * L + L + 4 * (L // g))
                     t = timeit(fn)
-                    emit({"op": op, "M": M, "L": L, "group": g, "us": round(t * 1e6, 2),
-                          "GB/s": round(nbytes / t / 1e9, 1),
-                          "frac_hbm": round(nbytes / t / 1e9 / hbm, 3)})
+                    d = {"op": op, "M": M, "L": L, "group": g, "us": round(t * 1e6, 2),
+                         "GB/s": round(nbytes / t / 1e9, 1),
+                         "frac_hbm": round(nbytes / t / 1e9 / hbm, 3)}
+                    if M <= 128:
+                        # small batches: 16 calls replayed from a CUDA graph (input L2-resident)
+                        d["graph_us_per_call"] = round(graph_time([fn] * 16) * 1e6, 2)
+                    emit(d)
                     del x
 
     def gemm_case(tag, M, N, K, blockwise):
@@ -508,10 +577,27 @@ def run_sweep(args):
         flops = 2.0 * M * N * K
         nbytes = M * K + N * K + 2 * M * N
         v = fq.fp8q_select_gemm_variant(M, N, K, blockwise)
-        emit({"op": "scaled_mm_blockwise" if blockwise else "scaled_mm", "shape": tag, "M": M,
-              "N": N, "K": K, "variant": v, "us": round(t * 1e6, 2),
-              "TFLOP/s": round(flops / t / 1e12, 1), "frac_fp8_peak": round(flops / t / 1e12 / fp8_peak, 3),
-              "GB/s": round(nbytes / t / 1e9, 1), "frac_hbm": round(nbytes / t / 1e9 / hbm, 3)})
+        d = {"op": "scaled_mm_blockwise" if blockwise else "scaled_mm", "shape": tag, "M": M,
+             "N": N, "K": K, "variant": v, "us": round(t * 1e6, 2),
+             "TFLOP/s": round(flops / t / 1e12, 1), "frac_fp8_peak": round(flops / t / 1e12 / fp8_peak, 3),
+             "GB/s": round(nbytes / t / 1e9, 1), "frac_hbm": round(nbytes / t / 1e9 / hbm, 3)}
+        if M <= 64:
+            # weight streaming: one CUDA graph replays a call on each of enough
+            # copies of the weights (384 MiB in all) that every call reads its
+            # weights from HBM, as a model's successive layers do
+            copies = max(2, min(64, -(-(384 << 20) // (N * K))))
+            bs = [b] + [torch.empty_like(b).copy_(b) for _ in range(copies - 1)]
+            if blockwise:
+                fns = [lambda bb=bb: fq.fp8q_scaled_mm_blockwise(
+                    a, bb, sa, sb, a_scale_layout="group_major", workspace=ws) for bb in bs]
+            else:
+                fns = [lambda bb=bb: fq.fp8q_scaled_mm(a, bb, sa, sb, workspace=ws) for bb in bs]
+            tg = graph_time(fns)
+            d.update({"graph_us_per_call": round(tg * 1e6, 2),
+                      "graph_GB/s": round(nbytes / tg / 1e9, 1),
+                      "graph_frac_hbm": round(nbytes / tg / 1e9 / hbm, 3)})
+            del bs, fns
+        emit(d)
 
     if which in ("gemm8b", "all"):
         sh = inp.linear_shapes(inp.QWEN3_8B)
