@@ -1,4 +1,5 @@
 // fp8q_abi.cu -- status, version and device-query entry points of libfp8q.
+#include <cstdlib>
 #include <mutex>
 
 #include "fp8q_common.cuh"
@@ -17,6 +18,14 @@ int* device_status_ptr() {
     cache[dev] = static_cast<int*>(p);
   }
   return cache[dev];
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("FP8Q_PDL");
+    return !(v && v[0] == '0' && v[1] == '\0');
+  }();
+  return on;
 }
 
 int num_sms() {

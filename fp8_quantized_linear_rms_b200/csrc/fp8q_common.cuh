@@ -27,6 +27,21 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Programmatic dependent launch.  Every kernel is launched with the
+// programmatic-stream-serialization attribute (unless FP8Q_PDL=0), so it may
+// start while the previous kernel of its stream is still finishing.  It runs
+// its prologue (barrier init, TMEM allocation, descriptor prefetch, and for
+// the GEMMs an L2 prefetch of the first weight tiles, which no kernel of the
+// path writes), then griddep_wait() blocks until every earlier kernel of the
+// stream has completed and its writes are visible.  Nothing before the wait
+// reads or writes memory an earlier kernel may write.  griddep_launch_dependents()
+// lets the next kernel begin its own prologue.  Launched without the
+// attribute, both instructions do nothing.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Host-side helpers shared by the entry points.
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -36,5 +51,37 @@ inline fp8q_status launch_status() {
 }
 
 int num_sms();  // SM count of the current device (cached per device)
+
+bool pdl_enabled();  // false when the environment sets FP8Q_PDL=0 (read once)
+
+// Launch `kern` on `stream` with programmatic dependent launch (when enabled)
+// and, for cluster_x > 1, clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+inline fp8q_status launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t stream, unsigned cluster_x, Args&&... args) {
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  if (cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...) != cudaSuccess) return FP8Q_ERR_CUDA;
+  return launch_status();
+}
 
 }  // namespace fp8q

@@ -219,6 +219,21 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (warp == 0 && lane == 0) {
+    // The first weight tiles of this CTA into L2 while the previous kernel
+    // finishes (weights: the MMA's A operand under Swap-AB, else B).
+    SegIter si(p);
+    Seg g;
+    if (si.next(p, g)) {
+      const int kend = min(g.kb1, g.kb0 + S);
+      for (int kb = g.kb0; kb < kend; ++kb) {
+        if (SWAP) tma_prefetch_2d(&tmA, kb * BK, g.ta * BM);
+        else tma_prefetch_2d(&tmB, kb * BK, g.tb * BN);
+      }
+    }
+  }
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -652,6 +667,15 @@ __global__ void __launch_bounds__(Cfg2<BN, BW>::THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int npairs = static_cast<int>(gridDim.x >> 1);
   const int pair = static_cast<int>(blockIdx.x >> 1);
+  if (warp == 0 && lane == 0 && pair < p.units) {
+    // this CTA's half of the first weight tiles into L2 (see gemm_kernel)
+    const int tb = pair / p.tiles_a;
+    const int kend = min(p.kblocks, S);
+    for (int kb = 0; kb < kend; ++kb)
+      tma_prefetch_2d(&tmB, kb * BK, tb * BN + static_cast<int>(rank) * C::HB);
+  }
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -946,8 +970,8 @@ fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
   int grid;
   if (p.streamk) grid = (p.total_iters + p.seg_len - 1) / p.seg_len;
   else grid = p.units < num_sms() ? p.units : num_sms();
-  gemm_kernel<BN, SWAP, BW><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(ma, mb, p);
-  return launch_status();
+  return launch_kernel(gemm_kernel<BN, SWAP, BW>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream,
+                       1, ma, mb, p);
 }
 
 // Clusters of two CTAs that can be resident at once (cached per kernel and
@@ -996,20 +1020,8 @@ fp8q_status launch_pair(const void* a_op, const void* b_op, const GemmArgs& p, c
   const int nc = pair_clusters<BN, BW>();
   if (nc < 1) return FP8Q_ERR_UNSUPPORTED;
   const int npairs = p.units < nc ? p.units : nc;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(2 * static_cast<unsigned>(npairs));
-  cfg.blockDim = dim3(C::THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, BW>, ma, mb, p) != cudaSuccess) return FP8Q_ERR_CUDA;
-  return launch_status();
+  return launch_kernel(gemm_pair_kernel<BN, BW>, dim3(2 * static_cast<unsigned>(npairs)),
+                       dim3(C::THREADS), C::SMEM_BYTES, stream, 2, ma, mb, p);
 }
 
 // ---------------------------------------------------------------- dispatch

@@ -559,6 +559,8 @@ template <int OP, bool PER_TOKEN, int CH, int MAXT, int MINB>
 __global__ void __launch_bounds__(MAXT, MINB) quant_rows_kernel(const QuantParams p) {
   __shared__ double red_d[32];
   __shared__ float red_f[32];
+  griddep_wait();                 // x (and w) may come from the previous kernel
+  griddep_launch_dependents();
   for (int64_t row = blockIdx.x; row < p.M; row += gridDim.x)
     process_row<OP, PER_TOKEN, CH>(p, row, GlobalRow{p.x + row * p.ldx}, threadIdx.x, blockDim.x,
                                    0, red_d, red_f, [] {});
@@ -601,6 +603,8 @@ __global__ void __launch_bounds__(ring_max_threads(OP, CH), 1)
     sm100::fence_mbar_init();
   }
   __syncthreads();
+  griddep_wait();                 // x may come from the previous kernel
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -685,9 +689,8 @@ fp8q_status launch_ring(const QuantParams& p, int T, int nteams, int nbuf, int s
   }
   int64_t grid = num_sms();
   if (grid > p.M) grid = p.M;
-  kern<<<static_cast<unsigned>(grid), 32 + nteams * T, smem, stream>>>(p, nbuf, nteams, T, stride,
-                                                                       device_status_ptr());
-  return launch_status();
+  return launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(32 + nteams * T), smem, stream,
+                       1, p, nbuf, nteams, T, stride, device_status_ptr());
 }
 
 template <int OP>
@@ -710,20 +713,14 @@ fp8q_status launch_quant(const QuantParams& p, cudaStream_t stream) {
                      : launch_ring<OP, false, 8>(p, T, nteams, nbuf, stride, stream);
   const int64_t grid = p.M < (1LL << 30) ? p.M : (1LL << 30);
   const dim3 g(static_cast<unsigned>(grid)), b(T);
-  if (ch == 8) {
-    if (per_token) quant_rows_kernel<OP, true, 8, 512, 1><<<g, b, 0, stream>>>(p);
-    else quant_rows_kernel<OP, false, 8, 512, 1><<<g, b, 0, stream>>>(p);
-  } else if (OP == OP_SILU && T <= 256) {
-    if (per_token) quant_rows_kernel<OP, true, 4, 256, 3><<<g, b, 0, stream>>>(p);
-    else quant_rows_kernel<OP, false, 4, 256, 3><<<g, b, 0, stream>>>(p);
-  } else if (OP == OP_SILU && T <= 384) {
-    if (per_token) quant_rows_kernel<OP, true, 4, 384, 2><<<g, b, 0, stream>>>(p);
-    else quant_rows_kernel<OP, false, 4, 384, 2><<<g, b, 0, stream>>>(p);
-  } else {
-    if (per_token) quant_rows_kernel<OP, true, 4, 512, 2><<<g, b, 0, stream>>>(p);
-    else quant_rows_kernel<OP, false, 4, 512, 2><<<g, b, 0, stream>>>(p);
-  }
-  return launch_status();
+  auto go = [&](auto kern) { return launch_kernel(kern, g, b, 0, stream, 1, p); };
+  if (ch == 8)
+    return per_token ? go(quant_rows_kernel<OP, true, 8, 512, 1>) : go(quant_rows_kernel<OP, false, 8, 512, 1>);
+  if (OP == OP_SILU && T <= 256)
+    return per_token ? go(quant_rows_kernel<OP, true, 4, 256, 3>) : go(quant_rows_kernel<OP, false, 4, 256, 3>);
+  if (OP == OP_SILU && T <= 384)
+    return per_token ? go(quant_rows_kernel<OP, true, 4, 384, 2>) : go(quant_rows_kernel<OP, false, 4, 384, 2>);
+  return per_token ? go(quant_rows_kernel<OP, true, 4, 512, 2>) : go(quant_rows_kernel<OP, false, 4, 512, 2>);
 }
 
 // Host-side validation shared by the three ops (row length L of y).

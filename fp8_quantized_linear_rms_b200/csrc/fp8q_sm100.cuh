@@ -112,6 +112,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// L2 prefetch of the tile of tensor map m at (x, y) (no shared memory, no
+// completion; rows outside the tensor are skipped).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* m, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(m), "r"(x),
+               "r"(y)
+               : "memory");
+}
+
 // Untiled bulk copy global -> shared of `bytes` (multiple of 16; both
 // addresses 16-byte aligned), completing transaction bytes on `bar`.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
