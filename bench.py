@@ -43,8 +43,8 @@ EPS = 1e-6
 # DRAM bytes (read + write) of one launch of each gate_up GEMM, from one ncu
 # capture of the current kernel build (profiles/gemm_kernel_qwen3_8b_mlp_m2048.md);
 # set to None whenever the kernel changes until it is captured again.
-GATE_UP_BW_TRAFFIC = 179.4e6
-GATE_UP_PT_TRAFFIC = 172.9e6
+GATE_UP_BW_TRAFFIC = 170.9e6
+GATE_UP_PT_TRAFFIC = 172.1e6
 
 
 def parse():
