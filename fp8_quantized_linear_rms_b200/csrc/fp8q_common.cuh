@@ -31,10 +31,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // programmatic-stream-serialization attribute (unless FP8Q_PDL=0), so it may
 // start while the previous kernel of its stream is still finishing.  It runs
 // its prologue (barrier init, TMEM allocation, descriptor prefetch, and for
-// the GEMMs an L2 prefetch of the first weight tiles, which no kernel of the
-// path writes), then griddep_wait() blocks until every earlier kernel of the
-// stream has completed and its writes are visible.  Nothing before the wait
-// reads or writes memory an earlier kernel may write.  griddep_launch_dependents()
+// the GEMMs an L2 prefetch of the first weight tiles: a cache hint with no
+// visible effect, the tiles are loaded again after the wait), then
+// griddep_wait() blocks until every earlier kernel of the stream has
+// completed and its writes are visible.  Nothing before the wait reads or
+// writes memory an earlier kernel may write.  griddep_launch_dependents()
 // lets the next kernel begin its own prologue.  Launched without the
 // attribute, both instructions do nothing.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

@@ -29,7 +29,16 @@
  *     dimension `ld*` given in ELEMENTS.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *     stream).  Calls are asynchronous: they enqueue kernels and return; no
- *     call synchronizes the host except fp8q_last_device_status.
+ *     call synchronizes the host except fp8q_last_device_status.  Calls can
+ *     be captured into CUDA graphs.
+ *   - Kernels are launched with programmatic dependent launch: one may begin
+ *     its setup while the previous kernel on the stream is still running, but
+ *     reads and writes nothing until that kernel has completed and its writes
+ *     are visible.  The one early access is an L2 prefetch of a GEMM's first
+ *     weight tiles, a cache hint with no visible effect (the data are read
+ *     again after the wait), so stream order holds for every buffer.  Setting
+ *     the environment variable FP8Q_PDL=0 before the first call launches
+ *     kernels without it.
  *   - Argument errors are found on the host before anything is launched; the
  *     call then returns FP8Q_ERR_INVALID_ARG (or FP8Q_ERR_UNSUPPORTED) and
  *     launches nothing.  A launch failure returns FP8Q_ERR_CUDA.  A GEMM

@@ -15,6 +15,12 @@ calls on the same inputs bit for bit, for the automatic variants and for
 forced split-K and stream-K variants, whose arrival counters must come back
 to zero between replays.  (The eager results themselves are checked against
 the oracle by the other GPU tests.)
+
+Every kernel is launched with programmatic dependent launch, so it may start
+before the previous kernel of the stream has finished and must wait before
+reading that kernel's output.  The same chains issued back to back must
+therefore equal the chains with a host synchronization after every call,
+where no two kernels can overlap.
 """
 import numpy as np
 import pytest
@@ -61,25 +67,34 @@ class Block:
             "gu_b": fq.make_workspace(M, 2 * I, H, True), "dn_b": fq.make_workspace(M, H, I, True),
         }
 
-    def run(self):
+    def run(self, sync_each=False):
         o, ws = self.out, self.ws
-        fq.fp8q_rmsnorm_quant(self.x, self.w, EPS, H, q=o["qa"], scales=o["sa"])
-        fq.fp8q_scaled_mm(o["qa"], self.gu, o["sa"].view(-1), self.sgu_ch, y=o["h"],
-                          workspace=ws["gu"])
-        fq.fp8q_silu_mul_quant(o["h"], I, q=o["qh"], scales=o["sh"])
-        fq.fp8q_scaled_mm(o["qh"], self.dn, o["sh"].view(-1), self.sdn_ch, y=o["y"],
-                          workspace=ws["dn"])
-        fq.fp8q_rmsnorm_quant(self.x, self.w, EPS, 128, q=o["qa_b"], scales=o["sa_b"],
-                              scale_layout="group_major")
-        fq.fp8q_scaled_mm_blockwise(o["qa_b"], self.gu, o["sa_b"], self.sgu_bl,
-                                    a_scale_layout="group_major", y=o["h_b"], workspace=ws["gu_b"])
-        fq.fp8q_silu_mul_quant(o["h_b"], 128, q=o["qh_b"], scales=o["sh_b"],
-                               scale_layout="group_major")
-        fq.fp8q_scaled_mm_blockwise(o["qh_b"], self.dn, o["sh_b"], self.sdn_bl,
-                                    a_scale_layout="group_major", y=o["y_b"], workspace=ws["dn_b"])
+        calls = [
+            lambda: fq.fp8q_rmsnorm_quant(self.x, self.w, EPS, H, q=o["qa"], scales=o["sa"]),
+            lambda: fq.fp8q_scaled_mm(o["qa"], self.gu, o["sa"].view(-1), self.sgu_ch, y=o["h"],
+                                      workspace=ws["gu"]),
+            lambda: fq.fp8q_silu_mul_quant(o["h"], I, q=o["qh"], scales=o["sh"]),
+            lambda: fq.fp8q_scaled_mm(o["qh"], self.dn, o["sh"].view(-1), self.sdn_ch, y=o["y"],
+                                      workspace=ws["dn"]),
+            lambda: fq.fp8q_rmsnorm_quant(self.x, self.w, EPS, 128, q=o["qa_b"], scales=o["sa_b"],
+                                          scale_layout="group_major"),
+            lambda: fq.fp8q_scaled_mm_blockwise(o["qa_b"], self.gu, o["sa_b"], self.sgu_bl,
+                                                a_scale_layout="group_major", y=o["h_b"],
+                                                workspace=ws["gu_b"]),
+            lambda: fq.fp8q_silu_mul_quant(o["h_b"], 128, q=o["qh_b"], scales=o["sh_b"],
+                                           scale_layout="group_major"),
+            lambda: fq.fp8q_scaled_mm_blockwise(o["qh_b"], self.dn, o["sh_b"], self.sdn_bl,
+                                                a_scale_layout="group_major", y=o["y_b"],
+                                                workspace=ws["dn_b"]),
+        ]
         if self.noalloc:
-            fq.fp8q_scaled_mm_blockwise_noalloc(o["qa_b"], self.gu, o["sa_b"], self.sgu_bl,
-                                                a_scale_layout="group_major", y=o["y_n"])
+            calls.append(lambda: fq.fp8q_scaled_mm_blockwise_noalloc(
+                o["qa_b"], self.gu, o["sa_b"], self.sgu_bl, a_scale_layout="group_major",
+                y=o["y_n"]))
+        for c in calls:
+            c()
+            if sync_each:
+                torch.cuda.synchronize()
 
     def snapshot(self) -> dict:
         torch.cuda.synchronize()
@@ -134,5 +149,32 @@ def test_chain_replays_in_a_cuda_graph(variant):
             _assert_same(ref, blk.snapshot(), what)
         assert fq.fp8q_last_device_status() == fq.OK
         del g
+    finally:
+        fq.fp8q_force_gemm_variant()
+
+
+@pytest.mark.parametrize("variant", [None, (1, 4, 16), (0, 2, 128)],
+                         ids=["auto", "swap-splitk4", "splitk2"])
+def test_back_to_back_calls_match_serialized_calls(variant):
+    if variant is None:
+        fq.fp8q_force_gemm_variant()
+    else:
+        fq.fp8q_force_gemm_variant(*variant)
+    try:
+        blk = Block(noalloc=variant is None)
+        for seed in (721, 722):
+            blk.x.copy_(_inputs(seed))
+            torch.cuda.synchronize()
+            blk.run(sync_each=True)
+            ref = blk.snapshot()
+            for rep in range(3):
+                # poison every intermediate and output, then the chain with no
+                # host sync: a kernel reading its producer's output too early
+                # would see the poison
+                for t in blk.out.values():
+                    t.view(torch.uint8).fill_(0xFF)
+                blk.run()
+                _assert_same(ref, blk.snapshot(), f"back-to-back chain, input {seed}, run {rep}")
+        assert fq.fp8q_last_device_status() == fq.OK
     finally:
         fq.fp8q_force_gemm_variant()
