@@ -76,6 +76,23 @@ def quant_bytes(M):
     return gq_tok + gq_grp + rms_tok + rms_grp + silu_tok + silu_grp
 
 
+def max_over_ranks(values, world, device="cpu"):
+    """Element-wise maximum of each rank's timings, returned on every rank (the
+    slowest rank sets the job's time)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tflops(flops_per_rank_step, steps, world, ms):
+    """Whole-job throughput: the GEMM FLOPs all ranks did in `steps` steps over
+    the (max-over-ranks) time `ms`; each rank runs its own batch (replicas)."""
+    return flops_per_rank_step * steps * world / (ms * 1e-3) / 1e12
+
+
 def workload_config(M, n):
     return {"workload": f"qwen3-8b-mlp-block-m{M}-per-token+blockwise",
             "model": "Qwen3-8B-shaped MLP (hidden 4096, intermediate 12288)",
@@ -313,14 +330,11 @@ def run_native(args, rank, world, local_rank):
         raise RuntimeError(f"device status after timing: {fq.fp8q_status_string(st)}")
 
     # ---- max over ranks
-    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = t.tolist()
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, dev)
 
     flops_step = gemm_flops(M)
-    value = flops_step * args.steps * world / (total_ms * 1e-3) / 1e12
-    e2e_value = flops_step * args.steps * world / (e2e_ms * 1e-3) / 1e12
+    value = job_tflops(flops_step, args.steps, world, total_ms)
+    e2e_value = job_tflops(flops_step, args.steps, world, e2e_ms)
     gu_flops = 2 * M * H * 2 * I
     gu_avg_s = statistics.mean(gu_ms) * 1e-3
     peaks = {}
