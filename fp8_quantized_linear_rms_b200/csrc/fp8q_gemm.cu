@@ -1093,6 +1093,16 @@ fp8q_gemm_variant heuristic_variant(int64_t M, int64_t N, int64_t K, int blockwi
   const int64_t tiles = ((rows_a + BM - 1) / BM) * ((rows_b + v.block_n - 1) / v.block_n);
   const int64_t kblocks = (K + BK - 1) / BK;
   const int64_t sms = num_sms();
+  // Per-token scales from M = 512 up: 256x256 tiles on CTA pairs once there
+  // are at least 40 of them (the measured table picks them for every layer
+  // shape from M = 512 or 1024 on; fewer tiles leave too many SMs idle).
+  const int64_t pair_tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + 255) / 256);
+  if (!blockwise && M >= 512 && pair_tiles >= 40) {
+    v.block_n = 256;
+    v.split_k = 1;
+    v.cta_pair = 1;
+    return v;
+  }
   if (tiles >= sms) {
     v.split_k = 1;
   } else if (blockwise && M > 16) {

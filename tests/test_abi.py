@@ -102,8 +102,14 @@ def test_variant_selection_host_logic():
     assert fq.fp8q_select_gemm_variant(1, N, K, True)["block_n"] == 16
     assert fq.fp8q_select_gemm_variant(33, N, K, True)["block_n"] == 64
     assert fq.fp8q_select_gemm_variant(100, N, K, False)["block_n"] == 128
-    v = fq.fp8q_select_gemm_variant(8192, N, K, False)
+    v = fq.fp8q_select_gemm_variant(8192, N, K, True)
     assert v == {"swap_ab": 0, "split_k": 1, "block_n": 256, "cta_pair": 0}
+    # per-token scales, M >= 512 and at least 40 tiles of 256 x 256: CTA pairs
+    v = fq.fp8q_select_gemm_variant(8192, N, K, False)
+    assert v == {"swap_ab": 0, "split_k": 1, "block_n": 256, "cta_pair": 1}
+    assert fq.fp8q_select_gemm_variant(512, 5120 - 128, K, False)["cta_pair"] == 1   # 2 x 20 tiles
+    assert fq.fp8q_select_gemm_variant(512, 4096 + 128, K, False)["cta_pair"] == 0   # 2 x 17 tiles
+    assert fq.fp8q_select_gemm_variant(256, 51200 + 128, K, False)["cta_pair"] == 0  # M < 512
     # 24 tiles: whole-K ranges split so that the tiles fill the SMs, each
     # range at least 8 K blocks; blockwise with M > 16 takes stream-K
     assert fq.fp8q_select_gemm_variant(16, N, K, False)["split_k"] == 2
