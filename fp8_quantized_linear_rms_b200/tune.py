@@ -51,6 +51,13 @@ def _tiles(rows_a: int, rows_b: int, bn: int) -> int:
     return -(-rows_a // 128) * -(-rows_b // bn)
 
 
+def _effective_split(s: int, kblocks: int) -> int:
+    """Split factor the library runs for a requested s: ceil(kblocks / s) K blocks
+    per split, so only ceil(kblocks / that) splits are non-empty."""
+    per = -(-kblocks // s)
+    return -(-kblocks // per)
+
+
 def _splits(tiles: int, kblocks: int, sms: int) -> list[int]:
     out = [1]
     if tiles < 2 * sms:
@@ -59,7 +66,9 @@ def _splits(tiles: int, kblocks: int, sms: int) -> list[int]:
         fit = sms // tiles
         for s in sorted({2, 3, 4, 6, 8, fit}):
             if 1 < s <= min(fit, kblocks):
-                out.append(s)
+                e = _effective_split(s, kblocks)
+                if e > 1 and e not in out:
+                    out.append(e)
     return out
 
 
@@ -155,8 +164,8 @@ def tune(reps: int = 5, shapes=SHAPES, buckets=M_BUCKETS, log=print):
     return rows
 
 
-def write_table(rows, path: str) -> None:
-    dev = torch.cuda.get_device_name()
+def write_table(rows, path: str, device: str | None = None) -> None:
+    dev = device or torch.cuda.get_device_name()
     with open(path, "w") as f:
         f.write(f"// Measured GEMM variant table, written by tune.py on {dev}\n")
         f.write(f"// ({datetime.date.today().isoformat()}): the fastest variant per scheme, (N, K)\n")
