@@ -1,4 +1,5 @@
 // fp8q_abi.cu -- status, version and device-query entry points of libfp8q.
+#include <atomic>
 #include <cstdlib>
 #include <mutex>
 
@@ -8,16 +9,20 @@ namespace fp8q {
 
 __device__ int g_device_status = 0;
 
+// Per-device caches below are atomics: concurrent first calls may both fill
+// an entry, with the same value.
 int* device_status_ptr() {
-  static int* cache[64] = {nullptr};
+  static std::atomic<int*> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (cache[dev] == nullptr) {
+  int* c = cache[dev].load(std::memory_order_relaxed);
+  if (c == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-    cache[dev] = static_cast<int*>(p);
+    c = static_cast<int*>(p);
+    cache[dev].store(c, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return c;
 }
 
 bool pdl_enabled() {
@@ -29,16 +34,16 @@ bool pdl_enabled() {
 }
 
 int num_sms() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 }  // namespace fp8q

@@ -31,6 +31,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
 #include <mutex>
 #include <unordered_map>
 
@@ -958,14 +959,14 @@ fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
   CUtensorMap ma, mb;
   if (!tensor_map(a_op, p.rows_a, p.K, BM, &ma) || !tensor_map(b_op, p.rows_b, p.K, BN, &mb))
     return FP8Q_ERR_CUDA;
-  static int attr_done[64] = {0};
+  static std::atomic<int> attr_done[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+  if (dev >= 0 && dev < 64 && !attr_done[dev].load(std::memory_order_relaxed)) {
     if (cudaFuncSetAttribute(gemm_kernel<BN, SWAP, BW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return FP8Q_ERR_CUDA;
-    attr_done[dev] = 1;
+    attr_done[dev].store(1, std::memory_order_relaxed);
   }
   int grid;
   if (p.streamk) grid = (p.total_iters + p.seg_len - 1) / p.seg_len;
@@ -978,11 +979,11 @@ fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
 // device); the pair kernel is persistent over that many pairs.
 template <int BN, bool BW>
 int pair_clusters() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return 0;
-  if (cache[dev] == 0) {
+  if (cache[dev].load(std::memory_order_relaxed) == 0) {
     using C = Cfg2<BN, BW>;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -997,9 +998,9 @@ int pair_clusters() {
     cfg.numAttrs = 1;
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<BN, BW>, &cfg) != cudaSuccess) n = 0;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return cache[dev].load(std::memory_order_relaxed);
 }
 
 template <int BN, bool BW>
@@ -1008,14 +1009,14 @@ fp8q_status launch_pair(const void* a_op, const void* b_op, const GemmArgs& p, c
   CUtensorMap ma, mb;
   if (!tensor_map(a_op, p.rows_a, p.K, BM, &ma) || !tensor_map(b_op, p.rows_b, p.K, C::HB, &mb))
     return FP8Q_ERR_CUDA;
-  static int attr_done[64] = {0};
+  static std::atomic<int> attr_done[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+  if (dev >= 0 && dev < 64 && !attr_done[dev].load(std::memory_order_relaxed)) {
     if (cudaFuncSetAttribute(gemm_pair_kernel<BN, BW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return FP8Q_ERR_CUDA;
-    attr_done[dev] = 1;
+    attr_done[dev].store(1, std::memory_order_relaxed);
   }
   const int nc = pair_clusters<BN, BW>();
   if (nc < 1) return FP8Q_ERR_UNSUPPORTED;

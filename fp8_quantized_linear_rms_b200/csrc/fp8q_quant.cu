@@ -32,6 +32,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include <atomic>
+
 #include "fp8q_common.cuh"
 #include "fp8q_sm100.cuh"
 
@@ -678,14 +680,14 @@ fp8q_status launch_ring(const QuantParams& p, int T, int nteams, int nbuf, int s
                         cudaStream_t stream) {
   const int smem = nbuf * stride;
   auto kern = quant_ring_kernel<OP, PER_TOKEN, CH>;
-  static int attr_done[64] = {0};
+  static std::atomic<int> attr_done[64];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
-  if (!attr_done[dev]) {
+  if (!attr_done[dev].load(std::memory_order_relaxed)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemMax) != cudaSuccess)
       return FP8Q_ERR_CUDA;
-    attr_done[dev] = 1;
+    attr_done[dev].store(1, std::memory_order_relaxed);
   }
   int64_t grid = num_sms();
   if (grid > p.M) grid = p.M;
