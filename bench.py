@@ -55,7 +55,8 @@ def parse():
     ap.add_argument("--m", type=int, default=2048)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--sweep", default=None,
-                    help="per-op timing instead of the step: quant, gemm8b, decode32b, prefill32b, all")
+                    help="per-op timing instead of the step: quant, gemm8b, decode32b, prefill32b, "
+                         "all (GPU), or oracle (the CPU oracle, all host cores and one core)")
     ap.add_argument("--reps", type=int, default=50)
     return ap.parse_args()
 
@@ -460,6 +461,84 @@ def cpu_baseline_leg(args):
 
 
 # ------------------------------------------------------------------ per-op sweep
+def run_oracle_sweep(args):
+    """The CPU oracle, as it stands, per op on the config shapes, on every host
+    core and on one core (one child process each, OMP_NUM_THREADS set before the
+    oracle library loads).  Quant ops run on their full shapes; GEMMs on the
+    full shape for M <= 128 and on a 64-row slice above, extrapolated linearly
+    in M (marked "extrapolated").  One JSON line per case."""
+    if os.environ.get("FP8Q_ORACLE_SWEEP_CHILD") != "1":
+        for threads in (os.cpu_count() or 1, 1):
+            env = dict(os.environ, OMP_NUM_THREADS=str(threads), OPENBLAS_NUM_THREADS=str(threads),
+                       FP8Q_ORACLE_SWEEP_CHILD="1")
+            r = subprocess.run([sys.executable, os.path.abspath(__file__), "--sweep", "oracle"],
+                               env=env, stdout=sys.stdout, stderr=sys.stderr)
+            if r.returncode != 0:
+                return r.returncode
+        return 0
+
+    import numpy as np
+
+    import fp8q_inputs as inp
+    import oracle
+
+    threads = int(os.environ["OMP_NUM_THREADS"])
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    def emit(d):
+        d.update({"impl": "oracle", "threads": threads})
+        print(json.dumps(d), flush=True)
+
+    w = {h: inp.rms_weight_bf16(2001, h) for h in (4096, 5120)}
+    for M in (2048, 8192):
+        for op, L in (("group_quant", 4096), ("rmsnorm_quant", 4096), ("rmsnorm_quant", 5120),
+                      ("silu_mul_quant", 12288), ("silu_mul_quant", 25600)):
+            x = inp.heavy_tailed_bf16(3000 + L, M, 2 * L if op == "silu_mul_quant" else L)
+            for g in (L, 128):
+                if op == "group_quant":
+                    t = timed(lambda: oracle.group_quant(x, g))
+                    nbytes = M * (2 * L + L + 4 * (L // g))
+                elif op == "rmsnorm_quant":
+                    t = timed(lambda: oracle.rmsnorm_quant(x, w[L], EPS, g))
+                    nbytes = M * (2 * L + L + 4 * (L // g)) + 2 * L
+                else:
+                    t = timed(lambda: oracle.silu_mul_quant(x, g))
+                    nbytes = M * (4 * L + L + 4 * (L // g))
+                emit({"op": op, "M": M, "L": L, "group": g, "s": round(t, 4),
+                      "GB/s": round(nbytes / t / 1e9, 3)})
+            del x
+
+    s8, s32 = inp.linear_shapes(inp.QWEN3_8B), inp.linear_shapes(inp.QWEN3_32B)
+    cases = ([("qwen3-8b", s8, L, M, False) for L in ("gate_up", "down") for M in (1, 16, 128, 2048)]
+             + [("qwen3-8b", s8, L, M, True) for L in ("qkv", "o", "gate_up", "down")
+                for M in (1, 128, 2048)]
+             + [("qwen3-32b", s32, L, 1, True) for L in ("qkv", "o", "gate_up", "down")]
+             + [("qwen3-32b", s32, L, 8192, bw) for bw in (False, True)
+                for L in ("qkv", "o", "gate_up", "down")])
+    for model, sh, layer, M, bw in cases:
+        K, N = sh[layer]
+        rows = min(M, 64)
+        a = inp.random_e4m3_codes(11, (rows, K))
+        b = inp.random_e4m3_codes(12, (N, K))
+        if bw:
+            sa, sb = inp.random_scales(13, (rows, K // 128)), inp.random_scales(14, (N // 128, K // 128))
+            t = timed(lambda: oracle.scaled_mm_blockwise(a, b, sa, sb))
+        else:
+            sa, sb = inp.random_scales(13, (rows,)), inp.random_scales(14, (N,))
+            t = timed(lambda: oracle.scaled_mm(a, b, sa, sb))
+        t *= M / rows
+        emit({"op": "scaled_mm_blockwise" if bw else "scaled_mm", "shape": f"{model} {layer}",
+              "M": M, "N": N, "K": K, "s": round(t, 4),
+              "TFLOP/s": round(2.0 * M * N * K / t / 1e12, 6), "extrapolated": rows < M,
+              "rows_timed": rows})
+        del a, b
+    return 0
+
+
 def run_sweep(args):
     """Time every op of the path on the config shapes, one JSON line per case:
     device time per launch (CUDA events, median of --reps, L2 flushed before each
@@ -644,6 +723,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.sweep == "oracle":
+        return run_oracle_sweep(args)
     if args.sweep:
         return run_sweep(args)
     if args.impl == "reference":
