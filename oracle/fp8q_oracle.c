@@ -15,7 +15,7 @@
  *   code   q = e4m3fn(fl32(x / s)), round to nearest even, saturating at +-448
  *   groups contiguous 1x128 chunks of a row, or the whole row (per token)
  *   GEMM   y = bf16(sum_k (qa*sa)(qb*sb)), fp32 scales, bf16 output
- * Readings where nothing fixes a step (each one listed in the design doc):
+ * Readings where nothing fixes a step:
  *   - RMSNorm: r = 1/sqrt(mean(x^2) + eps) in fp64; n = bf16(x*r); y = bf16(n*w).
  *   - SiLU*mul: gate = first half of the row, up = second half;
  *     y = bf16(silu(gate)*up), one rounding of the fp64 value.
