@@ -122,6 +122,9 @@ class ClockSampler:
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            if getattr(self, "f", None):
+                self.f.close()
+                os.remove(self.path)
 
     def stop(self):
         if self.proc is None:
