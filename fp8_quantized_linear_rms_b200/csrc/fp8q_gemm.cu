@@ -1254,6 +1254,14 @@ fp8q_status check_gemm(const void* a_q, const void* b_q, const void* sa, const v
   return FP8Q_OK;
 }
 
+// The blockwise kernels address activation scales with 32-bit element
+// offsets (m * as_stride_m + kb * as_stride_kb, kb running a few blocks past
+// the last one): every such offset must stay below 2^31.
+bool scale_offsets_fit(int64_t M, int64_t K, int64_t as_stride_m, int64_t as_stride_kb) {
+  const int64_t last = (M - 1) * as_stride_m + (K / 128 + 8) * as_stride_kb;
+  return last < (1LL << 31);
+}
+
 }  // namespace
 }  // namespace fp8q
 
@@ -1327,6 +1335,7 @@ extern "C" fp8q_status fp8q_scaled_mm_blockwise(const void* a_q, const void* b_q
   if (N % 128 != 0 || K % 128 != 0 || as_stride_m < 0 || as_stride_kb < 0)
     return FP8Q_ERR_INVALID_ARG;
   if (M == 0) return FP8Q_OK;
+  if (!scale_offsets_fit(M, K, as_stride_m, as_stride_kb)) return FP8Q_ERR_INVALID_ARG;
   const fp8q_gemm_variant v = pick_variant(M, N, K, 1);
   if (!variant_supported(v, 1)) return FP8Q_ERR_UNSUPPORTED;
   const Plan pl = make_plan(M, N, K, 1, v);
@@ -1382,6 +1391,7 @@ extern "C" fp8q_status fp8q_scaled_mm_blockwise_noalloc(const void* a_q, const v
   if (N % 128 != 0 || K % 128 != 0 || as_stride_m < 0 || as_stride_kb < 0)
     return FP8Q_ERR_INVALID_ARG;
   if (M == 0) return FP8Q_OK;
+  if (!scale_offsets_fit(M, K, as_stride_m, as_stride_kb)) return FP8Q_ERR_INVALID_ARG;
   bool forced = false;
   fp8q_gemm_variant v = pick_variant(M, N, K, 1, &forced);
   if (!variant_supported(v, 1)) return FP8Q_ERR_UNSUPPORTED;

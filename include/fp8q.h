@@ -164,7 +164,9 @@ FP8Q_API fp8q_status fp8q_scaled_mm(const void* a_q, const void* b_q, const floa
  *   P_kb = fp32 sum over k in [128 kb, 128 kb + 128) of qa[m, k] * qb[n, k]
  *
  *   a_scale  fp32, one scale per 1x128 group of A: sa[m, kb] at
- *            a_scale[m*as_stride_m + kb*as_stride_kb]
+ *            a_scale[m*as_stride_m + kb*as_stride_kb]; strides >= 0 and
+ *            (M-1)*as_stride_m + (K/128+8)*as_stride_kb < 2^31 (else
+ *            FP8Q_ERR_INVALID_ARG; any scale array that fits in memory does)
  *   b_scale  fp32 [N/128, K/128] row-major, one scale per 128x128 block of B
  *   N and K multiples of 128; other arguments as in fp8q_scaled_mm, with
  *   fp8q_workspace_bytes(M, N, K, 1).

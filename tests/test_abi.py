@@ -51,6 +51,11 @@ def test_invalid_arguments_rejected_before_launch():
                                       None) == fq.ERR_INVALID_ARG
     assert L.fp8q_scaled_mm_blockwise(fake, fake, fake, 2, 1, fake, 4, 192, 256, fake, 192, None, 0,
                                       None) == fq.ERR_INVALID_ARG
+    # activation-scale strides whose offsets leave the 32-bit range
+    assert L.fp8q_scaled_mm_blockwise(fake, fake, fake, 1 << 30, 1, fake, 4, 128, 256, fake, 128, None,
+                                      0, None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_scaled_mm_blockwise_noalloc(fake, fake, fake, 1, 1 << 29, fake, 4, 128, 256, fake,
+                                              128, None) == fq.ERR_INVALID_ARG
 
 
 def test_zero_rows_is_a_noop_without_pointers():
