@@ -61,10 +61,13 @@ def _load():
         lib.oracle_e4m3_decode_array.argtypes = [P, i64, P]
         lib.oracle_bf16_round_array.argtypes = [P, i64, P]
         lib.oracle_scale_array.argtypes = [P, i64, ctypes.c_int, P]
+        lib.oracle_e8m0_encode_array.argtypes = [P, i64, P]
+        lib.oracle_e8m0_decode_array.argtypes = [P, i64, P]
         for f in ("oracle_group_quant", "oracle_rmsnorm_quant", "oracle_silu_mul_quant",
                   "oracle_scaled_mm_rows", "oracle_scaled_mm_blockwise_rows",
                   "oracle_e4m3_encode_array", "oracle_e4m3_decode_array",
-                  "oracle_bf16_round_array", "oracle_scale_array"):
+                  "oracle_bf16_round_array", "oracle_scale_array", "oracle_e8m0_encode_array",
+                  "oracle_e8m0_decode_array"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -112,6 +115,30 @@ def scale(amax, ue8m0: bool = False) -> np.ndarray:
     return out
 
 
+def e8m0_encode(s) -> np.ndarray:
+    """E8M0 bytes of power-of-two fp32 scales (255 for anything that is not a
+    power of two in [2^-127, 2^127])."""
+    s = _c(s, np.float32)
+    out = np.empty(s.shape, np.uint8)
+    _load().oracle_e8m0_encode_array(_ptr(s), s.size, _ptr(out))
+    return out
+
+
+def e8m0_decode(b) -> np.ndarray:
+    """Values 2^(b - 127) of E8M0 bytes (NaN for 255), as float64."""
+    b = _c(b, np.uint8)
+    out = np.empty(b.shape, np.float64)
+    _load().oracle_e8m0_decode_array(_ptr(b), b.size, _ptr(out))
+    return out
+
+
+def _packed(res, ue8m0):
+    """For ue8m0 == "packed": the UE8M0 scales as E8M0 bytes."""
+    if ue8m0 != "packed":
+        return res
+    return (res[0], e8m0_encode(res[1])) + tuple(res[2:])
+
+
 # ---------------------------------------------------------------- quant ops
 def _quant_out(M, L, g, want_y):
     q = np.empty((M, L), np.uint8)
@@ -134,8 +161,9 @@ def group_quant(x_bits: np.ndarray, group_size: int, ue8m0: bool = False, want_y
     M, K = x.shape
     _check_group(K, group_size)
     q, s, y = _quant_out(M, K, group_size, want_y)
-    _load().oracle_group_quant(_ptr(x), M, K, K, group_size, int(ue8m0), _ptr(q), _ptr(s), _ptr(y))
-    return (q, s, y) if want_y else (q, s)
+    _load().oracle_group_quant(_ptr(x), M, K, K, group_size, int(bool(ue8m0)), _ptr(q), _ptr(s),
+                               _ptr(y))
+    return _packed((q, s, y) if want_y else (q, s), ue8m0)
 
 
 def rmsnorm_quant(x_bits, w_bits, eps: float, group_size: int, ue8m0: bool = False,
@@ -148,8 +176,8 @@ def rmsnorm_quant(x_bits, w_bits, eps: float, group_size: int, ue8m0: bool = Fal
     _check_group(H, group_size)
     q, s, y = _quant_out(M, H, group_size, want_y)
     _load().oracle_rmsnorm_quant(_ptr(x), _ptr(w), ctypes.c_float(eps), M, H, H, group_size,
-                                 int(ue8m0), _ptr(q), _ptr(s), _ptr(y))
-    return (q, s, y) if want_y else (q, s)
+                                 int(bool(ue8m0)), _ptr(q), _ptr(s), _ptr(y))
+    return _packed((q, s, y) if want_y else (q, s), ue8m0)
 
 
 def silu_mul_quant(x_bits, group_size: int, ue8m0: bool = False, want_y: bool = False):
@@ -163,9 +191,9 @@ def silu_mul_quant(x_bits, group_size: int, ue8m0: bool = False, want_y: bool = 
     I = I2 // 2
     _check_group(I, group_size)
     q, s, y = _quant_out(M, I, group_size, want_y)
-    _load().oracle_silu_mul_quant(_ptr(x), M, I, I2, group_size, int(ue8m0), _ptr(q), _ptr(s),
-                                  _ptr(y))
-    return (q, s, y) if want_y else (q, s)
+    _load().oracle_silu_mul_quant(_ptr(x), M, I, I2, group_size, int(bool(ue8m0)), _ptr(q),
+                                  _ptr(s), _ptr(y))
+    return _packed((q, s, y) if want_y else (q, s), ue8m0)
 
 
 # ---------------------------------------------------------------------- GEMMs
@@ -219,3 +247,11 @@ def scaled_mm_blockwise(a_q, b_q, sa, sb, rows=None):
     _load().oracle_scaled_mm_blockwise_rows(_ptr(a), _ptr(b), _ptr(sa), _ptr(sb), M, N, K,
                                             _ptr(rows), rows.size, _ptr(y), _ptr(ad))
     return y, ad
+
+
+def scaled_mm_blockwise_e8m0(a_q, b_q, sa_e8m0, sb_e8m0, rows=None):
+    """scaled_mm_blockwise with E8M0 scale bytes: sa [M, K/128], sb [N/128, K/128]
+    (uint8), each byte b standing for the scale 2^(b - 127)."""
+    sa = e8m0_decode(sa_e8m0).astype(np.float32)
+    sb = e8m0_decode(sb_e8m0).astype(np.float32)
+    return scaled_mm_blockwise(a_q, b_q, sa, sb, rows)

@@ -121,6 +121,29 @@ float oracle_scale(float amax, int ue8m0)
     return s;
 }
 
+/* E8M0 ("UE8M0"): an 8-bit unsigned biased exponent, bias 127, no sign and no
+ * mantissa; byte b stands for 2^(b - 127); b = 255 is NaN.  It is the packed
+ * storage of a power-of-two scale: the exponent byte that the FP8 GEMM pages'
+ * B200 path needs ("Helion in vLLM", section "Practical limits": UE8M0 scales
+ * for DeepGEMM on B200).  Encode takes a scale that must be a power of two
+ * in [2^-127, 2^127] and returns its byte; anything else gives 255. */
+uint8_t oracle_e8m0_encode(float s)
+{
+    if (!(s > 0.0f) || isinf(s)) return 0xFF;
+    int e2;
+    double f = frexp((double)s, &e2);            /* s = f * 2^e2, f in [0.5, 1) */
+    if (f != 0.5) return 0xFF;                   /* not a power of two */
+    int e = e2 - 1;                              /* s = 2^e */
+    if (e < -127 || e > 127) return 0xFF;
+    return (uint8_t)(e + 127);
+}
+
+double oracle_e8m0_decode(uint8_t b)
+{
+    if (b == 0xFF) return NAN;
+    return ldexp(1.0, (int)b - 127);
+}
+
 /* Quantize L values of one group: scale from the group's amax, then codes. */
 static void quantize_group(const float* v, int64_t L, int ue8m0, uint8_t* q, float* s_out)
 {
@@ -307,4 +330,14 @@ void oracle_bf16_round_array(const double* v, int64_t n, float* out)
 void oracle_scale_array(const float* amax, int64_t n, int ue8m0, float* out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_scale(amax[i], ue8m0);
+}
+
+void oracle_e8m0_encode_array(const float* s, int64_t n, uint8_t* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e8m0_encode(s[i]);
+}
+
+void oracle_e8m0_decode_array(const uint8_t* b, int64_t n, double* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e8m0_decode(b[i]);
 }

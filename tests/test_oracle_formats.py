@@ -112,3 +112,63 @@ def test_scale_properties(ue8m0):
         m, _ = np.frexp(s)
         assert np.all(m == 0.5)                       # powers of two
         assert np.all(s >= base) and np.all(s < 2 * base)
+
+
+# ------------------------------------------------------------------ E8M0
+def test_e8m0_decode_all_bytes_vs_ml_dtypes():
+    # Every byte, against an independent library's E8M0 type (2^(b-127), 255 = NaN).
+    b = np.arange(256, dtype=np.uint8)
+    ref = b.view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    got = oracle.e8m0_decode(b)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    np.testing.assert_array_equal(got[:255], ref[:255])
+    assert got[127] == 1.0 and got[0] == 2.0 ** -127 and got[254] == 2.0 ** 127
+
+
+def test_e8m0_encode_powers_of_two_and_rejects():
+    # Every power of two an fp32 holds in [2^-126, 2^127] (fp32 normals; 2^-127 is an
+    # fp32 subnormal, also a power of two) encodes to its exponent + 127, as the
+    # library's cast does; anything that is not a power of two gives 255.
+    k = np.arange(-127, 128)
+    s = np.ldexp(np.float32(1.0), k).astype(np.float32)
+    got = oracle.e8m0_encode(s)
+    np.testing.assert_array_equal(got, (k + 127).astype(np.uint8))
+    np.testing.assert_array_equal(got, s.astype(ml_dtypes.float8_e8m0fnu).view(np.uint8))
+    bad = np.array([0.0, -1.0, 3.0, 1.5, np.inf, np.nan, 2.0 ** -128, 0.75], np.float32)
+    np.testing.assert_array_equal(oracle.e8m0_encode(bad), 0xFF)
+
+
+@pytest.mark.parametrize("op", ["group", "rms", "silu"])
+def test_packed_ue8m0_scales_are_the_ue8m0_exponents(op):
+    # The packed mode stores the byte of the UE8M0 scale: same codes as ue8m0=1,
+    # and every byte decodes to exactly the fp32 power-of-two scale.
+    import fp8q_inputs as inp
+    x = inp.heavy_tailed_bf16(31, 9, 512)
+    w = inp.rms_weight_bf16(32, 512)
+    for g in (128, 512):
+        if op == "group":
+            q1, s1 = oracle.group_quant(x, g, True)
+            qp, sp = oracle.group_quant(x, g, "packed")
+        elif op == "rms":
+            q1, s1 = oracle.rmsnorm_quant(x, w, 1e-6, g, True)
+            qp, sp = oracle.rmsnorm_quant(x, w, 1e-6, g, "packed")
+        else:
+            xs = inp.heavy_tailed_bf16(33, 9, 1024)
+            q1, s1 = oracle.silu_mul_quant(xs, g, True)
+            qp, sp = oracle.silu_mul_quant(xs, g, "packed")
+        assert sp.dtype == np.uint8 and sp.shape == s1.shape
+        np.testing.assert_array_equal(qp, q1)
+        np.testing.assert_array_equal(sp.view(ml_dtypes.float8_e8m0fnu).astype(np.float32), s1)
+
+
+def test_packed_ue8m0_hand_cases():
+    # amax 448 -> s = 1 -> byte 127; amax 1 -> 1/448 rounds up to 2^-8 -> 119;
+    # amax 0 -> floored 1e-10/448 ~ 2^-42.03 rounds up to 2^-42 -> 85;
+    # amax 3.5 -> 3.5/448 = 2^-7 exactly -> kept -> 120.
+    import fp8q_inputs as inp
+    rows = np.zeros((4, 128))
+    rows[0, 5] = 448.0
+    rows[1, 7] = -1.0
+    rows[3, 0] = 3.5
+    _, sp = oracle.group_quant(inp.to_bf16_bits(rows), 128, "packed")
+    np.testing.assert_array_equal(sp.reshape(-1), np.array([127, 119, 85, 120], np.uint8))

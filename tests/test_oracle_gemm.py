@@ -97,3 +97,18 @@ def test_row_subset_matches_full():
     ys, ads = oracle.scaled_mm(a, b, sa, sb, rows)
     np.testing.assert_array_equal(ys, y[rows])
     np.testing.assert_array_equal(ads, ad[rows])
+
+
+@pytest.mark.parametrize("M,N,K", [(2, 128, 256), (3, 256, 384)])
+def test_scaled_mm_blockwise_e8m0_exact_rationals(M, N, K):
+    # E8M0 scale bytes decoded by an independent library (ml_dtypes) into the
+    # exact-rational GEMM must agree with the oracle's E8M0 entry.
+    import ml_dtypes
+    a = inp.random_e4m3_codes(M + 7 * K, (M, K))
+    b = inp.random_e4m3_codes(N + 5 * K, (N, K))
+    g = np.random.default_rng(M + N)
+    sa = g.integers(100, 140, size=(M, K // 128)).astype(np.uint8)
+    sb = g.integers(110, 130, size=(N // 128, K // 128)).astype(np.uint8)
+    y, ad = oracle.scaled_mm_blockwise_e8m0(a, b, sa, sb)
+    dec = lambda t: t.view(ml_dtypes.float8_e8m0fnu).astype(np.float32)
+    _close_to_exact(y, ad, exact.scaled_mm_blockwise_exact(a, b, dec(sa), dec(sb)))
