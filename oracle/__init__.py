@@ -54,6 +54,8 @@ def _load():
         lib.oracle_rmsnorm_quant.argtypes = [P, P, ctypes.c_float, i64, i64, i64, i64,
                                              ctypes.c_int, P, P, P]
         lib.oracle_silu_mul_quant.argtypes = [P, i64, i64, i64, i64, ctypes.c_int, P, P, P]
+        lib.oracle_add_rmsnorm_quant.argtypes = [P, P, P, ctypes.c_float, i64, i64, i64,
+                                                 ctypes.c_int, P, P, P, P]
         lib.oracle_scaled_mm_rows.argtypes = [P, P, P, ctypes.c_int, P, ctypes.c_int, i64, i64,
                                               i64, P, i64, P, P]
         lib.oracle_scaled_mm_blockwise_rows.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, P]
@@ -64,6 +66,7 @@ def _load():
         lib.oracle_e8m0_encode_array.argtypes = [P, i64, P]
         lib.oracle_e8m0_decode_array.argtypes = [P, i64, P]
         for f in ("oracle_group_quant", "oracle_rmsnorm_quant", "oracle_silu_mul_quant",
+                  "oracle_add_rmsnorm_quant",
                   "oracle_scaled_mm_rows", "oracle_scaled_mm_blockwise_rows",
                   "oracle_e4m3_encode_array", "oracle_e4m3_decode_array",
                   "oracle_bf16_round_array", "oracle_scale_array", "oracle_e8m0_encode_array",
@@ -178,6 +181,25 @@ def rmsnorm_quant(x_bits, w_bits, eps: float, group_size: int, ue8m0: bool = Fal
     _load().oracle_rmsnorm_quant(_ptr(x), _ptr(w), ctypes.c_float(eps), M, H, H, group_size,
                                  int(bool(ue8m0)), _ptr(q), _ptr(s), _ptr(y))
     return _packed((q, s, y) if want_y else (q, s), ue8m0)
+
+
+def add_rmsnorm_quant(x_bits, res_bits, w_bits, eps: float, group_size: int, ue8m0=False,
+                      want_y: bool = False):
+    """Residual add + RMSNorm quant: h = bf16(x + residual) (returned as the
+    updated residual), then rmsnorm_quant(h).  Returns (q, s, residual_out[, y])."""
+    x = _c(x_bits, np.uint16)
+    r = _c(res_bits, np.uint16)
+    w = _c(w_bits, np.uint16)
+    M, H = x.shape
+    assert r.shape == (M, H) and w.shape == (H,)
+    _check_group(H, group_size)
+    q, s, y = _quant_out(M, H, group_size, want_y)
+    r_out = np.empty((M, H), np.uint16)
+    _load().oracle_add_rmsnorm_quant(_ptr(x), _ptr(r), _ptr(w), ctypes.c_float(eps), M, H,
+                                     group_size, int(bool(ue8m0)), _ptr(q), _ptr(s), _ptr(r_out),
+                                     _ptr(y))
+    res = (q, s, r_out, y) if want_y else (q, s, r_out)
+    return _packed(res, ue8m0)
 
 
 def silu_mul_quant(x_bits, group_size: int, ue8m0: bool = False, want_y: bool = False):

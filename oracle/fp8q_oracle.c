@@ -210,6 +210,29 @@ void oracle_rmsnorm_quant(const uint16_t* x, const uint16_t* w, float eps, int64
     }
 }
 
+/* Residual-add variant of the RMSNorm quant (the fusion "on either side of
+ * the path" that continues the pages' call-count reduction, "Helion in vLLM",
+ * section "Kernels integrated into vLLM").  Reading: the fused op feeds the
+ * norm what the unfused chain would -- the residual stream is kept in the
+ * model dtype, so h = bf16(x + residual) with one rounding of the exact sum;
+ * h is written to res_out and then RMSNorm-quantized exactly as
+ * oracle_rmsnorm_quant does. */
+void oracle_add_rmsnorm_quant(const uint16_t* x, const uint16_t* res, const uint16_t* w, float eps,
+                              int64_t M, int64_t H, int64_t g, int ue8m0, uint8_t* q, float* s,
+                              uint16_t* res_out, float* y_out)
+{
+    uint16_t* h = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(M * H));
+    for (int64_t i = 0; i < M * H; ++i) {
+        float v = oracle_bf16_round(bf16_bits_value(x[i]) + bf16_bits_value(res[i]));
+        uint32_t u;
+        memcpy(&u, &v, 4);
+        h[i] = (uint16_t)(u >> 16);              /* v is a bf16 value: its upper half */
+    }
+    oracle_rmsnorm_quant(h, w, eps, M, H, H, g, ue8m0, q, s, y_out);
+    memcpy(res_out, h, sizeof(uint16_t) * (size_t)(M * H));
+    free(h);
+}
+
 /* silu_and_mul_dynamic_per_token_quant (g == I) and silu_and_mul_per_block_quant
  * (g == 128) ("Helion in vLLM", "Kernels integrated into vLLM", items 3, 7).
  * Input row [gate(I) | up(I)]; silu(t) = t / (1 + e^-t). */

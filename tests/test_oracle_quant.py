@@ -163,3 +163,54 @@ def test_fused_ops_quantize_their_y(fn, ue8m0):
     q2, s2 = oracle.group_quant(inp.to_bf16_bits(y), 128, ue8m0)
     np.testing.assert_array_equal(q, q2)
     np.testing.assert_array_equal(s, s2)
+
+
+# ------------------------------------------------------------ residual add + RMSNorm quant
+def test_add_rmsnorm_quant_reduces_to_rmsnorm_quant():
+    # residual 0: the sum is x itself, so everything equals rmsnorm_quant(x)
+    x = inp.heavy_tailed_bf16(91, 5, 512)
+    w = inp.rms_weight_bf16(92, 512)
+    zero = np.zeros_like(x)
+    for g in (128, 512):
+        for ue in (False, True):
+            q, s, r = oracle.add_rmsnorm_quant(x, zero, w, 1e-6, g, ue)
+            q0, s0 = oracle.rmsnorm_quant(x, w, 1e-6, g, ue)
+            np.testing.assert_array_equal(r, x)
+            np.testing.assert_array_equal(q, q0)
+            np.testing.assert_array_equal(s, s0)
+
+
+def test_add_rmsnorm_quant_cancelling_residual():
+    # residual = -x: the sum is +0 everywhere -> floored scale, all codes 0
+    x = inp.heavy_tailed_bf16(93, 3, 256)
+    q, s, r = oracle.add_rmsnorm_quant(x, x ^ np.uint16(0x8000), inp.rms_weight_bf16(94, 256), 1e-6, 128)
+    assert np.all((r & 0x7FFF) == 0)
+    assert np.all(q & 0x7F == 0)
+    np.testing.assert_array_equal(s, np.float32(np.float32(1e-10) / np.float32(448.0)))
+
+
+def test_add_rmsnorm_quant_sum_rounding_hand_cases():
+    # bf16 has 8 significant bits (ulp(1) = 2^-7); ties of the sum go to the even significand:
+    #   1 + 2^-8          halfway between 1 and 1 + 2^-7          -> 1.0
+    #   1 + 3*2^-8        halfway between 1 + 2^-7 and 1 + 2^-6   -> 1 + 2^-6
+    #   1 + 2^-8 + 2^-15  just above the first midpoint           -> 1 + 2^-7
+    x = inp.to_bf16_bits(np.array([[1.0, 1.0, 1.0] + [0.0] * 125]))
+    r = inp.to_bf16_bits(np.array([[2.0 ** -8, 3 * 2.0 ** -8, 2.0 ** -8 + 2.0 ** -15] + [0.0] * 125]))
+    _, _, h = oracle.add_rmsnorm_quant(x, r, inp.to_bf16_bits(np.ones(128)), 0.0, 128)
+    got = inp.bf16_bits_to_f32(h[0, :3])
+    np.testing.assert_array_equal(got, np.array([1.0, 1.0 + 2.0 ** -6, 1.0 + 2.0 ** -7], np.float32))
+
+
+def test_add_rmsnorm_quant_matches_the_unfused_chain():
+    # the fused op equals: torch's bf16 add (round to nearest even), then rmsnorm_quant
+    import torch
+    x = inp.heavy_tailed_bf16(95, 7, 1024)
+    r = inp.normal_bf16(96, (7, 1024), std=4.0)
+    w = inp.rms_weight_bf16(97, 1024)
+    tb = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)
+    h = (tb(x) + tb(r)).view(torch.int16).numpy().view(np.uint16)
+    q, s, r_out = oracle.add_rmsnorm_quant(x, r, w, 1e-6, 128)
+    q0, s0 = oracle.rmsnorm_quant(h, w, 1e-6, 128)
+    np.testing.assert_array_equal(r_out, h)
+    np.testing.assert_array_equal(q, q0)
+    np.testing.assert_array_equal(s, s0)
