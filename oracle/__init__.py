@@ -63,6 +63,13 @@ def _load():
         lib.oracle_e4m3_decode_array.argtypes = [P, i64, P]
         lib.oracle_bf16_round_array.argtypes = [P, i64, P]
         lib.oracle_scale_array.argtypes = [P, i64, ctypes.c_int, P]
+        lib.oracle_int8_quant_rows.argtypes = [P, i64, i64, i64, P, P]
+        lib.oracle_scaled_mm_i8_rows.argtypes = [P, P, P, ctypes.c_int, P, ctypes.c_int, i64, i64,
+                                                 i64, P, i64, P, P]
+        lib.oracle_int8_encode.argtypes = [ctypes.c_float]
+        lib.oracle_int8_encode.restype = ctypes.c_int8
+        lib.oracle_int8_scale.argtypes = [ctypes.c_float]
+        lib.oracle_int8_scale.restype = ctypes.c_float
         lib.oracle_e8m0_encode_array.argtypes = [P, i64, P]
         lib.oracle_e8m0_decode_array.argtypes = [P, i64, P]
         for f in ("oracle_group_quant", "oracle_rmsnorm_quant", "oracle_silu_mul_quant",
@@ -70,7 +77,7 @@ def _load():
                   "oracle_scaled_mm_rows", "oracle_scaled_mm_blockwise_rows",
                   "oracle_e4m3_encode_array", "oracle_e4m3_decode_array",
                   "oracle_bf16_round_array", "oracle_scale_array", "oracle_e8m0_encode_array",
-                  "oracle_e8m0_decode_array"):
+                  "oracle_e8m0_decode_array", "oracle_int8_quant_rows", "oracle_scaled_mm_i8_rows"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -277,3 +284,59 @@ def scaled_mm_blockwise_e8m0(a_q, b_q, sa_e8m0, sb_e8m0, rows=None):
     sa = e8m0_decode(sa_e8m0).astype(np.float32)
     sb = e8m0_decode(sb_e8m0).astype(np.float32)
     return scaled_mm_blockwise(a_q, b_q, sa, sb, rows)
+
+
+# --------------------------------------------------------------------- W8A8_INT8
+def int8_quantize(y, group_size: int):
+    """int8 codes and fp32 scales of fp32 values y [M, L] in groups of g:
+    s = fl32(max(amax, 1e-10)/127), q = sat_int8(RNE(fl32(y/s)))."""
+    y = _c(y, np.float32)
+    M, L = y.shape
+    _check_group(L, group_size)
+    q = np.empty((M, L), np.int8)
+    s = np.empty((M, L // group_size), np.float32)
+    _load().oracle_int8_quant_rows(_ptr(y), M, L, group_size, _ptr(q), _ptr(s))
+    return q, s
+
+
+def int8_encode_scalar(v: float) -> int:
+    return int(_load().oracle_int8_encode(ctypes.c_float(v)))
+
+
+def group_quant_i8(x_bits, group_size: int):
+    """W8A8_INT8 per-token (g = K) / per-group quant of bf16 x: (q int8, s fp32)."""
+    _, _, y = group_quant(x_bits, group_size, False, want_y=True)
+    return int8_quantize(y, group_size)
+
+
+def rmsnorm_quant_i8(x_bits, w_bits, eps: float, group_size: int):
+    """RMSNorm (same reading as rmsnorm_quant) followed by int8 quant."""
+    _, _, y = rmsnorm_quant(x_bits, w_bits, eps, group_size, False, want_y=True)
+    return int8_quantize(y, group_size)
+
+
+def silu_mul_quant_i8(x_bits, group_size: int):
+    """SiLU*mul (same reading as silu_mul_quant) followed by int8 quant."""
+    _, _, y = silu_mul_quant(x_bits, group_size, False, want_y=True)
+    return int8_quantize(y, group_size)
+
+
+def scaled_mm_i8(a_q, b_q, sa, sb, rows=None):
+    """fp64 reference of the int8 scaled_mm for the listed rows of A: the
+    integer dot products exact, then times sa (per token or per tensor) and
+    sb (per channel or per tensor).  Returns (y_ref, absdot)."""
+    a = _c(a_q, np.int8)
+    b = _c(b_q, np.int8)
+    M, K = a.shape
+    N, K2 = b.shape
+    assert K == K2
+    sa = _c(sa, np.float32).reshape(-1)
+    sb = _c(sb, np.float32).reshape(-1)
+    assert sa.size in (1, M) and sb.size in (1, N)
+    rows = _rows(M, rows)
+    y = np.empty((rows.size, N), np.float64)
+    ad = np.empty((rows.size, N), np.float64)
+    _load().oracle_scaled_mm_i8_rows(_ptr(a), _ptr(b), _ptr(sa), int(sa.size == M), _ptr(sb),
+                                     int(sb.size == N), M, N, K, _ptr(rows), rows.size, _ptr(y),
+                                     _ptr(ad))
+    return y, ad

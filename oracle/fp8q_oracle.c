@@ -364,3 +364,74 @@ void oracle_e8m0_decode_array(const uint8_t* b, int64_t n, double* out)
 {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_e8m0_decode(b[i]);
 }
+
+/* ------------------------------------------------------------------------ */
+/* W8A8_INT8 ("Helion linear backend" (aihirek.info), section "Autotuning    */
+/* selects the variant": the W8A8_INT8 scheme next to FP8_Dynamic and        */
+/* Block_FP8).  The pages name the scheme only; the reading taken is the     */
+/* FP8 path's with int8 codes:                                               */
+/*   scale s = fl32(max(amax, 1e-10) / 127)      (IEEE fp32 division)         */
+/*   code  q = int8(RNE(fl32(y / s))), saturated to [-128, 127]              */
+/*   GEMM  y = bf16(sa * sb * sum_k qa * qb), the sum exact in integers.     */
+/* ------------------------------------------------------------------------ */
+
+/* Nearest integer (ties to even) of an fp32 value, saturated to int8; NaN -> 0. */
+int8_t oracle_int8_encode(float v)
+{
+    if (isnan(v)) return 0;
+    double a = fabs((double)v);
+    double r = rne_integer(a);
+    if (v < 0) r = -r;
+    if (r > 127.0) r = 127.0;
+    if (r < -128.0) r = -128.0;
+    return (int8_t)r;
+}
+
+float oracle_int8_scale(float amax)
+{
+    return fmaxf(amax, 1e-10f) / 127.0f;         /* IEEE fp32 division */
+}
+
+/* Quantize M rows of L values (the values a producer op feeds the quantizer)
+ * in groups of g to int8 codes, scales s [M, L/g] row-major. */
+void oracle_int8_quant_rows(const float* y, int64_t M, int64_t L, int64_t g, int8_t* q, float* s)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t j = 0; j < L / g; ++j) {
+            const float* v = y + m * L + j * g;
+            float amax = 0.0f;
+            for (int64_t i = 0; i < g; ++i) {
+                float a = fabsf(v[i]);
+                if (a > amax) amax = a;
+            }
+            float sc = oracle_int8_scale(amax);
+            for (int64_t i = 0; i < g; ++i) q[m * L + j * g + i] = oracle_int8_encode(v[i] / sc);
+            s[m * (L / g) + j] = sc;
+        }
+    }
+}
+
+/* int8 scaled_mm: y_ref[m, n] = sa * sb * sum_k qa[m,k] qb[n,k] (the integer
+ * sum exact in int64), absdot = |sa sb| sum_k |qa qb|. */
+void oracle_scaled_mm_i8_rows(const int8_t* a, const int8_t* b, const float* sa, int a_per_token,
+                              const float* sb, int b_per_channel, int64_t M, int64_t N, int64_t K,
+                              const int64_t* rows, int64_t nrows, double* y, double* absdot)
+{
+    (void)M;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t i = 0; i < nrows; ++i) {
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t m = rows[i];
+            int64_t acc = 0, aacc = 0;
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t t = (int64_t)a[m * K + k] * (int64_t)b[n * K + k];
+                acc += t;
+                aacc += t < 0 ? -t : t;
+            }
+            double sc = (double)(a_per_token ? sa[m] : sa[0]) * (double)(b_per_channel ? sb[n] : sb[0]);
+            y[i * N + n] = (double)acc * sc;
+            absdot[i * N + n] = (double)aacc * fabs(sc);
+        }
+    }
+}
