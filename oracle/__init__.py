@@ -70,6 +70,8 @@ def _load():
         lib.oracle_int8_encode.restype = ctypes.c_int8
         lib.oracle_int8_scale.argtypes = [ctypes.c_float]
         lib.oracle_int8_scale.restype = ctypes.c_float
+        lib.oracle_qk_norm_rope.argtypes = [P, i64, i64, i64, i64, i64, ctypes.c_float, P, P, P, P,
+                                            ctypes.c_int]
         lib.oracle_e8m0_encode_array.argtypes = [P, i64, P]
         lib.oracle_e8m0_decode_array.argtypes = [P, i64, P]
         for f in ("oracle_group_quant", "oracle_rmsnorm_quant", "oracle_silu_mul_quant",
@@ -77,7 +79,8 @@ def _load():
                   "oracle_scaled_mm_rows", "oracle_scaled_mm_blockwise_rows",
                   "oracle_e4m3_encode_array", "oracle_e4m3_decode_array",
                   "oracle_bf16_round_array", "oracle_scale_array", "oracle_e8m0_encode_array",
-                  "oracle_e8m0_decode_array", "oracle_int8_quant_rows", "oracle_scaled_mm_i8_rows"):
+                  "oracle_e8m0_decode_array", "oracle_int8_quant_rows", "oracle_scaled_mm_i8_rows",
+                  "oracle_qk_norm_rope"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -340,3 +343,24 @@ def scaled_mm_i8(a_q, b_q, sa, sb, rows=None):
                                      int(sb.size == N), M, N, K, _ptr(rows), rows.size, _ptr(y),
                                      _ptr(ad))
     return y, ad
+
+
+# --------------------------------------------------------------- fused_qk_norm_rope
+def qk_norm_rope(qkv_bits, hq: int, hk: int, hv: int, head_dim: int, eps: float, q_w_bits, k_w_bits,
+                 cos_sin, positions, is_neox: bool):
+    """Per-head RMSNorm of the q and k heads, then the rotary embedding at each
+    token's position; returns a new qkv (uint16 bf16 bits [T, (hq+hk+hv)*D]),
+    v heads unchanged.  cos_sin: fp32 [max_pos, D] = [cos (D/2) | sin (D/2)]."""
+    x = np.array(qkv_bits, dtype=np.uint16, copy=True, order="C")
+    T, L = x.shape
+    D = head_dim
+    assert L == (hq + hk + hv) * D and D % 2 == 0
+    qw = _c(q_w_bits, np.uint16)
+    kw = _c(k_w_bits, np.uint16)
+    cs = _c(cos_sin, np.float32)
+    pos = _c(positions, np.int64)
+    assert qw.shape == (D,) and kw.shape == (D,) and cs.shape[1] == D and pos.shape == (T,)
+    assert pos.size == 0 or (pos.min() >= 0 and pos.max() < cs.shape[0])
+    _load().oracle_qk_norm_rope(_ptr(x), T, L, hq, hk, D, ctypes.c_float(eps), _ptr(qw), _ptr(kw),
+                                _ptr(cs), _ptr(pos), int(bool(is_neox)))
+    return x

@@ -435,3 +435,56 @@ void oracle_scaled_mm_i8_rows(const int8_t* a, const int8_t* b, const float* sa,
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* fused_qk_norm_rope (vllm PR #44010 page, section "Code analysis": the op  */
+/* takes qkv, the q / k / v head counts, head_dim, eps, q_weight, k_weight,  */
+/* the rope cos_sin_cache, is_neox and positions; "Helion in vLLM", section  */
+/* "Kernels integrated into vLLM", item 4).  Reading taken (the pages print  */
+/* no arithmetic):                                                           */
+/*   qkv row t = [q heads (hq) | k heads (hk) | v heads (hv)], D each, bf16; */
+/*   every q and k head: the RMSNorm of this library over its D values       */
+/*     r = 1/sqrt(mean(x^2) + eps), n = bf16(x r), y = bf16(n w)             */
+/*   (w = q_weight or k_weight, [D]), then the rotary embedding at position  */
+/*   p = positions[t] with cos = cache[p][0 .. D/2), sin = cache[p][D/2 .. D) */
+/*   (fp32 cache), pairs (i, i + D/2) when is_neox, else (2i, 2i + 1):       */
+/*     out_a = bf16(y_a cos_i - y_b sin_i),  out_b = bf16(y_b cos_i + y_a sin_i) */
+/*   written back in place; v heads are left as they are.                    */
+/* ------------------------------------------------------------------------ */
+void oracle_qk_norm_rope(uint16_t* qkv, int64_t T, int64_t ld, int64_t hq, int64_t hk, int64_t D,
+                         float eps, const uint16_t* qw, const uint16_t* kw, const float* cos_sin,
+                         const int64_t* positions, int is_neox)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double* y = (double*)malloc(sizeof(double) * (size_t)D);
+        const float* cs = cos_sin + positions[t] * D;
+        for (int64_t h = 0; h < hq + hk; ++h) {
+            uint16_t* x = qkv + t * ld + h * D;
+            const uint16_t* w = h < hq ? qw : kw;
+            double ss = 0.0;
+            for (int64_t i = 0; i < D; ++i) {
+                double v = bf16_bits_value(x[i]);
+                ss += v * v;
+            }
+            double r = 1.0 / sqrt(ss / (double)D + (double)eps);
+            for (int64_t i = 0; i < D; ++i) {
+                double n = oracle_bf16_round(bf16_bits_value(x[i]) * r);
+                y[i] = oracle_bf16_round(n * bf16_bits_value(w[i]));
+            }
+            for (int64_t i = 0; i < D / 2; ++i) {
+                int64_t a = is_neox ? i : 2 * i;
+                int64_t b = is_neox ? i + D / 2 : 2 * i + 1;
+                double c = cs[i], sn = cs[D / 2 + i];
+                float oa = oracle_bf16_round(y[a] * c - y[b] * sn);
+                float ob = oracle_bf16_round(y[b] * c + y[a] * sn);
+                uint32_t ua, ub;
+                memcpy(&ua, &oa, 4);
+                memcpy(&ub, &ob, 4);
+                x[a] = (uint16_t)(ua >> 16);
+                x[b] = (uint16_t)(ub >> 16);
+            }
+        }
+        free(y);
+    }
+}
