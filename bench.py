@@ -2,26 +2,36 @@
 """Benchmark of the FP8 W8A8 linear path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--m M] [--impl reference]
+                    [--no-e8m0] [--sweep quant|gemm8b|decode32b|prefill32b|all|oracle]
 
-Workload: one Qwen3-8B-shaped MLP block (hidden 4096, intermediate 12288) on a
-batch of M tokens (default 2048), through both FP8 schemes.  One step runs every
-op of the path once:
-  per-token quant and 1x128-group quant of the block input x,
-  per-token chain:  rmsnorm_quant(g=H) -> scaled_mm gate_up [4096->24576]
-                    -> silu_mul_quant(g=I) -> scaled_mm down [12288->4096],
-  blockwise chain:  rmsnorm_quant(g=128) -> scaled_mm_blockwise gate_up
-                    -> silu_mul_quant(g=128) -> scaled_mm_blockwise down.
-x is heavy-tailed Student-t(3) with 1% outlier channels x20 (seeded); weights
-W ~ N(0, 0.02), quantized once per output channel / per 128x128 block.
+Workload: the linear stack of one Qwen3-32B-shaped decoder block in prefill
+(hidden 5120, intermediate 25600, 64 query / 8 kv heads of 128) on a batch of
+M = 8192 tokens, through both FP8 schemes.  One step runs, per scheme,
+    rmsnorm_quant(x)        -> scaled_mm qkv      [5120 -> 10240]
+    group_quant(attn)       -> scaled_mm o        [8192 -> 5120]
+    rmsnorm_quant(o out)    -> scaled_mm gate_up  [5120 -> 51200]
+    silu_mul_quant(gate_up) -> scaled_mm down     [25600 -> 5120]
+with per-token activation scales and per-channel weight scales (scaled_mm),
+then with 1x128 activation groups and 128x128 weight blocks
+(scaled_mm_blockwise, fp32 scales): 16 launches.  The attention output that
+feeds the o projection is a seeded stand-in (attention itself is not part of
+this path).  x is heavy-tailed Student-t(3) with 1% outlier channels x20,
+attn ~ N(0, 1) (seeded); weights W ~ N(0, 0.02), quantized once per output
+channel / per 128x128 block.
 
 `value` is whole-job TFLOP/s (GEMM FLOPs of all ranks / max-over-ranks device
-time), inputs resident in HBM; each timed step is bracketed by CUDA events and
-followed by an untimed L2 flush.  `e2e` is the same metric through the public
-API with each step's activations copied from pinned host memory and both of its
-outputs copied back inside the timed region, the copies on their own streams
-overlapping the neighbouring steps' kernels (double-buffered, as a serving loop
-runs); there the L2 flush before each step is inside the timed region.  `--impl reference` times the CPU oracle on a
-bounded sample of the same workload.
+time), inputs resident in HBM; each timed step is bracketed by CUDA events,
+every launch of the step is followed by an event (the per-kernel times), and
+an untimed 256 MiB write flushes L2 between steps.  `e2e` is the same metric
+through the public API with each step's inputs copied from pinned host memory
+and its two block outputs copied back inside the timed region, the copies on
+their own streams overlapping the neighbouring steps' kernels
+(double-buffered, as a serving loop runs).  `roofline` is the dominant kernel
+(the launch with the largest device time), `gemms` and `roofline_quant` every
+GEMM and quant launch against the measured peaks.  `e8m0_chain` times the
+blockwise stack again with packed UE8M0 scales and the block-scaled GEMM;
+`qk_norm_rope` times the attention-side fused op on the step's qkv output.
+`--impl reference` times the CPU oracle on a bounded sample of the workload.
 """
 from __future__ import annotations
 
@@ -31,50 +41,50 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-H, I = 4096, 12288
-METRIC = "FP8 quant+scaled_mm TFLOP/s (Qwen3-8B MLP block, per-token + blockwise)"
+# Qwen3-32B block: hidden, intermediate, attention width (64 heads x 128)
+H, I, ATT = 5120, 25600, 8192
+QKV = (64 + 2 * 8) * 128
+LAYERS = (("qkv", H, QKV), ("o", ATT, H), ("gate_up", H, 2 * I), ("down", I, H))   # (name, K, N)
+DEFAULT_M = 8192
+METRIC = "FP8 quant+scaled_mm TFLOP/s (Qwen3-32B prefill linear stack, per-token + blockwise)"
 EPS = 1e-6
-
-# DRAM bytes (read + write) of one launch of each gate_up GEMM, from one ncu
-# capture of the current kernel build (profiles/gemm_kernel_qwen3_8b_mlp_m2048.md);
-# set to None whenever the kernel changes until it is captured again.
-GATE_UP_BW_TRAFFIC = 170.9e6
-GATE_UP_PT_TRAFFIC = 172.1e6
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1500)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--m", type=int, default=2048)
+    ap.add_argument("--m", type=int, default=DEFAULT_M)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-e8m0", action="store_true", help="skip the E8M0 (UE8M0) chain")
+    ap.add_argument("--no-rope", action="store_true", help="skip timing fused_qk_norm_rope")
     ap.add_argument("--sweep", default=None,
                     help="per-op timing instead of the step: quant, gemm8b, decode32b, prefill32b, "
-                         "all (GPU), or oracle (the CPU oracle, all host cores and one core)")
+                         "e8m0, all (GPU), or oracle (the CPU oracle, all host cores and one core)")
     ap.add_argument("--reps", type=int, default=50)
     return ap.parse_args()
 
 
 def gemm_flops(M):
-    return 2 * (2 * M * H * 2 * I + 2 * M * I * H)     # two chains x (gate_up + down)
+    """GEMM FLOPs of one step: both schemes x the four layers."""
+    return 2 * sum(2 * M * N * K for _, K, N in LAYERS)
 
 
-def quant_bytes(M):
-    """Algorithmic HBM bytes of the six quant launches of one step: the bf16 input
-    read once, e4m3 codes and fp32 scales written once, the RMSNorm weight once."""
-    gq_tok = 2 * M * H + M * H + 4 * M
-    gq_grp = 2 * M * H + M * H + 4 * M * (H // 128)
-    rms_tok = 2 * M * H + M * H + 4 * M + 2 * H
-    rms_grp = 2 * M * H + M * H + 4 * M * (H // 128) + 2 * H
-    silu_tok = 4 * M * I + M * I + 4 * M
-    silu_grp = 4 * M * I + M * I + 4 * M * (I // 128)
-    return gq_tok + gq_grp + rms_tok + rms_grp + silu_tok + silu_grp
+def quant_bytes(op, M, L, g):
+    """Algorithmic HBM bytes of one quant launch over M rows of length L (the
+    row length of the quantized values) in groups of g: the bf16 input read
+    once, e4m3 codes and fp32 scales written once, the RMSNorm weight once."""
+    if op == "silu_mul_quant":
+        return M * (4 * L + L + 4 * (L // g))
+    b = M * (2 * L + L + 4 * (L // g))
+    return b + 2 * L if op == "rmsnorm_quant" else b
 
 
 def max_over_ranks(values, world, device="cpu"):
@@ -95,25 +105,85 @@ def job_tflops(flops_per_rank_step, steps, world, ms):
 
 
 def workload_config(M, n):
-    return {"workload": f"qwen3-8b-mlp-block-m{M}-per-token+blockwise",
-            "model": "Qwen3-8B-shaped MLP (hidden 4096, intermediate 12288)",
+    return {"workload": f"qwen3-32b-prefill-m{M}-linear-stack-per-token+blockwise",
+            "model": "Qwen3-32B-shaped decoder block linears (hidden 5120, intermediate 25600, "
+                     "64 q / 8 kv heads of 128): qkv, o, gate_up, down",
             "global_batch": M * n, "tokens_per_gpu": M, "seq_len": None,
             "parallelism": f"replicas{n}" if n > 1 else "single-gpu",
-            "l2": "flushed between timed steps (256 MiB write)"}
+            "l2": "flushed between timed steps (256 MiB write); the step's weights "
+                  "(0.98 GB of e4m3) exceed L2 as well"}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except Exception:
+        return {}
+
+
+def fp8_peak(peaks, timed_s):
+    """Dense FP8 denominator: 2 x the measured bf16 GEMM rate (nominal fp8:bf16
+    = 4.5:2.25); the burst figure for a timed region under a second, the
+    sustained one (measured over seconds under the power cap) beyond."""
+    burst, sust = peaks.get("bf16_tflops"), peaks.get("bf16_tflops_sustained")
+    if timed_s >= 1.0:
+        if sust:
+            return 2.0 * sust, f"of measured: 2 x bf16 sustained (timed region {timed_s:.2f} s)"
+        return 2.0 * 1400.0, "of fallback: 2 x 1.4 PF bf16 sustained"
+    if burst:
+        return 2.0 * burst, f"of measured: 2 x bf16 burst (timed region {timed_s:.2f} s)"
+    return 2.0 * 1590.0, "of fallback: 2 x 1.59 PF bf16 burst"
 
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
+    """SM clock and throttle reasons sampled every 10 ms during the timed
+    region (NVML; nvidia-smi at 200 ms when NVML is unavailable)."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
+
     def __init__(self, index):
         self.index = index
-        self.proc = None
-        import tempfile
-        self.path = os.path.join(tempfile.gettempdir(), f"fp8q_clocks_{os.getpid()}.csv")
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
 
     def start(self):
         try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
+                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        for nm, bit in self.REASONS.items():
+                            if r & bit:
+                                self.reasons.add(nm)
+                    except Exception:
+                        pass
+                    self._stop.wait(0.01)
+
+            self._thread = threading.Thread(target=run, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._thread = None
+            self._start_smi()
+
+    def _start_smi(self):
+        import tempfile
+        self.path = os.path.join(tempfile.gettempdir(), f"fp8q_clocks_{os.getpid()}.csv")
+        try:
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
+            self._proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}",
                  "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -121,40 +191,41 @@ class ClockSampler:
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
-            self.proc = None
+            self._proc = None
             if getattr(self, "f", None):
                 self.f.close()
                 os.remove(self.path)
 
     def stop(self):
-        if self.proc is None:
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        elif self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except Exception:
+                self._proc.kill()
+            self.f.close()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) < 7:
+                        continue
+                    try:
+                        self.samples.append(float(parts[0]))
+                        self.max_mhz = max(self.max_mhz or 0.0, float(parts[1]))
+                    except ValueError:
+                        continue
+                    for nm, v in zip(names, parts[3:7]):
+                        if v.lower() == "active":
+                            self.reasons.add(nm)
+            os.remove(self.path)
+        if not self.samples:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 7:
-                    continue
-                try:
-                    sm.append(float(parts[0]))
-                    mx.append(float(parts[1]))
-                except ValueError:
-                    continue
-                for nm, v in zip(names, parts[3:7]):
-                    if v.lower() == "active":
-                        reasons.add(nm)
-        os.remove(self.path)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 # ------------------------------------------------------------------ native arm
@@ -170,11 +241,16 @@ def run_native(args, rank, world, local_rank):
     M = args.m
     torch.manual_seed(1234 + rank)
 
+    def host_bf16(bits):
+        return torch.from_numpy(bits.view("int16")).view(torch.bfloat16)
+
     # ---- inputs (seeded, synthetic) and weights, resident in HBM
-    x_host = torch.from_numpy(inp.heavy_tailed_bf16(2000 + rank, M, H).view("int16")).view(torch.bfloat16)
-    x_pinned = x_host.pin_memory()
-    x = x_host.to(dev)
-    w_norm = torch.from_numpy(inp.rms_weight_bf16(2001, H).view("int16")).view(torch.bfloat16).to(dev)
+    x_host = host_bf16(inp.heavy_tailed_bf16(2000 + rank, M, H))
+    a_host = host_bf16(inp.normal_bf16(2100 + rank, (M, ATT)))
+    x_pinned, a_pinned = x_host.pin_memory(), a_host.pin_memory()
+    x, attn = x_host.to(dev), a_host.to(dev)
+    w_in = host_bf16(inp.rms_weight_bf16(2001, H)).to(dev)
+    w_post = host_bf16(inp.rms_weight_bf16(2002, H)).to(dev)
 
     def make_weight(N, K, seed):
         g = torch.Generator(device=dev).manual_seed(seed)
@@ -184,77 +260,105 @@ def run_native(args, rank, world, local_rank):
         q, s = fq.fp8q_group_quant(W, W.shape[1])
         return q, s.reshape(-1).contiguous()
 
-    def per_block(W):
+    def per_block(W, pow2=False):
+        # weight block scales: amax of each 128x128 block / 448 (setup, untimed)
         N, K = W.shape
         wb = W.float().view(N // 128, 128, K // 128, 128)
-        amax = wb.abs().amax(dim=(1, 3)).clamp_min(1e-10)
-        s = (amax / 448.0).float()
+        s = (wb.abs().amax(dim=(1, 3)).clamp_min(1e-10) / 448.0).float()
+        if pow2:
+            s = torch.pow(2.0, torch.ceil(torch.log2(s)))
         q = (wb / s[:, None, :, None]).clamp(-448, 448).to(torch.float8_e4m3fn).view(N, K)
         return q.contiguous(), s.contiguous()
 
-    Wgu = make_weight(2 * I, H, 11)
-    Wd = make_weight(H, I, 12)
-    gu_pt, sgu_pt = per_channel(Wgu)
-    d_pt, sd_pt = per_channel(Wd)
-    gu_bw, sgu_bw = per_block(Wgu)
-    d_bw, sd_bw = per_block(Wd)
-    del Wgu, Wd
-
-    # ---- activation buffers
     f8 = torch.float8_e4m3fn
-    q_tok = torch.empty((M, H), dtype=f8, device=dev)
-    s_tok = torch.empty((M, 1), dtype=torch.float32, device=dev)
-    q_grp = torch.empty((M, H), dtype=f8, device=dev)
-    s_grp = torch.empty((M, H // 128), dtype=torch.float32, device=dev)
-    qa = torch.empty((M, H), dtype=f8, device=dev)
-    sa = torch.empty((M, 1), dtype=torch.float32, device=dev)
-    h = torch.empty((M, 2 * I), dtype=torch.bfloat16, device=dev)
-    qh = torch.empty((M, I), dtype=f8, device=dev)
-    sh = torch.empty((M, 1), dtype=torch.float32, device=dev)
-    out_pt = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
-    qa_b = torch.empty((M, H), dtype=f8, device=dev)
-    sa_b = torch.empty((H // 128, M), dtype=torch.float32, device=dev)
-    h_b = torch.empty((M, 2 * I), dtype=torch.bfloat16, device=dev)
-    qh_b = torch.empty((M, I), dtype=f8, device=dev)
-    sh_b = torch.empty((I // 128, M), dtype=torch.float32, device=dev)
-    out_b = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
-    ws = {k: fq.make_workspace(M, N, K, bw, dev) for k, (N, K, bw) in
-          {"gu": (2 * I, H, False), "d": (H, I, False), "gub": (2 * I, H, True),
-           "db": (H, I, True)}.items()}
+    W = {}
+    for i, (name, K, N) in enumerate(LAYERS):
+        Wt = make_weight(N, K, 11 + i)
+        W[("pt", name)] = per_channel(Wt)
+        W[("bw", name)] = per_block(Wt)
+        if not args.no_e8m0:
+            q8, s8 = per_block(Wt, pow2=True)
+            W[("e8", name)] = (q8, (torch.log2(s8).round() + 127).to(torch.uint8).contiguous())
+        del Wt
+
+    # ---- activation buffers and workspaces, per scheme
+    def scheme_buffers(sc):
+        gm = sc != "pt"                      # group-major 1x128 scales
+        sdt = torch.uint8 if sc == "e8" else torch.float32
+
+        def sc_buf(L):
+            return torch.empty((L // 128, M) if gm else (M, 1), dtype=sdt, device=dev)
+
+        b = {"qa": torch.empty((M, H), dtype=f8, device=dev), "sa": sc_buf(H),
+             "yqkv": torch.empty((M, QKV), dtype=torch.bfloat16, device=dev),
+             "qo": torch.empty((M, ATT), dtype=f8, device=dev), "so": sc_buf(ATT),
+             "h1": torch.empty((M, H), dtype=torch.bfloat16, device=dev),
+             "qm": torch.empty((M, H), dtype=f8, device=dev), "sm": sc_buf(H),
+             "gu": torch.empty((M, 2 * I), dtype=torch.bfloat16, device=dev),
+             "qh": torch.empty((M, I), dtype=f8, device=dev), "sh": sc_buf(I),
+             "out": torch.empty((M, H), dtype=torch.bfloat16, device=dev)}
+        mode = {"pt": False, "bw": True, "e8": 2}[sc]
+        b["ws"] = {name: fq.make_workspace(M, N, K, mode, dev) for name, K, N in LAYERS}
+        return b
+
+    schemes = ["pt", "bw"] + ([] if args.no_e8m0 else ["e8"])
+    B = {sc: scheme_buffers(sc) for sc in schemes}
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    ev_gu = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
 
-    def step(xin, ev=None, y_pt=None, y_b=None):
-        # ev: [pt_start, pt_end, bw_start, bw_end] events around the two gate_up GEMMs;
-        # y_pt, y_b: the block outputs of the two chains (default out_pt, out_b)
-        fq.fp8q_group_quant(xin, H, q=q_tok, scales=s_tok)
-        fq.fp8q_group_quant(xin, 128, q=q_grp, scales=s_grp)
-        fq.fp8q_rmsnorm_quant(xin, w_norm, EPS, H, q=qa, scales=sa)
-        if ev:
-            ev[0].record(stream)
-        fq.fp8q_scaled_mm(qa, gu_pt, sa.view(-1), sgu_pt, y=h, workspace=ws["gu"])
-        if ev:
-            ev[1].record(stream)
-        fq.fp8q_silu_mul_quant(h, I, q=qh, scales=sh)
-        fq.fp8q_scaled_mm(qh, d_pt, sh.view(-1), sd_pt, y=out_pt if y_pt is None else y_pt,
-                          workspace=ws["d"])
-        fq.fp8q_rmsnorm_quant(xin, w_norm, EPS, 128, q=qa_b, scales=sa_b, scale_layout="group_major")
-        if ev:
-            ev[2].record(stream)
-        fq.fp8q_scaled_mm_blockwise(qa_b, gu_bw, sa_b, sgu_bw, a_scale_layout="group_major", y=h_b,
-                                    workspace=ws["gub"])
-        if ev:
-            ev[3].record(stream)
-        fq.fp8q_silu_mul_quant(h_b, 128, q=qh_b, scales=sh_b, scale_layout="group_major")
-        fq.fp8q_scaled_mm_blockwise(qh_b, d_bw, sh_b, sd_bw, a_scale_layout="group_major",
-                                    y=out_b if y_b is None else y_b, workspace=ws["db"])
+    def chain(sc, xin, ain, out=None):
+        """The launches of one scheme's stack: list of (name, kind, units, fn)."""
+        b = B[sc]
+        out = b["out"] if out is None else out
+        ue = {"pt": False, "bw": False, "e8": "packed"}[sc]
+        lay = "row_major" if sc == "pt" else "group_major"
+        gs = (lambda L: L) if sc == "pt" else (lambda L: 128)
+        tag = {"pt": "per-token", "bw": "1x128", "e8": "1x128 e8m0"}[sc]
 
-    LAUNCHES_PER_STEP = 10
+        def gemm(name, a, sa, y):
+            Wq, Ws = W[(sc, name)]
+            ws = b["ws"][name]
+            if sc == "pt":
+                return lambda: fq.fp8q_scaled_mm(a, Wq, sa.view(-1), Ws, y=y, workspace=ws)
+            if sc == "bw":
+                return lambda: fq.fp8q_scaled_mm_blockwise(a, Wq, sa, Ws, a_scale_layout="group_major",
+                                                           y=y, workspace=ws)
+            return lambda: fq.fp8q_scaled_mm_blockwise_e8m0(a, Wq, sa, Ws, a_scale_layout="group_major",
+                                                            y=y, workspace=ws)
+
+        gname = {"pt": "scaled_mm", "bw": "scaled_mm_blockwise", "e8": "scaled_mm_blockwise_e8m0"}[sc]
+        fl = {name: 2 * M * N * K for name, K, N in LAYERS}
+        return [
+            (f"rmsnorm_quant {tag} (H={H})", "quant", quant_bytes("rmsnorm_quant", M, H, gs(H)),
+             lambda: fq.fp8q_rmsnorm_quant(xin, w_in, EPS, gs(H), ue, q=b["qa"], scales=b["sa"],
+                                           scale_layout=lay)),
+            (f"{gname} qkv ({M}x{QKV}x{H})", "gemm", fl["qkv"], gemm("qkv", b["qa"], b["sa"], b["yqkv"])),
+            (f"group_quant {tag} (K={ATT})", "quant", quant_bytes("group_quant", M, ATT, gs(ATT)),
+             lambda: fq.fp8q_group_quant(ain, gs(ATT), ue, q=b["qo"], scales=b["so"], scale_layout=lay)),
+            (f"{gname} o ({M}x{H}x{ATT})", "gemm", fl["o"], gemm("o", b["qo"], b["so"], b["h1"])),
+            (f"rmsnorm_quant {tag} (H={H}, o output)", "quant", quant_bytes("rmsnorm_quant", M, H, gs(H)),
+             lambda: fq.fp8q_rmsnorm_quant(b["h1"], w_post, EPS, gs(H), ue, q=b["qm"], scales=b["sm"],
+                                           scale_layout=lay)),
+            (f"{gname} gate_up ({M}x{2 * I}x{H})", "gemm", fl["gate_up"],
+             gemm("gate_up", b["qm"], b["sm"], b["gu"])),
+            (f"silu_mul_quant {tag} (I={I})", "quant", quant_bytes("silu_mul_quant", M, I, gs(I)),
+             lambda: fq.fp8q_silu_mul_quant(b["gu"], gs(I), ue, q=b["qh"], scales=b["sh"],
+                                            scale_layout=lay)),
+            (f"{gname} down ({M}x{H}x{I})", "gemm", fl["down"], gemm("down", b["qh"], b["sh"], out)),
+        ]
+
+    launches = chain("pt", x, attn) + chain("bw", x, attn)
+    LAUNCHES_PER_STEP = len(launches)
+
+    def run_step(ls, evs=None):
+        for j, (_, _, _, fn) in enumerate(ls):
+            fn()
+            if evs is not None:
+                evs[j].record(stream)
 
     # ---- warm-up
     for _ in range(args.warmup):
-        step(x)
+        run_step(launches)
     torch.cuda.synchronize()
     st = fq.fp8q_last_device_status()
     if st != fq.OK:
@@ -264,41 +368,46 @@ def run_native(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
+    def timed(ls, steps, sampler=None):
+        """Per step: untimed L2 flush, start event, every launch followed by an
+        event.  Returns (step times, per-launch times), ms."""
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        starts = [ev() for _ in range(steps)]
+        per = [[ev() for _ in ls] for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        if sampler:
+            sampler.start()
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            run_step(ls, per[i])
+        torch.cuda.synchronize()
+        clocks = sampler.stop() if sampler else None
+        barrier()
+        step_ms = [s.elapsed_time(p[-1]) for s, p in zip(starts, per)]
+        launch_ms = [[(starts[i] if j == 0 else per[i][j - 1]).elapsed_time(per[i][j])
+                      for i in range(steps)] for j in range(len(ls))]
+        return step_ms, launch_ms, clocks
+
     # ---- timed: device-resident inputs
     sampler = ClockSampler(local_rank)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    gu_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    for i in range(args.steps):
-        flush.zero_()                                   # untimed L2 flush
-        starts[i].record(stream)
-        step(x, gu_ev[i])
-        ends[i].record(stream)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    barrier()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    gu_ms = [e[0].elapsed_time(e[1]) for e in gu_ev]
-    gub_ms = [e[2].elapsed_time(e[3]) for e in gu_ev]
+    step_ms, launch_ms, clocks = timed(launches, args.steps, sampler)
     total_ms = sum(step_ms)
 
-    # ---- timed: end to end through host buffers.  Every step copies its input
-    # from pinned host memory and both block outputs back to pinned host memory;
-    # as in a serving loop the copies run on their own streams, double-buffered,
-    # so step i+1's upload and step i-1's download overlap step i's kernels.
-    # The L2 flush before each step's kernels stays inside this timed region.
+    # ---- timed: end to end through host buffers (see the module docstring)
     NBUF = 2
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    xd = [torch.empty_like(x) for _ in range(NBUF)]
-    yd = [(torch.empty_like(out_pt), torch.empty_like(out_b)) for _ in range(NBUF)]
+    xd = [(torch.empty_like(x), torch.empty_like(attn)) for _ in range(NBUF)]
+    yd = [(torch.empty((M, H), dtype=torch.bfloat16, device=dev),
+           torch.empty((M, H), dtype=torch.bfloat16, device=dev)) for _ in range(NBUF)]
+    e2e_launches = [chain("pt", xd[b][0], xd[b][1], yd[b][0]) + chain("bw", xd[b][0], xd[b][1], yd[b][1])
+                    for b in range(NBUF)]
     out_pinned = [torch.empty((2, M, H), dtype=torch.bfloat16).pin_memory() for _ in range(NBUF)]
-    ev = lambda: torch.cuda.Event(enable_timing=False)
-    in_done = [ev() for _ in range(args.steps)]
-    comp_done = [ev() for _ in range(args.steps)]
-    out_done = [ev() for _ in range(args.steps)]
+    evn = lambda: torch.cuda.Event(enable_timing=False)
+    in_done = [evn() for _ in range(args.steps)]
+    comp_done = [evn() for _ in range(args.steps)]
+    out_done = [evn() for _ in range(args.steps)]
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
     barrier()
@@ -311,13 +420,14 @@ def run_native(args, rank, world, local_rank):
         with torch.cuda.stream(s_in):
             if i >= NBUF:
                 s_in.wait_event(comp_done[i - NBUF])       # step i-2 has read xd[b]
-            xd[b].copy_(x_pinned, non_blocking=True)
+            xd[b][0].copy_(x_pinned, non_blocking=True)
+            xd[b][1].copy_(a_pinned, non_blocking=True)
             in_done[i].record(s_in)
         stream.wait_event(in_done[i])
         if i >= NBUF:
             stream.wait_event(out_done[i - NBUF])          # yd[b] has reached the host
         flush.zero_()
-        step(xd[b], y_pt=yd[b][0], y_b=yd[b][1])
+        run_step(e2e_launches[b])
         comp_done[i].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[i])
@@ -329,6 +439,32 @@ def run_native(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e_start.elapsed_time(e_end)
+
+    # ---- the E8M0 chain (blockwise stack with packed UE8M0 scales), timed alone
+    e8 = None
+    if not args.no_e8m0:
+        l8 = chain("e8", x, attn)
+        for _ in range(max(1, args.warmup)):
+            run_step(l8)
+        s8, lm8, _ = timed(l8, args.steps)
+        e8 = (l8, s8, lm8)
+    # ---- fused_qk_norm_rope on the step's qkv output (the attention-side op of
+    # the same forward pass; not part of the quant+GEMM metric), timed alone
+    rope = None
+    if not args.no_rope:
+        hq, hk, hv, hd = 64, 8, 8, 128
+        qkv = B["pt"]["yqkv"]
+        cs = torch.randn((32768, hd), device=dev)
+        pos = torch.randint(0, 32768, (M,), dtype=torch.int64, device=dev)
+        qw = (1.0 + 0.1 * torch.randn(hd, device=dev)).to(torch.bfloat16)
+        kw = (1.0 + 0.1 * torch.randn(hd, device=dev)).to(torch.bfloat16)
+        rl = [(f"qk_norm_rope neox (T={M}, {hq}+{hk} heads of {hd})", "quant",
+               M * (hq + hk) * hd * 2 * 2 + M * (hd * 4 + 8),
+               lambda: fq.fp8q_qk_norm_rope(qkv, hq, hk, hv, hd, EPS, qw, kw, cs, pos, True))]
+        for _ in range(max(1, args.warmup)):
+            run_step(rl)
+        _, lmr, _ = timed(rl, args.steps)
+        rope = (rl, lmr)
     st = fq.fp8q_last_device_status()
     if st != fq.OK:
         raise RuntimeError(f"device status after timing: {fq.fp8q_status_string(st)}")
@@ -339,96 +475,123 @@ def run_native(args, rank, world, local_rank):
     flops_step = gemm_flops(M)
     value = job_tflops(flops_step, args.steps, world, total_ms)
     e2e_value = job_tflops(flops_step, args.steps, world, e2e_ms)
-    gu_flops = 2 * M * H * 2 * I
-    gu_avg_s = statistics.mean(gu_ms) * 1e-3
-    peaks = {}
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peaks = json.load(f)
-    except Exception:
-        pass
-    bf16_sust = peaks.get("bf16_tflops_sustained")
-    if bf16_sust:
-        peak, peak_src = 2.0 * bf16_sust, "of measured: 2 x bf16 sustained (fp8:bf16 nominal 4.5:2.25)"
+    peaks = load_peaks()
+    peak, peak_src = fp8_peak(peaks, total_ms * 1e-3)
+    hbm = peaks.get("hbm_gbs")
+    hbm_src = "of measured: copy bandwidth" if hbm else "of fallback: 6.65 TB/s"
+    hbm = hbm or 6650.0
+
+    def kernel_rows(ls, lms):
+        gemms, quants = [], []
+        for (name, kind, units, _), ms in zip(ls, lms):
+            avg_s = statistics.mean(ms) * 1e-3
+            if kind == "gemm":
+                a = units / avg_s / 1e12
+                gemms.append({"kernel": name, "us": round(avg_s * 1e6, 1), "bound": "tensor",
+                              "achieved": round(a, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                              "frac": round(a / peak, 4), "flops": units})
+            else:
+                a = units / avg_s / 1e9
+                quants.append({"kernel": name, "us": round(avg_s * 1e6, 1), "bound": "hbm",
+                               "achieved": round(a, 1), "peak": round(hbm, 1), "unit": "GB/s",
+                               "frac": round(a / hbm, 4), "bytes": units})
+        return gemms, quants
+
+    gemms, quants = kernel_rows(launches, launch_ms)
+    share = [statistics.mean(ms) for ms in launch_ms]
+    dom = max(range(len(launches)), key=lambda j: share[j])
+    dname, dkind, dunits, _ = launches[dom]
+    davg = share[dom] * 1e-3
+    if dkind == "gemm":
+        roof = {"bound": "tensor", "kernel": dname, "achieved": round(dunits / davg / 1e12, 1),
+                "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(dunits / davg / 1e12 / peak, 4),
+                "peak_source": peak_src}
     else:
-        peak, peak_src = 2.0 * 1400.0, "of fallback: 2 x 1.4 PF bf16 sustained"
-    achieved = gu_flops / gu_avg_s / 1e12
-    achieved_bw = gu_flops / (statistics.mean(gub_ms) * 1e-3) / 1e12
-    qb = quant_bytes(M)
+        roof = {"bound": "hbm", "kernel": dname, "achieved": round(dunits / davg / 1e9, 1),
+                "peak": round(hbm, 1), "unit": "GB/s", "frac": round(dunits / davg / 1e9 / hbm, 4),
+                "peak_source": hbm_src}
+    roof["share_of_step"] = round(share[dom] / (sum(share)), 4)
+    roof["traffic"] = None
+    roof["traffic_note"] = ("DRAM read+write bytes per launch come from an ncu capture of the same "
+                            "kernel build, kept with the profiles; not measured in this run")
+
     line = {
         "metric": METRIC,
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
-        "data": "synthetic (seeded Student-t(3) activations, N(0,0.02) weights)",
+        "data": "synthetic (seeded Student-t(3) activations with outlier channels, N(0,1) attention "
+                "output stand-in, N(0,0.02) weights)",
         "config": workload_config(M, world),
-        "quant_hbm_gbs": round(qb * args.steps / (total_ms * 1e-3) / 1e9, 1),
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": M * H * 2, "d2h_bytes_per_step": 2 * M * H * 2,
+                "h2d_bytes_per_step": (x.numel() + attn.numel()) * 2,
+                "d2h_bytes_per_step": 2 * M * H * 2,
                 "ms_per_step": round(e2e_ms / args.steps, 4),
                 "copies": "pinned host buffers, own streams, double-buffered against the "
                           "neighbouring steps' kernels; L2 flush inside the timed region"},
-        # The dominant kernel of the step (largest share of the ncu launch list):
-        # the blockwise gate_up GEMM.  traffic = ncu dram read + write bytes of one
-        # launch of the same kernel build (profiles/gemm_kernel_qwen3_8b_mlp_m2048.md).
-        "roofline": {"bound": "tensor",
-                     "kernel": "scaled_mm_blockwise gate_up (2048x24576x4096, 128x256 tiles)",
-                     "achieved": round(achieved_bw, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-                     "frac": round(achieved_bw / peak, 4), "peak_source": peak_src,
-                     "traffic": GATE_UP_BW_TRAFFIC},
-        "roofline_per_token_gemm": {
-                     "bound": "tensor",
-                     "kernel": "scaled_mm gate_up (per-token, 2048x24576x4096, 256x256 CTA-pair tiles)",
-                     "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "peak_source": peak_src,
-                     "traffic": GATE_UP_PT_TRAFFIC},
+        "roofline": roof,
+        "gemms": gemms,
+        "roofline_quant": quants,
         "clocks": clocks,
     }
+    if clocks:
+        line["clocks"]["time_x_sm_mhz"] = round(total_ms / args.steps * clocks["sm_mhz"], 1)
+    if rope is not None:
+        _, qr = kernel_rows(*rope)
+        line["qk_norm_rope"] = qr[0]
+        line["qk_norm_rope"]["bytes_note"] = ("q and k heads read and written once, the token's "
+                                              "cos/sin row and position read once")
+        line["gpu_launches"] += args.steps
+    if e8 is not None:
+        l8, s8, lm8 = e8
+        g8, q8 = kernel_rows(l8, lm8)
+        t8 = sum(s8)
+        f8_step = sum(2 * M * N * K for _, K, N in LAYERS)
+        line["e8m0_chain"] = {
+            "what": "the blockwise stack with packed UE8M0 (E8M0 byte) scales: fused quant ops with "
+                    "ue8m0='packed' -> scaled_mm_blockwise_e8m0 (block-scaled tcgen05 MMA)",
+            "ms_per_step": round(t8 / args.steps, 4),
+            "value": round(f8_step * args.steps / (t8 * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "gemms": g8, "roofline_quant": q8}
+        line["gpu_launches"] += len(l8) * args.steps
     return line
 
 
 # ------------------------------------------------------------------ oracle arm
 def run_reference(args):
     """The CPU oracle, as it stands, on a bounded sample of the same workload:
-    all quant ops on `rows` tokens and both GEMM chains on those rows."""
+    every op of the step on `rows` tokens (weights: seeded random e4m3 codes
+    with random scales -- the oracle's cost does not depend on the values)."""
     import numpy as np
 
     import fp8q_inputs as inp
     import oracle
 
     M = args.m
-    rows = int(os.environ.get("FP8Q_REF_ROWS", "16"))
+    rows = int(os.environ.get("FP8Q_REF_ROWS", "8"))
     x = inp.heavy_tailed_bf16(2000, rows, H)
-    w = inp.rms_weight_bf16(2001, H)
-    rng = np.random.default_rng(7)
-    # weights: per channel and per block, quantized by the oracle (setup, untimed)
-    Wgu = inp.to_bf16_bits(rng.normal(0, 0.02, (2 * I, H)))
-    Wd = inp.to_bf16_bits(rng.normal(0, 0.02, (H, I)))
-    gu_q, gu_s = oracle.group_quant(Wgu, H)
-    d_q, d_s = oracle.group_quant(Wd, I)
+    att = inp.normal_bf16(2100, (rows, ATT))
+    w_in, w_post = inp.rms_weight_bf16(2001, H), inp.rms_weight_bf16(2002, H)
+    Wq = {name: inp.random_e4m3_codes_u8(31 + i, (N, K)) for i, (name, K, N) in enumerate(LAYERS)}
+    s_ch = {name: inp.random_scales(41 + i, (N,)) for i, (name, K, N) in enumerate(LAYERS)}
+    s_bl = {name: inp.random_scales(51 + i, (N // 128, K // 128)) for i, (name, K, N) in enumerate(LAYERS)}
 
-    def blocks(Wb, N, K):
-        wf = inp.bf16_bits_to_f32(Wb).reshape(N // 128, 128, K // 128, 128)
-        s = oracle.scale(np.abs(wf).max(axis=(1, 3)).astype(np.float32))
-        q = oracle.e4m3_encode((wf / s[:, None, :, None]).astype(np.float32)).reshape(N, K)
-        return q, s
-
-    gu_bq, gu_bs = blocks(Wgu, 2 * I, H)
-    d_bq, d_bs = blocks(Wd, H, I)
+    def stack(g, mm):
+        qa, sa = oracle.rmsnorm_quant(x, w_in, EPS, g(H))
+        mm("qkv", qa, sa)
+        qo, so = oracle.group_quant(att, g(ATT))
+        h1 = inp.to_bf16_bits(mm("o", qo, so))
+        qm, sm = oracle.rmsnorm_quant(h1, w_post, EPS, g(H))
+        gu = inp.to_bf16_bits(mm("gate_up", qm, sm))
+        qh, sh = oracle.silu_mul_quant(gu, g(I))
+        mm("down", qh, sh)
 
     def step():
-        oracle.group_quant(x, H)
-        oracle.group_quant(x, 128)
-        qa, sa = oracle.rmsnorm_quant(x, w, EPS, H)
-        h, _ = oracle.scaled_mm(qa, gu_q, sa.reshape(-1), gu_s.reshape(-1))
-        hb = inp.to_bf16_bits(h)
-        qh, sh = oracle.silu_mul_quant(hb, I)
-        oracle.scaled_mm(qh, d_q, sh.reshape(-1), d_s.reshape(-1))
-        qa, sa = oracle.rmsnorm_quant(x, w, EPS, 128)
-        h, _ = oracle.scaled_mm_blockwise(qa, gu_bq, sa, gu_bs)
-        qh, sh = oracle.silu_mul_quant(inp.to_bf16_bits(h), 128)
-        oracle.scaled_mm_blockwise(qh, d_bq, sh, d_bs)
+        stack(lambda L: L,
+              lambda n, a, s: oracle.scaled_mm(a, Wq[n], s.reshape(-1), s_ch[n])[0])
+        stack(lambda L: 128,
+              lambda n, a, s: oracle.scaled_mm_blockwise(a, Wq[n], s, s_bl[n])[0])
 
     for _ in range(max(1, min(args.warmup, 1))):
         step()
@@ -436,10 +599,9 @@ def run_reference(args):
     for _ in range(args.steps):
         step()
     dt = time.perf_counter() - t0
-    flops = gemm_flops(rows) * args.steps
-    value = flops / dt / 1e12
+    value = gemm_flops(rows) * args.steps / dt / 1e12
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    sample = (f"{rows} of {M} tokens per step (all ops of the step on those tokens; "
+    sample = (f"{rows} of {M} tokens per step (every op of the step on those tokens; "
               f"value = their GEMM FLOPs / oracle time)")
     return {
         "metric": METRIC,
@@ -455,7 +617,7 @@ def run_reference(args):
 
 def cpu_baseline_leg(args):
     """Oracle timed on a bounded sample (rank 0, N=1 only)."""
-    os.environ.setdefault("FP8Q_REF_ROWS", "64")
+    os.environ.setdefault("FP8Q_REF_ROWS", "32")
     a = argparse.Namespace(**vars(args))
     a.steps, a.warmup = 1, 0
     r = run_reference(a)
@@ -656,24 +818,38 @@ def run_sweep(args):
                     del x
 
     def gemm_case(tag, M, N, K, blockwise):
-        a = torch.randint(0, 126, (M, K), dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
-        b = torch.randint(0, 126, (N, K), dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
-        if blockwise:
+        """blockwise: False (scaled_mm), True (fp32 block scales), "e8m0" (E8M0 block
+        scales, block-scaled MMA) or "i8" (W8A8_INT8)."""
+        scheme = {False: 0, True: 1, "e8m0": 2, "i8": 3}[blockwise]
+        if scheme == 3:
+            a = torch.randint(-128, 128, (M, K), dtype=torch.int8, device=dev)
+            b = torch.randint(-128, 128, (N, K), dtype=torch.int8, device=dev)
+        else:
+            a = torch.randint(0, 126, (M, K), dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
+            b = torch.randint(0, 126, (N, K), dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
+        ws = fq.make_workspace(M, N, K, scheme, dev)
+        if scheme == 1:
             sa = torch.rand((K // 128, M), device=dev) * 1e-3 + 1e-4
             sb = torch.rand((N // 128, K // 128), device=dev) * 1e-3 + 1e-4
-            ws = fq.make_workspace(M, N, K, True, dev)
-            fn = lambda: fq.fp8q_scaled_mm_blockwise(a, b, sa, sb, a_scale_layout="group_major",
-                                                     workspace=ws)
+            call = lambda bb: fq.fp8q_scaled_mm_blockwise(a, bb, sa, sb, a_scale_layout="group_major",
+                                                          workspace=ws)
+        elif scheme == 2:
+            sa = torch.randint(110, 130, (K // 128, M), dtype=torch.uint8, device=dev)
+            sb = torch.randint(110, 130, (N // 128, K // 128), dtype=torch.uint8, device=dev)
+            call = lambda bb: fq.fp8q_scaled_mm_blockwise_e8m0(a, bb, sa, sb, a_scale_layout="group_major",
+                                                               workspace=ws)
         else:
             sa = torch.rand(M, device=dev) * 1e-3 + 1e-4
             sb = torch.rand(N, device=dev) * 1e-3 + 1e-4
-            ws = fq.make_workspace(M, N, K, False, dev)
-            fn = lambda: fq.fp8q_scaled_mm(a, b, sa, sb, workspace=ws)
+            mm = fq.fp8q_scaled_mm_i8 if scheme == 3 else fq.fp8q_scaled_mm
+            call = lambda bb: mm(a, bb, sa, sb, workspace=ws)
+        fn = lambda: call(b)
         t = timeit(fn)
         flops = 2.0 * M * N * K
         nbytes = M * K + N * K + 2 * M * N
-        v = fq.fp8q_select_gemm_variant(M, N, K, blockwise)
-        d = {"op": "scaled_mm_blockwise" if blockwise else "scaled_mm", "shape": tag, "M": M,
+        v = fq.fp8q_select_gemm_variant(M, N, K, scheme)
+        op = ["scaled_mm", "scaled_mm_blockwise", "scaled_mm_blockwise_e8m0", "scaled_mm_i8"][scheme]
+        d = {"op": op, "shape": tag, "M": M,
              "N": N, "K": K, "variant": v, "us": round(t * 1e6, 2),
              "TFLOP/s": round(flops / t / 1e12, 1), "frac_fp8_peak": round(flops / t / 1e12 / fp8_peak, 3),
              "GB/s": round(nbytes / t / 1e9, 1), "frac_hbm": round(nbytes / t / 1e9 / hbm, 3)}
@@ -683,11 +859,7 @@ def run_sweep(args):
             # weights from HBM, as a model's successive layers do
             copies = max(2, min(64, -(-(384 << 20) // (N * K))))
             bs = [b] + [torch.empty_like(b).copy_(b) for _ in range(copies - 1)]
-            if blockwise:
-                fns = [lambda bb=bb: fq.fp8q_scaled_mm_blockwise(
-                    a, bb, sa, sb, a_scale_layout="group_major", workspace=ws) for bb in bs]
-            else:
-                fns = [lambda bb=bb: fq.fp8q_scaled_mm(a, bb, sa, sb, workspace=ws) for bb in bs]
+            fns = [lambda bb=bb: call(bb) for bb in bs]
             tg = graph_time(fns)
             d.update({"graph_us_per_call": round(tg * 1e6, 2),
                       "graph_GB/s": round(nbytes / tg / 1e9, 1),
@@ -713,10 +885,20 @@ def run_sweep(args):
                 gemm_case(f"qwen3-32b {layer}", M, N, K, True)
     if which in ("prefill32b", "all"):
         sh = inp.linear_shapes(inp.QWEN3_32B)
-        for bw in (False, True):
+        for bw in (False, True, "e8m0", "i8"):
             for layer in ("qkv", "o", "gate_up", "down"):
                 K, N = sh[layer]
                 gemm_case(f"qwen3-32b {layer}", 8192, N, K, bw)
+    if which in ("e8m0", "all"):
+        sh8, sh32 = inp.linear_shapes(inp.QWEN3_8B), inp.linear_shapes(inp.QWEN3_32B)
+        for M in (1, 16, 64, 256, 1024, 4096):
+            for layer in ("qkv", "o", "gate_up", "down"):
+                K, N = sh8[layer]
+                gemm_case(f"qwen3-8b {layer}", M, N, K, "e8m0")
+        for M in (1, 8, 64):
+            for layer in ("qkv", "o", "gate_up", "down"):
+                K, N = sh32[layer]
+                gemm_case(f"qwen3-32b {layer}", M, N, K, "e8m0")
     return 0
 
 

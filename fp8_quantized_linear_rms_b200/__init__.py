@@ -8,8 +8,10 @@ package fails loudly if ``libfp8q.so`` is missing (build it with
 ``python fp8_quantized_linear_rms_b200/build.py``).
 
 The names match the C ABI:
-  fp8q_group_quant, fp8q_rmsnorm_quant, fp8q_silu_mul_quant   (activation quant)
-  fp8q_scaled_mm, fp8q_scaled_mm_blockwise                      (scaled FP8 GEMMs)
+  fp8q_group_quant, fp8q_rmsnorm_quant, fp8q_add_rmsnorm_quant, fp8q_silu_mul_quant
+                                                                (activation quant)
+  fp8q_scaled_mm, fp8q_scaled_mm_blockwise, fp8q_scaled_mm_blockwise_e8m0
+                                                                (scaled FP8 GEMMs)
   fp8q_workspace_bytes, fp8q_select_gemm_variant, fp8q_force_gemm_variant,
   fp8q_last_device_status, fp8q_status_string, fp8q_version
 """
@@ -54,12 +56,24 @@ _SIGS = {
                                   _P, _I64, _I64, _P]),
     "fp8q_silu_mul_quant": (_INT, [_P, _I64, _I64, _I64, _INT, _INT, _P, _I64, _P, _I64, _I64,
                                    _P]),
+    "fp8q_add_rmsnorm_quant": (_INT, [_P, _P, _P, ctypes.c_float, _I64, _I64, _I64, _I64, _INT, _INT,
+                                      _P, _I64, _P, _I64, _I64, _P]),
     "fp8q_scaled_mm": (_INT, [_P, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P, _I64, _P,
                               ctypes.c_size_t, _P]),
     "fp8q_scaled_mm_blockwise": (_INT, [_P, _P, _P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I64,
                                         _P, ctypes.c_size_t, _P]),
+    "fp8q_scaled_mm_blockwise_e8m0": (_INT, [_P, _P, _P, _I64, _I64, _P, _I64, _I64, _I64, _P,
+                                             _I64, _P, ctypes.c_size_t, _P]),
     "fp8q_scaled_mm_blockwise_noalloc": (_INT, [_P, _P, _P, _I64, _I64, _P, _I64, _I64, _I64, _P,
                                                 _I64, _P]),
+    "fp8q_qk_norm_rope": (_INT, [_P, _I64, _I64, _INT, _INT, _INT, _INT, ctypes.c_float, _P, _P, _P,
+                                 _I64, _P, _INT, _P]),
+    "fp8q_group_quant_i8": (_INT, [_P, _I64, _I64, _I64, _INT, _P, _I64, _P, _I64, _I64, _P]),
+    "fp8q_rmsnorm_quant_i8": (_INT, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _INT, _P, _I64, _P,
+                                     _I64, _I64, _P]),
+    "fp8q_silu_mul_quant_i8": (_INT, [_P, _I64, _I64, _I64, _INT, _P, _I64, _P, _I64, _I64, _P]),
+    "fp8q_scaled_mm_i8": (_INT, [_P, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P, _I64, _P,
+                                 ctypes.c_size_t, _P]),
     "fp8q_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, _INT]),
     "fp8q_select_gemm_variant": (_INT, [_I64, _I64, _I64, _INT, ctypes.POINTER(GemmVariant)]),
     "fp8q_force_gemm_variant": (_INT, [ctypes.POINTER(GemmVariant)]),
@@ -112,13 +126,25 @@ def _rowmajor(t: torch.Tensor, name: str) -> int:
     return t.stride(0)
 
 
-def _scales_out(M, L, group, layout, device, scales):
+def _ue8m0_mode(ue8m0) -> int:
+    """False / True / "packed" -> the ABI's 0 (fp32) / 1 (power-of-two fp32) / 2 (E8M0 bytes)."""
+    if ue8m0 == "packed":
+        return 2
+    if ue8m0 in (False, True, 0, 1):
+        return int(ue8m0)
+    raise ValueError(f"ue8m0 must be False, True or 'packed', got {ue8m0!r}")
+
+
+def _scales_out(M, L, group, layout, device, scales, mode=0):
     G = L // group if group > 0 and L % group == 0 else 0
+    dt = torch.uint8 if mode == 2 else torch.float32
     if scales is None:
         if layout == "group_major":
-            scales = torch.empty((G, M), dtype=torch.float32, device=device)
+            scales = torch.empty((G, M), dtype=dt, device=device)
         else:
-            scales = torch.empty((M, G), dtype=torch.float32, device=device)
+            scales = torch.empty((M, G), dtype=dt, device=device)
+    elif scales.dtype != dt:
+        raise TypeError(f"scales must be {dt} for ue8m0 mode {mode}")
     if layout == "group_major":
         return scales, 1, M
     return scales, G, 1
@@ -130,15 +156,17 @@ def fp8q_group_quant(x: torch.Tensor, group_size: int, ue8m0: bool = False, q=No
     """per_token_group_fp8_quant (group_size=128) / per-token quant (group_size=K).
 
     x: bf16 [M, K].  Returns (q float8_e4m3fn [M, K], scales fp32 [M, K/g]
-    (row_major) or [K/g, M] (group_major)).
+    (row_major) or [K/g, M] (group_major)).  ue8m0: False, True (power-of-two
+    fp32 scales) or "packed" (the same scales as uint8 E8M0 bytes).
     """
     _need(x, torch.bfloat16, "x")
     ldx = _rowmajor(x, "x")
     M, K = x.shape
+    mode = _ue8m0_mode(ue8m0)
     if q is None:
         q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
-    scales, ssm, ssg = _scales_out(M, K, group_size, scale_layout, x.device, scales)
-    st = lib.fp8q_group_quant(x.data_ptr(), M, K, ldx, group_size, int(ue8m0), q.data_ptr(),
+    scales, ssm, ssg = _scales_out(M, K, group_size, scale_layout, x.device, scales, mode)
+    st = lib.fp8q_group_quant(x.data_ptr(), M, K, ldx, group_size, mode, q.data_ptr(),
                               _rowmajor(q, "q"), scales.data_ptr(), ssm, ssg, _stream(stream))
     _check("fp8q_group_quant", st)
     return q, scales
@@ -152,13 +180,38 @@ def fp8q_rmsnorm_quant(x: torch.Tensor, w: torch.Tensor, eps: float, group_size:
     _need(w, torch.bfloat16, "w")
     ldx = _rowmajor(x, "x")
     M, H = x.shape
+    mode = _ue8m0_mode(ue8m0)
     if q is None:
         q = torch.empty((M, H), dtype=torch.float8_e4m3fn, device=x.device)
-    scales, ssm, ssg = _scales_out(M, H, group_size, scale_layout, x.device, scales)
+    scales, ssm, ssg = _scales_out(M, H, group_size, scale_layout, x.device, scales, mode)
     st = lib.fp8q_rmsnorm_quant(x.data_ptr(), w.data_ptr(), ctypes.c_float(eps), M, H, ldx,
-                                group_size, int(ue8m0), q.data_ptr(), _rowmajor(q, "q"),
+                                group_size, mode, q.data_ptr(), _rowmajor(q, "q"),
                                 scales.data_ptr(), ssm, ssg, _stream(stream))
     _check("fp8q_rmsnorm_quant", st)
+    return q, scales
+
+
+def fp8q_add_rmsnorm_quant(x: torch.Tensor, residual: torch.Tensor, w: torch.Tensor, eps: float,
+                           group_size: int, ue8m0=False, q=None, scales=None,
+                           scale_layout: str = "row_major", stream=None):
+    """Residual add + RMSNorm quant: residual <- bf16(x + residual) in place, then
+    rms_norm quant of the new residual.  Returns (q, scales)."""
+    _need(x, torch.bfloat16, "x")
+    _need(residual, torch.bfloat16, "residual")
+    _need(w, torch.bfloat16, "w")
+    ldx = _rowmajor(x, "x")
+    ldr = _rowmajor(residual, "residual")
+    M, H = x.shape
+    if tuple(residual.shape) != (M, H):
+        raise ValueError("residual must have x's shape")
+    mode = _ue8m0_mode(ue8m0)
+    if q is None:
+        q = torch.empty((M, H), dtype=torch.float8_e4m3fn, device=x.device)
+    scales, ssm, ssg = _scales_out(M, H, group_size, scale_layout, x.device, scales, mode)
+    st = lib.fp8q_add_rmsnorm_quant(x.data_ptr(), residual.data_ptr(), w.data_ptr(), ctypes.c_float(eps),
+                                    M, H, ldx, ldr, group_size, mode, q.data_ptr(), _rowmajor(q, "q"),
+                                    scales.data_ptr(), ssm, ssg, _stream(stream))
+    _check("fp8q_add_rmsnorm_quant", st)
     return q, scales
 
 
@@ -172,21 +225,23 @@ def fp8q_silu_mul_quant(x: torch.Tensor, group_size: int, ue8m0: bool = False, q
     ldx = _rowmajor(x, "x")
     M, I2 = x.shape
     I = I2 // 2
+    mode = _ue8m0_mode(ue8m0)
     if q is None:
         q = torch.empty((M, I), dtype=torch.float8_e4m3fn, device=x.device)
-    scales, ssm, ssg = _scales_out(M, I, group_size, scale_layout, x.device, scales)
-    st = lib.fp8q_silu_mul_quant(x.data_ptr(), M, I, ldx, group_size, int(ue8m0), q.data_ptr(),
+    scales, ssm, ssg = _scales_out(M, I, group_size, scale_layout, x.device, scales, mode)
+    st = lib.fp8q_silu_mul_quant(x.data_ptr(), M, I, ldx, group_size, mode, q.data_ptr(),
                                  _rowmajor(q, "q"), scales.data_ptr(), ssm, ssg, _stream(stream))
     _check("fp8q_silu_mul_quant", st)
     return q, scales
 
 
 # --------------------------------------------------------------------- GEMMs
-def fp8q_workspace_bytes(M: int, N: int, K: int, blockwise: bool) -> int:
+def fp8q_workspace_bytes(M: int, N: int, K: int, blockwise) -> int:
+    """blockwise: False (scaled_mm), True (scaled_mm_blockwise) or 2 (the E8M0 GEMM)."""
     return int(lib.fp8q_workspace_bytes(M, N, K, int(blockwise)))
 
 
-def make_workspace(M: int, N: int, K: int, blockwise: bool, device="cuda") -> torch.Tensor | None:
+def make_workspace(M: int, N: int, K: int, blockwise, device="cuda") -> torch.Tensor | None:
     """A zero-filled workspace for a GEMM of this shape (None if it needs none)."""
     n = fp8q_workspace_bytes(M, N, K, blockwise)
     return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
@@ -254,6 +309,31 @@ def fp8q_scaled_mm_blockwise(a_q: torch.Tensor, b_q: torch.Tensor, a_scale: torc
     return y
 
 
+def fp8q_scaled_mm_blockwise_e8m0(a_q: torch.Tensor, b_q: torch.Tensor, a_sf: torch.Tensor,
+                                  b_sf: torch.Tensor, a_scale_layout: str = "row_major", y=None,
+                                  workspace=None, stream=None):
+    """Block-scaled GEMM with E8M0 scale bytes (uint8): a_sf one byte per 1x128 group of
+    A ([M, K/128] row_major or [K/128, M] group_major), b_sf [N/128, K/128]; the
+    tensor core applies the scales (2^(byte - 127))."""
+    for t, n in ((a_q, "a_q"), (b_q, "b_q")):
+        _need(t, torch.float8_e4m3fn, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _need(a_sf, torch.uint8, "a_sf")
+    _need(b_sf, torch.uint8, "b_sf")
+    M, K = a_q.shape
+    N = b_q.shape[0]
+    sm, skb = (1, M) if a_scale_layout == "group_major" else (K // 128, 1)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_q.device)
+    wp, wn, _keep = _ws(workspace, M, N, K, 2, a_q.device)
+    st = lib.fp8q_scaled_mm_blockwise_e8m0(a_q.data_ptr(), b_q.data_ptr(), a_sf.data_ptr(), sm,
+                                           skb, b_sf.data_ptr(), M, N, K, y.data_ptr(),
+                                           _rowmajor(y, "y"), wp, wn, _stream(stream))
+    _check("fp8q_scaled_mm_blockwise_e8m0", st)
+    return y
+
+
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -277,6 +357,105 @@ def fp8q_scaled_mm_blockwise_noalloc(a_q: torch.Tensor, b_q: torch.Tensor, a_sca
                                               sm, skb, b_scale.data_ptr(), M, N, K, y.data_ptr(),
                                               _rowmajor(y, "y"), _stream(stream))
     _check("fp8q_scaled_mm_blockwise_noalloc", st)
+    return y
+
+
+# --------------------------------------------------------------- fused_qk_norm_rope
+def fp8q_qk_norm_rope(qkv: torch.Tensor, num_heads_q: int, num_heads_k: int, num_heads_v: int,
+                      head_dim: int, eps: float, q_weight: torch.Tensor, k_weight: torch.Tensor,
+                      cos_sin_cache: torch.Tensor, positions: torch.Tensor, is_neox: bool,
+                      stream=None) -> torch.Tensor:
+    """In place on qkv (bf16 [T, (hq+hk+hv)*D]): per-head RMSNorm of the q and k heads,
+    then the rotary embedding at positions (int64 [T]) from cos_sin_cache (fp32
+    [max_pos, D] = cos | sin).  Returns qkv."""
+    _need(qkv, torch.bfloat16, "qkv")
+    _need(q_weight, torch.bfloat16, "q_weight")
+    _need(k_weight, torch.bfloat16, "k_weight")
+    _need(cos_sin_cache, torch.float32, "cos_sin_cache")
+    _need(positions, torch.int64, "positions")
+    if not cos_sin_cache.is_contiguous() or not positions.is_contiguous():
+        raise ValueError("cos_sin_cache and positions must be contiguous")
+    ld = _rowmajor(qkv, "qkv")
+    T = qkv.shape[0]
+    _check("fp8q_qk_norm_rope", lib.fp8q_qk_norm_rope(
+        qkv.data_ptr(), T, ld, num_heads_q, num_heads_k, num_heads_v, head_dim, ctypes.c_float(eps),
+        q_weight.data_ptr(), k_weight.data_ptr(), cos_sin_cache.data_ptr(), cos_sin_cache.shape[0],
+        positions.data_ptr(), int(bool(is_neox)), _stream(stream)))
+    return qkv
+
+
+# --------------------------------------------------------------- W8A8_INT8
+def _quant_i8_out(M, L, group_size, layout, device, q, scales):
+    if q is None:
+        q = torch.empty((M, L), dtype=torch.int8, device=device)
+    elif q.dtype != torch.int8:
+        raise TypeError("q must be int8")
+    scales, ssm, ssg = _scales_out(M, L, group_size, layout, device, scales)
+    return q, scales, ssm, ssg
+
+
+def fp8q_group_quant_i8(x: torch.Tensor, group_size: int, q=None, scales=None,
+                        scale_layout: str = "row_major", stream=None):
+    """W8A8_INT8 quant (group_size = K per token, or 128): int8 codes, scale amax/127."""
+    _need(x, torch.bfloat16, "x")
+    ldx = _rowmajor(x, "x")
+    M, K = x.shape
+    q, scales, ssm, ssg = _quant_i8_out(M, K, group_size, scale_layout, x.device, q, scales)
+    _check("fp8q_group_quant_i8", lib.fp8q_group_quant_i8(
+        x.data_ptr(), M, K, ldx, group_size, q.data_ptr(), _rowmajor(q, "q"), scales.data_ptr(), ssm,
+        ssg, _stream(stream)))
+    return q, scales
+
+
+def fp8q_rmsnorm_quant_i8(x: torch.Tensor, w: torch.Tensor, eps: float, group_size: int, q=None,
+                          scales=None, scale_layout: str = "row_major", stream=None):
+    """RMSNorm + W8A8_INT8 quant."""
+    _need(x, torch.bfloat16, "x")
+    _need(w, torch.bfloat16, "w")
+    ldx = _rowmajor(x, "x")
+    M, H = x.shape
+    q, scales, ssm, ssg = _quant_i8_out(M, H, group_size, scale_layout, x.device, q, scales)
+    _check("fp8q_rmsnorm_quant_i8", lib.fp8q_rmsnorm_quant_i8(
+        x.data_ptr(), w.data_ptr(), ctypes.c_float(eps), M, H, ldx, group_size, q.data_ptr(),
+        _rowmajor(q, "q"), scales.data_ptr(), ssm, ssg, _stream(stream)))
+    return q, scales
+
+
+def fp8q_silu_mul_quant_i8(x: torch.Tensor, group_size: int, q=None, scales=None,
+                           scale_layout: str = "row_major", stream=None):
+    """SiLU*mul + W8A8_INT8 quant; x [M, 2I] = [gate | up]."""
+    _need(x, torch.bfloat16, "x")
+    ldx = _rowmajor(x, "x")
+    M, I2 = x.shape
+    I = I2 // 2
+    q, scales, ssm, ssg = _quant_i8_out(M, I, group_size, scale_layout, x.device, q, scales)
+    _check("fp8q_silu_mul_quant_i8", lib.fp8q_silu_mul_quant_i8(
+        x.data_ptr(), M, I, ldx, group_size, q.data_ptr(), _rowmajor(q, "q"), scales.data_ptr(), ssm,
+        ssg, _stream(stream)))
+    return q, scales
+
+
+def fp8q_scaled_mm_i8(a_q: torch.Tensor, b_q: torch.Tensor, a_scale: torch.Tensor,
+                      b_scale: torch.Tensor, y=None, workspace=None, stream=None):
+    """W8A8_INT8 GEMM: y [M, N] bf16 = sa * sb * (a_q [M, K] @ b_q [N, K]^T), int8 operands,
+    exact integer sums; a_scale fp32 [M] or [1], b_scale fp32 [N] or [1]."""
+    for t, n in ((a_q, "a_q"), (b_q, "b_q")):
+        _need(t, torch.int8, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _need(a_scale, torch.float32, "a_scale")
+    _need(b_scale, torch.float32, "b_scale")
+    M, K = a_q.shape
+    N = b_q.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=a_q.device)
+    if a_scale.numel() not in (1, M) or b_scale.numel() not in (1, N):
+        raise ValueError("a_scale must have 1 or M entries, b_scale 1 or N")
+    wp, wn, _keep = _ws(workspace, M, N, K, 3, a_q.device)
+    _check("fp8q_scaled_mm_i8", lib.fp8q_scaled_mm_i8(
+        a_q.data_ptr(), b_q.data_ptr(), a_scale.data_ptr(), int(a_scale.numel() == M),
+        b_scale.data_ptr(), int(b_scale.numel() == N), M, N, K, y.data_ptr(), _rowmajor(y, "y"), wp,
+        wn, _stream(stream)))
     return y
 
 

@@ -81,5 +81,28 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_variant(out_dir: str, defines: list[str]) -> str:
+    """Build a separate copy of the library with extra preprocessor defines
+    (test-only builds, e.g. a shortened device wait limit) into out_dir; the
+    shipped libfp8q.so is not touched."""
+    os.makedirs(out_dir, exist_ok=True)
+    lib = os.path.join(out_dir, "libfp8q.so")
+    objs, jobs = [], []
+    for src in _sources():
+        obj = os.path.join(out_dir, os.path.splitext(os.path.basename(src))[0] + ".o")
+        objs.append(obj)
+        jobs.append([nvcc(), *NVCC_FLAGS, *[f"-D{d}" for d in defines], "-c", src, "-o", obj])
+    with cf.ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 4)) as ex:
+        results = list(ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), jobs))
+    for c, r in zip(jobs, results):
+        if r.returncode != 0:
+            raise RuntimeError(f"nvcc failed: {' '.join(c)}\n{r.stderr[-4000:]}")
+    r = subprocess.run([nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", lib],
+                       capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"link failed:\n{r.stderr[-4000:]}")
+    return lib
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True)

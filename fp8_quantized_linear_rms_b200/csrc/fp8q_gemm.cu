@@ -49,6 +49,16 @@ constexpr int UMMA_K = 32;    // K per tcgen05.mma for 8-bit operands
 constexpr int A_BYTES = BM * BK;
 constexpr int kSmemBudget = 200 * 1024;
 
+// Test-only build switch (-DFP8Q_TEST_STALL_PRODUCER=1, never in the shipped
+// library): the GEMM's TMA producer issues nothing, so the MMA thread's first
+// pipeline wait runs out and the kernel takes its timeout path (abort flag,
+// FP8Q_ERR_TIMEOUT in the status word, drain, TMEM release, return).
+#ifdef FP8Q_TEST_STALL_PRODUCER
+constexpr bool kTestStallProducer = FP8Q_TEST_STALL_PRODUCER != 0;
+#else
+constexpr bool kTestStallProducer = false;
+#endif
+
 struct GemmArgs {
   int rows_a, rows_b, K;              // MMA-A rows (TMEM lanes), MMA-B rows (columns)
   int kblocks, tiles_a, tiles_b, split, kb_per_split, units;  // classic: tiles x split units
@@ -65,27 +75,46 @@ struct GemmArgs {
   float* ws;                          // split-K partials
   int* counters;                      // split-K arrival counters (zero between calls)
   int* status;                        // device status word
+  // E8M0 block scales (block-scaled MMA): activations sfa[m*sfa_sm + kb*sfa_skb],
+  // weights sfb[(n/128)*sfb_snb + kb]
+  const uint8_t* sfa;
+  int64_t sfa_sm, sfa_skb;
+  const uint8_t* sfb;
+  int64_t sfb_snb;
 };
 
-template <int BN, bool SWAP, bool BW>
+// MX: E8M0 block scales applied by the tensor core (kind::mxf8f6f4.block_scale);
+// the accumulator then needs no scaling, as with unit per-token scales.
+// I8: W8A8_INT8, signed 8-bit operands (kind::i8) with s32 accumulators and
+// per-token / per-channel scales.
+template <int BN, bool SWAP, bool BW, bool MX = false, bool I8 = false>
 struct Cfg {
+  static_assert(!(BW && MX) && !(I8 && (BW || MX)), "one scale scheme");
   static constexpr int B_BYTES = BN * BK;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;           // TMA bytes per stage
+  // Scale factors per stage (MX): one 512-byte chunk for the 128 MMA rows,
+  // one per 128 MMA columns; in TMEM 4 columns per chunk, double-buffered.
+  static constexpr int SFB_CHUNKS = (BN + 127) / 128;
+  static constexpr int SF_BYTES = MX ? 512 * (1 + SFB_CHUNKS) : 0;
+  static constexpr int SF_COLS = 4 * (1 + SFB_CHUNKS);
+  static constexpr int STAGES_RAW = kSmemBudget / (STAGE_BYTES + SF_BYTES);
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
-  static constexpr int EPI_WARPS = (BW && BN >= 256) ? 16 : ((BW && BN >= 128) ? 8 : 4);
+  static constexpr int EPI_WARPS = (BW && BN >= 128) ? 8 : 4;
   static constexpr int COL_GROUPS = EPI_WARPS / 4;        // column slices per TMEM lane quadrant
   static constexpr int CPT = BN / COL_GROUPS;              // columns per epilogue thread
-  // Columns per tcgen05.ld.  The 16-warp variant holds 64 fp32 accumulators
-  // per thread in a 96-register budget, so it reads 8 columns at a time.
-  static constexpr int CHUNK = EPI_WARPS == 16 ? 8 : (CPT < 32 ? 16 : 32);
+  // Columns per tcgen05.ld.  The blockwise epilogue keeps two chunks in
+  // flight (the next one loads while the current one is scaled); its
+  // 256-column tile holds 128 fp32 accumulators per thread (8 epilogue warps,
+  // 10 in all: 168 registers a thread), so it reads 8 columns at a time.
+  static constexpr int CHUNK = BW ? (CPT >= 128 ? 8 : 16) : (CPT < 32 ? 16 : 32);
   static constexpr int NBUF = (BW && BN < 256) ? 4 : 2;    // TMEM accumulator buffers
-  static constexpr int TMEM_NEED = NBUF * BN;
+  static constexpr int SF_COL0 = NBUF * BN;                 // first scale-factor column (MX)
+  static constexpr int TMEM_NEED = NBUF * BN + (MX ? 2 * SF_COLS : 0);
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                  : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * NBUF + 1) + 16;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * (STAGE_BYTES + SF_BYTES) + BAR_BYTES;
   static_assert(STAGES >= 2, "pipeline too shallow");
   static_assert(TMEM_NEED <= 512, "accumulators exceed TMEM");
   static_assert(CPT % CHUNK == 0 && (CHUNK == 8 || CHUNK == 16 || CHUNK == 32), "chunking");
@@ -173,11 +202,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int BN, bool SWAP, bool BW>
-__global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
+template <int BN, bool SWAP, bool BW, bool MX, bool I8>
+__global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs p) {
-  using C = Cfg<BN, SWAP, BW>;
+  using C = Cfg<BN, SWAP, BW, MX, I8>;
   constexpr int S = C::STAGES;
   constexpr int NB = C::NBUF;
   extern __shared__ uint8_t smem_raw[];
@@ -185,7 +214,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * C::B_BYTES);
+  uint8_t* sSF = sB + S * C::B_BYTES;                      // MX: scale factors per stage
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSF + S * C::SF_BYTES);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + NB;
@@ -237,8 +267,9 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
   griddep_launch_dependents();
 
   if (warp == 0) {
+   if constexpr (!MX) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && !kTestStallProducer) {
       int it = 0;
       bool ok = true;
       SegIter si(p);
@@ -260,10 +291,131 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
       }
     }
     __syncwarp();
+   } else {
+    // ------------------------------------------------------------ producer (MX, whole warp)
+    // Per stage, lane l writes the E8M0 scale factors of MMA rows l + 32 j
+    // (chunk 0) and MMA columns 128 h + l + 32 j (chunk 1 + h), each byte
+    // repeated over the four 32-deep K slices of the stage, at byte
+    // l * 16 + j * 4 of its chunk; then lane 0 arms the stage and issues its
+    // TMA loads.  Rows or columns outside the problem take the scale 1 (byte
+    // 127): their operands are zero-filled by TMA.  The scale bytes of a
+    // stage are loaded SFD stages ahead (a register ring), so their global
+    // latency hides behind the MMAs of the stages before it.
+    //   no swap: raw[0..3] = A bytes of rows l + 32 j, raw[4..6] = the B
+    //            bytes of the (at most three) 128-row weight blocks the
+    //            tile's columns fall in;
+    //   swap:    raw[0] = the weight block row's byte (the 128 MMA rows are
+    //            one block row), raw[1 + 4 h + j] = token column 128 h + l + 32 j.
+    constexpr int SFD = 4;
+    constexpr int NRAW = SWAP ? 1 + 4 * C::SFB_CHUNKS : 7;
+    constexpr uint32_t kOneByte = 127u;
+    const int nb_rows = p.N >> 7;                    // weight block rows
+    uint32_t raw[SFD][NRAW];
+    // iterator SFD stages ahead of the one being armed
+    SegIter sai(p);
+    Seg ga;
+    bool amore = sai.next(p, ga);
+    int akb = amore ? ga.kb0 : 0;
+    auto load_ahead = [&](uint32_t* r) {
+      if (!amore) {
+#pragma unroll
+        for (int i = 0; i < NRAW; ++i) r[i] = kOneByte;
+        return;
+      }
+      if (!SWAP) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int m = ga.ta * BM + lane + 32 * j;
+          r[j] = m < p.M ? __ldg(p.sfa + m * p.sfa_sm + akb * p.sfa_skb) : kOneByte;
+        }
+        const int nb0 = (ga.tb * BN) >> 7;
+#pragma unroll
+        for (int i = 0; i < 3; ++i)
+          r[4 + i] = nb0 + i < nb_rows ? __ldg(p.sfb + (nb0 + i) * p.sfb_snb + akb) : kOneByte;
+      } else {
+        r[0] = __ldg(p.sfb + ga.ta * p.sfb_snb + akb);
+#pragma unroll
+        for (int h = 0; h < C::SFB_CHUNKS; ++h)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = 128 * h + lane + 32 * j;
+            const int m = ga.tb * BN + c;
+            r[1 + 4 * h + j] = (c < BN && m < p.M) ? __ldg(p.sfa + m * p.sfa_sm + akb * p.sfa_skb) : kOneByte;
+          }
+      }
+      if (++akb >= ga.kb1) {
+        amore = sai.next(p, ga);
+        if (amore) akb = ga.kb0;
+      }
+    };
+#pragma unroll
+    for (int d = 0; d < SFD; ++d) load_ahead(raw[d]);
+    int it = 0;
+    bool ok = true;
+    SegIter si(p);
+    Seg g;
+    while (ok && si.next(p, g)) {
+      for (int kb = g.kb0; kb < g.kb1; ++kb, ++it) {
+        const int st = it % S;
+        const uint32_t ph = (it / S) & 1;
+        uint32_t cur[NRAW];
+#pragma unroll
+        for (int i = 0; i < NRAW; ++i) cur[i] = raw[0][i];
+#pragma unroll
+        for (int d = 0; d + 1 < SFD; ++d)
+#pragma unroll
+          for (int i = 0; i < NRAW; ++i) raw[d][i] = raw[d + 1][i];
+        load_ahead(raw[SFD - 1]);
+        int w_ok = 1;
+        if (lane == 0) w_ok = mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status);
+        if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) { ok = false; break; }
+        uint32_t wa[4], wb[C::SFB_CHUNKS][4];
+        if (!SWAP) {
+          const int nb0 = (g.tb * BN) >> 7;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) wa[j] = cur[j] * 0x01010101u;
+#pragma unroll
+          for (int h = 0; h < C::SFB_CHUNKS; ++h)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int c = 128 * h + lane + 32 * j;
+              const int rel = ((g.tb * BN + c) >> 7) - nb0;        // 0, 1 or 2
+              const uint32_t b = rel == 0 ? cur[4] : (rel == 1 ? cur[5] : cur[6]);
+              wb[h][j] = (c < BN ? b : kOneByte) * 0x01010101u;
+            }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) wa[j] = cur[0] * 0x01010101u;
+#pragma unroll
+          for (int h = 0; h < C::SFB_CHUNKS; ++h)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) wb[h][j] = cur[1 + 4 * h + j] * 0x01010101u;
+        }
+        uint32_t* sf = reinterpret_cast<uint32_t*>(sSF + st * C::SF_BYTES);
+        *reinterpret_cast<uint4*>(sf + lane * 4) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+#pragma unroll
+        for (int h = 0; h < C::SFB_CHUNKS; ++h)
+          *reinterpret_cast<uint4*>(sf + 128 * (1 + h) + lane * 4) =
+              make_uint4(wb[h][0], wb[h][1], wb[h][2], wb[h][3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+          tma_load_2d(sA + st * A_BYTES, &tmA, &full[st], kb * BK, g.ta * BM);
+          tma_load_2d(sB + st * C::B_BYTES, &tmB, &full[st], kb * BK, g.tb * BN);
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      const int first = it - S > 0 ? it - S : 0;
+      for (int j = first; j < it; ++j) drain_wait(&full[j % S], (j / S) & 1);
+    }
+    __syncwarp();
+   }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      constexpr uint32_t idesc = I8 ? idesc_s8_s32(BM, BN) : idesc_e4m3_f32(BM, BN);
       int it = 0, t = 0, pc = 0;
       bool ok = true;
       SegIter si(p);
@@ -291,10 +443,29 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
           tc_fence_after();
           const uint64_t adesc = smem_desc_kmajor_sw128(sA + st * A_BYTES);
           const uint64_t bdesc = smem_desc_kmajor_sw128(sB + st * C::B_BYTES);
+          if constexpr (MX) {
+            // this stage's scale factors into TMEM (slot alternates per
+            // stage), then the four block-scaled MMAs of the stage; tcgen05
+            // ops of one thread run in issue order.
+            const uint32_t sf = tmem_base + C::SF_COL0 + (it & 1) * C::SF_COLS;
+            const uint8_t* ssf = sSF + st * C::SF_BYTES;
+            tmem_cp_sf_chunk(sf, ssf);
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
-            const uint32_t acc = BW ? (k > 0) : (kb > kb0 || k > 0);
-            mma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);  // +32 bytes of K
+            for (int h = 0; h < C::SFB_CHUNKS; ++h) tmem_cp_sf_chunk(sf + 4 + 4 * h, ssf + 512 * (1 + h));
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              const uint32_t acc = (kb > kb0 || k > 0);
+              const uint32_t kid = static_cast<uint32_t>(k) << 30;
+              mma_mxf8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc_mx_e4m3(BM, BN, k), acc, sf | kid,
+                           (sf + 4) | kid);
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              const uint32_t acc = BW ? (k > 0) : (kb > kb0 || k > 0);
+              if constexpr (I8) mma_i8(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
+              else mma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);  // +32 bytes of K
+            }
           }
           mma_commit(&empty[st]);
           if (BW) {
@@ -432,22 +603,24 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
         }
       };
 
-      if (!BW) {
+      if constexpr (!BW) {
         // -------- per-token / per-channel scales: one accumulator per tile
         // Column scales: lane l of the warp loads the scale of column c + l of
         // every chunk (one load per 32 columns, issued before the wait), and the
         // products broadcast it with a shuffle.
         constexpr int NCH = C::CPT / C::CHUNK;
         const int buf = t & 1;
-        float srow;
-        if (!SWAP) srow = a_valid ? __ldg(p.sa + a_idx * p.sa_sm) : 0.0f;
-        else srow = a_valid ? __ldg(p.sb + a_idx * p.sb_sn) : 0.0f;
+        float srow = 1.0f;
         float colsc[NCH];
+        if constexpr (!MX) {
+          if (!SWAP) srow = a_valid ? __ldg(p.sa + a_idx * p.sa_sm) : 0.0f;
+          else srow = a_valid ? __ldg(p.sb + a_idx * p.sb_sn) : 0.0f;
 #pragma unroll
-        for (int j = 0; j < NCH; ++j) {
-          const int b_idx = b_base + col0 + j * C::CHUNK + lane;
-          if (!SWAP) colsc[j] = (lane < C::CHUNK && b_idx < p.N) ? __ldg(p.sb + b_idx * p.sb_sn) : 0.0f;
-          else colsc[j] = (lane < C::CHUNK && b_idx < p.M) ? __ldg(p.sa + b_idx * p.sa_sm) : 0.0f;
+          for (int j = 0; j < NCH; ++j) {
+            const int b_idx = b_base + col0 + j * C::CHUNK + lane;
+            if (!SWAP) colsc[j] = (lane < C::CHUNK && b_idx < p.N) ? __ldg(p.sb + b_idx * p.sb_sn) : 0.0f;
+            else colsc[j] = (lane < C::CHUNK && b_idx < p.M) ? __ldg(p.sa + b_idx * p.sa_sm) : 0.0f;
+          }
         }
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[buf], (t >> 1) & 1, abort_flag, p.status))) {
           ok = false;
@@ -461,8 +634,12 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
           tmem_ld_waited<C::CHUNK>(tmem_base + lane_addr + buf * BN + c, r);
           float v[C::CHUNK];
 #pragma unroll
-          for (int i = 0; i < C::CHUNK; ++i)
-            v[i] = __uint_as_float(r[i]) * (srow * __shfl_sync(0xFFFFFFFFu, colsc[j], i));
+          for (int i = 0; i < C::CHUNK; ++i) {
+            if constexpr (MX) v[i] = __uint_as_float(r[i]);
+            else if constexpr (I8)   // exact s32 sum -> fp32 (one rounding beyond 2^24)
+              v[i] = __int2float_rn(static_cast<int>(r[i])) * (srow * __shfl_sync(0xFFFFFFFFu, colsc[j], i));
+            else v[i] = __uint_as_float(r[i]) * (srow * __shfl_sync(0xFFFFFFFFu, colsc[j], i));
+          }
           if (g.ncontrib == 1) emit(c, v);
           else stash(c, v);
         }
@@ -479,7 +656,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
         // before it.  Swap-AB: the scale varies per column (token); lane l
         // holds that of column c + l of every chunk.
         constexpr int NCH = C::CPT / C::CHUNK;
-        constexpr int SD = C::EPI_WARPS == 16 ? 1 : 4;
+        constexpr int SD = 4;
         uint64_t acc[C::CPT / 2];                      // fp32 pairs, columns 2i, 2i+1
 #pragma unroll
         for (int i = 0; i < C::CPT / 2; ++i) acc[i] = 0ull;
@@ -533,14 +710,19 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
             break;
           }
           tc_fence_after();
-          // One chunk per load+wait; the buffer is handed back to the MMA as
-          // soon as the last chunk has landed, before its FMAs.
+          // Chunk j + 1 is loaded while chunk j is scaled into the
+          // accumulators; the buffer is handed back to the MMA as soon as the
+          // last chunk has landed, before its FMAs.
           const uint32_t tbuf = tmem_base + lane_addr + pb * BN + col0;
+          uint32_t r[2][C::CHUNK];
+          tmem_ld_async<C::CHUNK>(tbuf, r[0]);
 #pragma unroll
           for (int j = 0; j < NCH; ++j) {
-            uint32_t r[C::CHUNK];
-            tmem_ld_waited<C::CHUNK>(tbuf + j * C::CHUNK, r);
-            if (j == NCH - 1) {
+            uint32_t* rc = r[j & 1];
+            tmem_wait_regs<C::CHUNK>(rc);
+            if (j + 1 < NCH) {
+              tmem_ld_async<C::CHUNK>(tbuf + (j + 1) * C::CHUNK, r[(j + 1) & 1]);
+            } else {
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&tempty[pb]);
@@ -550,7 +732,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW>::THREADS, 1)
               const uint64_t sc = SWAP ? pair_f32(__shfl_sync(0xFFFFFFFFu, sc0[SWAP ? j : 0], i),
                                                   __shfl_sync(0xFFFFFFFFu, sc0[SWAP ? j : 0], i + 1))
                                        : srow2;
-              ffma2_acc(acc[(j * C::CHUNK + i) / 2], r[i], r[i + 1], sc);
+              ffma2_acc(acc[(j * C::CHUNK + i) / 2], rc[i], rc[i + 1], sc);
             }
           }
           if (++pb == NB) {
@@ -616,7 +798,7 @@ struct Cfg2 {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-template <int BN, bool BW>
+template <int BN, bool BW, bool I8 = false>
 __global__ void __launch_bounds__(Cfg2<BN, BW>::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmArgs p) {
@@ -706,7 +888,7 @@ __global__ void __launch_bounds__(Cfg2<BN, BW>::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(2 * BM, BN);
+      constexpr uint32_t idesc = I8 ? idesc_s8_s32(2 * BM, BN) : idesc_e4m3_f32(2 * BM, BN);
       int it = 0, t = 0, pc = 0;
       bool ok = true;
       for (int u = pair; ok && u < p.units; u += npairs) {
@@ -734,7 +916,8 @@ __global__ void __launch_bounds__(Cfg2<BN, BW>::THREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
             const uint32_t acc = BW ? (k > 0) : (kb > 0 || k > 0);
-            mma_f8f6f4_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
+            if constexpr (I8) mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
+            else mma_f8f6f4_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
           }
           mma_commit_pair(&empty[st], 0x3);
           if (BW) {
@@ -807,8 +990,10 @@ __global__ void __launch_bounds__(Cfg2<BN, BW>::THREADS, 1)
           tmem_ld_waited<C::CHUNK>(tmem_base + lane_addr + buf * BN + col0 + j * C::CHUNK, r);
           float v[C::CHUNK];
 #pragma unroll
-          for (int i = 0; i < C::CHUNK; ++i)
-            v[i] = __uint_as_float(r[i]) * (srow * __shfl_sync(0xFFFFFFFFu, colsc[j], i));
+          for (int i = 0; i < C::CHUNK; ++i) {
+            const float a = I8 ? __int2float_rn(static_cast<int>(r[i])) : __uint_as_float(r[i]);
+            v[i] = a * (srow * __shfl_sync(0xFFFFFFFFu, colsc[j], i));
+          }
           emit(col0 + j * C::CHUNK, v);
         }
         tc_fence_before();
@@ -952,10 +1137,10 @@ bool tensor_map(const void* ptr, int64_t rows, int64_t k, int box_rows, CUtensor
   return true;
 }
 
-template <int BN, bool SWAP, bool BW>
+template <int BN, bool SWAP, bool BW, bool MX = false, bool I8 = false>
 fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
                         cudaStream_t stream) {
-  using C = Cfg<BN, SWAP, BW>;
+  using C = Cfg<BN, SWAP, BW, MX, I8>;
   CUtensorMap ma, mb;
   if (!tensor_map(a_op, p.rows_a, p.K, BM, &ma) || !tensor_map(b_op, p.rows_b, p.K, BN, &mb))
     return FP8Q_ERR_CUDA;
@@ -963,7 +1148,7 @@ fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev].load(std::memory_order_relaxed)) {
-    if (cudaFuncSetAttribute(gemm_kernel<BN, SWAP, BW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gemm_kernel<BN, SWAP, BW, MX, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return FP8Q_ERR_CUDA;
     attr_done[dev].store(1, std::memory_order_relaxed);
@@ -971,13 +1156,13 @@ fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
   int grid;
   if (p.streamk) grid = (p.total_iters + p.seg_len - 1) / p.seg_len;
   else grid = p.units < num_sms() ? p.units : num_sms();
-  return launch_kernel(gemm_kernel<BN, SWAP, BW>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream,
-                       1, ma, mb, p);
+  return launch_kernel(gemm_kernel<BN, SWAP, BW, MX, I8>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES,
+                       stream, 1, ma, mb, p);
 }
 
 // Clusters of two CTAs that can be resident at once (cached per kernel and
 // device); the pair kernel is persistent over that many pairs.
-template <int BN, bool BW>
+template <int BN, bool BW, bool I8 = false>
 int pair_clusters() {
   static std::atomic<int> cache[64];
   int dev = 0;
@@ -997,13 +1182,13 @@ int pair_clusters() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<BN, BW>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<BN, BW, I8>, &cfg) != cudaSuccess) n = 0;
     cache[dev].store(n, std::memory_order_relaxed);
   }
   return cache[dev].load(std::memory_order_relaxed);
 }
 
-template <int BN, bool BW>
+template <int BN, bool BW, bool I8 = false>
 fp8q_status launch_pair(const void* a_op, const void* b_op, const GemmArgs& p, cudaStream_t stream) {
   using C = Cfg2<BN, BW>;
   CUtensorMap ma, mb;
@@ -1013,15 +1198,15 @@ fp8q_status launch_pair(const void* a_op, const void* b_op, const GemmArgs& p, c
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev].load(std::memory_order_relaxed)) {
-    if (cudaFuncSetAttribute(gemm_pair_kernel<BN, BW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gemm_pair_kernel<BN, BW, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return FP8Q_ERR_CUDA;
     attr_done[dev].store(1, std::memory_order_relaxed);
   }
-  const int nc = pair_clusters<BN, BW>();
+  const int nc = pair_clusters<BN, BW, I8>();
   if (nc < 1) return FP8Q_ERR_UNSUPPORTED;
   const int npairs = p.units < nc ? p.units : nc;
-  return launch_kernel(gemm_pair_kernel<BN, BW>, dim3(2 * static_cast<unsigned>(npairs)),
+  return launch_kernel(gemm_pair_kernel<BN, BW, I8>, dim3(2 * static_cast<unsigned>(npairs)),
                        dim3(C::THREADS), C::SMEM_BYTES, stream, 2, ma, mb, p);
 }
 
@@ -1031,8 +1216,17 @@ std::mutex g_force_mu;
 bool g_forced = false;
 fp8q_gemm_variant g_force{0, 1, 128, 0};
 
+// blockwise: 0 per-token / per-channel scales, 1 fp32 block scales, 2 E8M0
+// block scales (block-scaled MMA).
 bool variant_supported(const fp8q_gemm_variant& v, int blockwise) {
   if (v.cta_pair != 0 && v.cta_pair != 1) return false;
+  if (blockwise == 3) blockwise = 0;   // int8: the per-token scheme's variants
+  if (blockwise == 2) {
+    // single CTAs only; 224-column tiles leave TMEM room for the scale factors
+    if (v.cta_pair || v.split_k < 0 || v.split_k > 64) return false;
+    if (v.swap_ab) return v.block_n == 16 || v.block_n == 32 || v.block_n == 64 || v.block_n == 128;
+    return v.block_n == 128 || v.block_n == 224;
+  }
   // (pairs: blockwise with 128-column tiles -- four accumulator buffers --,
   // per token with 128 or 256)
   if (v.cta_pair) return !v.swap_ab && v.split_k == 1 && (v.block_n == 128 || (!blockwise && v.block_n == 256));
@@ -1043,7 +1237,8 @@ bool variant_supported(const fp8q_gemm_variant& v, int blockwise) {
 }
 
 int epi_warps(const fp8q_gemm_variant& v, int blockwise) {
-  if (blockwise && v.block_n >= 256) return 16;
+  if (blockwise == 2 || blockwise == 3) return 4;
+  if (v.cta_pair) return blockwise ? (v.block_n >= 256 ? 16 : 8) : 4;
   return (blockwise && v.block_n >= 128) ? 8 : 4;
 }
 
@@ -1133,6 +1328,16 @@ fp8q_gemm_variant pick_variant(int64_t M, int64_t N, int64_t K, int blockwise,
     if (forced) *forced = g_forced;
     if (g_forced) return g_force;
   }
+  if (blockwise == 3) return auto_variant(M, N, K, 0);   // int8: same kernel structure
+  if (blockwise == 2) {
+    // The block-scaled MMA keeps the whole K loop in TMEM like the per-token
+    // kernel, so it follows the per-token scheme's measured choice, on
+    // single CTAs with 224-column tiles where that takes 256-column tiles.
+    fp8q_gemm_variant v = auto_variant(M, N, K, 0);
+    if (v.cta_pair) v = fp8q_gemm_variant{0, 1, 224, 0};
+    if (!v.swap_ab && v.block_n == 256) v.block_n = 224;
+    return v;
+  }
   return auto_variant(M, N, K, blockwise);
 }
 
@@ -1194,7 +1399,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int blockwise, const fp8q_gemm_v
   return pl;
 }
 
-template <bool BW>
+template <bool BW, bool MX = false, bool I8 = false>
 fp8q_status run_gemm(const void* a_q, const void* b_q, GemmArgs& p, const Plan& pl, void* ws,
                      cudaStream_t stream) {
   p.tiles_a = pl.tiles_a;
@@ -1211,12 +1416,31 @@ fp8q_status run_gemm(const void* a_q, const void* b_q, GemmArgs& p, const Plan& 
   p.ws = pl.max_contrib > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.counter_bytes) : nullptr;
   p.status = device_status_ptr();
   const int bn = pl.v.block_n;
+  if constexpr (MX) {
+    if (pl.v.cta_pair) return FP8Q_ERR_UNSUPPORTED;
+    if (pl.v.swap_ab) {
+      p.rows_a = p.N;
+      p.rows_b = p.M;
+      switch (bn) {
+        case 16: return launch_gemm<16, true, false, true>(b_q, a_q, p, stream);
+        case 32: return launch_gemm<32, true, false, true>(b_q, a_q, p, stream);
+        case 64: return launch_gemm<64, true, false, true>(b_q, a_q, p, stream);
+        case 128: return launch_gemm<128, true, false, true>(b_q, a_q, p, stream);
+        default: return FP8Q_ERR_UNSUPPORTED;
+      }
+    }
+    p.rows_a = p.M;
+    p.rows_b = p.N;
+    if (bn == 128) return launch_gemm<128, false, false, true>(a_q, b_q, p, stream);
+    if (bn == 224) return launch_gemm<224, false, false, true>(a_q, b_q, p, stream);
+    return FP8Q_ERR_UNSUPPORTED;
+  }
   if (pl.v.cta_pair) {
     p.rows_a = p.M;
     p.rows_b = p.N;
-    if (bn == 128) return launch_pair<128, BW>(a_q, b_q, p, stream);
+    if (bn == 128) return launch_pair<128, BW, I8>(a_q, b_q, p, stream);
     if constexpr (!BW) {
-      if (bn == 256) return launch_pair<256, false>(a_q, b_q, p, stream);
+      if (bn == 256) return launch_pair<256, false, I8>(a_q, b_q, p, stream);
     }
     return FP8Q_ERR_UNSUPPORTED;
   }
@@ -1224,17 +1448,17 @@ fp8q_status run_gemm(const void* a_q, const void* b_q, GemmArgs& p, const Plan& 
     p.rows_a = p.N;
     p.rows_b = p.M;
     switch (bn) {
-      case 16: return launch_gemm<16, true, BW>(b_q, a_q, p, stream);
-      case 32: return launch_gemm<32, true, BW>(b_q, a_q, p, stream);
-      case 64: return launch_gemm<64, true, BW>(b_q, a_q, p, stream);
-      case 128: return launch_gemm<128, true, BW>(b_q, a_q, p, stream);
+      case 16: return launch_gemm<16, true, BW, false, I8>(b_q, a_q, p, stream);
+      case 32: return launch_gemm<32, true, BW, false, I8>(b_q, a_q, p, stream);
+      case 64: return launch_gemm<64, true, BW, false, I8>(b_q, a_q, p, stream);
+      case 128: return launch_gemm<128, true, BW, false, I8>(b_q, a_q, p, stream);
       default: return FP8Q_ERR_UNSUPPORTED;
     }
   }
   p.rows_a = p.M;
   p.rows_b = p.N;
-  if (bn == 128) return launch_gemm<128, false, BW>(a_q, b_q, p, stream);
-  if (bn == 256) return launch_gemm<256, false, BW>(a_q, b_q, p, stream);
+  if (bn == 128) return launch_gemm<128, false, BW, false, I8>(a_q, b_q, p, stream);
+  if (bn == 256) return launch_gemm<256, false, BW, false, I8>(a_q, b_q, p, stream);
   return FP8Q_ERR_UNSUPPORTED;
 }
 
@@ -1282,14 +1506,15 @@ extern "C" fp8q_status fp8q_force_gemm_variant(const fp8q_gemm_variant* v) {
     g_forced = false;
     return FP8Q_OK;
   }
-  if (!variant_supported(*v, 0) && !variant_supported(*v, 1)) return FP8Q_ERR_INVALID_ARG;
+  if (!variant_supported(*v, 0) && !variant_supported(*v, 1) && !variant_supported(*v, 2))
+    return FP8Q_ERR_INVALID_ARG;
   g_force = *v;
   g_forced = true;
   return FP8Q_OK;
 }
 
 extern "C" size_t fp8q_workspace_bytes(int64_t M, int64_t N, int64_t K, int blockwise) {
-  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  if (M <= 0 || N <= 0 || K <= 0 || blockwise < 0 || blockwise > 3) return 0;
   const fp8q_gemm_variant v = pick_variant(M, N, K, blockwise);
   return make_plan(M, N, K, blockwise, v).ws_bytes;
 }
@@ -1355,6 +1580,67 @@ extern "C" fp8q_status fp8q_scaled_mm_blockwise(const void* a_q, const void* b_q
   p.y = static_cast<uint16_t*>(y);
   p.ldy = ldy;
   return run_gemm<true>(a_q, b_q, p, pl, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fp8q_status fp8q_scaled_mm_i8(const void* a_q, const void* b_q, const float* a_scale,
+                                         int a_per_token, const float* b_scale, int b_per_channel,
+                                         int64_t M, int64_t N, int64_t K, void* y, int64_t ldy,
+                                         void* workspace, size_t ws_bytes, void* stream) {
+  fp8q_status st = check_gemm(a_q, b_q, a_scale, b_scale, M, N, K, y, ldy);
+  if (st != FP8Q_OK) return st;
+  if ((a_per_token != 0 && a_per_token != 1) || (b_per_channel != 0 && b_per_channel != 1))
+    return FP8Q_ERR_INVALID_ARG;
+  if (K > 133152) return FP8Q_ERR_INVALID_ARG;   // 128^2 K must stay below 2^31
+  if (M == 0) return FP8Q_OK;
+  const fp8q_gemm_variant v = pick_variant(M, N, K, 3);
+  if (!variant_supported(v, 3)) return FP8Q_ERR_UNSUPPORTED;
+  const Plan pl = make_plan(M, N, K, 3, v);
+  if (pl.ws_bytes > 0 && (!workspace || ws_bytes < pl.ws_bytes || !aligned(workspace, 256)))
+    return FP8Q_ERR_INVALID_ARG;
+  GemmArgs p{};
+  p.K = static_cast<int>(K);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.sa = a_scale;
+  p.sa_sm = a_per_token ? 1 : 0;
+  p.sb = b_scale;
+  p.sb_sn = b_per_channel ? 1 : 0;
+  p.y = static_cast<uint16_t*>(y);
+  p.ldy = ldy;
+  return run_gemm<false, false, true>(a_q, b_q, p, pl, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fp8q_status fp8q_scaled_mm_blockwise_e8m0(const void* a_q, const void* b_q,
+                                                     const uint8_t* a_sf, int64_t as_stride_m,
+                                                     int64_t as_stride_kb, const uint8_t* b_sf,
+                                                     int64_t M, int64_t N, int64_t K, void* y,
+                                                     int64_t ldy, void* workspace, size_t ws_bytes,
+                                                     void* stream) {
+  if (M < 0 || N <= 0 || K <= 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
+    return FP8Q_ERR_INVALID_ARG;
+  if (N % 128 != 0 || K % 128 != 0 || ldy < N || ldy % 8 != 0 || as_stride_m < 0 || as_stride_kb < 0)
+    return FP8Q_ERR_INVALID_ARG;
+  if (M == 0) return FP8Q_OK;
+  if (!a_q || !b_q || !a_sf || !b_sf || !y) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(a_q, 16) || !aligned(b_q, 16) || !aligned(y, 16)) return FP8Q_ERR_INVALID_ARG;
+  if (!scale_offsets_fit(M, K, as_stride_m, as_stride_kb)) return FP8Q_ERR_INVALID_ARG;
+  const fp8q_gemm_variant v = pick_variant(M, N, K, 2);
+  if (!variant_supported(v, 2)) return FP8Q_ERR_UNSUPPORTED;
+  const Plan pl = make_plan(M, N, K, 2, v);
+  if (pl.ws_bytes > 0 && (!workspace || ws_bytes < pl.ws_bytes || !aligned(workspace, 256)))
+    return FP8Q_ERR_INVALID_ARG;
+  GemmArgs p{};
+  p.K = static_cast<int>(K);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.sfa = a_sf;
+  p.sfa_sm = as_stride_m;
+  p.sfa_skb = as_stride_kb;
+  p.sfb = b_sf;
+  p.sfb_snb = K / 128;
+  p.y = static_cast<uint16_t*>(y);
+  p.ldy = ldy;
+  return run_gemm<false, true>(a_q, b_q, p, pl, workspace, static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------ no-allocation path

@@ -42,7 +42,9 @@ namespace {
 
 using namespace sm100;
 
-enum { OP_PLAIN = 0, OP_RMS = 1, OP_SILU = 2 };
+// OP_ADD_RMS: residual add, then RMSNorm (h = bf16(x + residual) is written
+// back to the residual and normalized).
+enum { OP_PLAIN = 0, OP_RMS = 1, OP_SILU = 2, OP_ADD_RMS = 3 };
 constexpr int kMaxThreads = 512;  // rows up to 8 * 8 * 512 = 32768 elements
 
 struct QuantParams {
@@ -51,11 +53,14 @@ struct QuantParams {
   float eps;
   int64_t M, L, ldx;   // L = row length of y (K, H or I)
   int group;           // 128 or L
-  int ue8m0;
+  int ue8m0;           // 0 fp32 scales, 1 power-of-two fp32, 2 E8M0 bytes
   uint8_t* q;
   int64_t ldq;
   float* s;
   int64_t s_sm, s_sg;
+  uint16_t* res;       // residual (bf16 bits, read and written) for OP_ADD_RMS
+  int64_t ldr;
+  int i8;              // 1: int8 codes, scale amax / 127 (W8A8_INT8)
 };
 
 // ---------------------------------------------------------------------------
@@ -195,9 +200,10 @@ struct QScale {
   float s;
   uint64_t rcp2, neg2;
 };
-__device__ __forceinline__ QScale make_qscale(float amax, int ue8m0) {
+__device__ __forceinline__ QScale make_qscale(float amax, int ue8m0, int i8 = 0) {
   QScale q;
-  q.s = group_scale(amax, ue8m0);
+  // int8 codes: s = fl32(max(amax, 1e-10) / 127), IEEE division
+  q.s = i8 ? __fdiv_rn(fmaxf(amax, 1e-10f), 127.0f) : group_scale(amax, ue8m0);
   q.rcp2 = dup2(__frcp_rn(q.s));
   q.neg2 = dup2(-q.s);
   return q;
@@ -226,6 +232,42 @@ __device__ __forceinline__ uint2 quant_chunk(const uint4& y, const QScale& qs) {
   // (bytes 1 and 3 of each bf16x2 word hold the two signs in their bit 7).
   return make_uint2((c[0] | (c[1] << 16)) | (__byte_perm(w[0], w[1], 0x7531) & 0x80808080u),
                     (c[2] | (c[3] << 16)) | (__byte_perm(w[2], w[3], 0x7531) & 0x80808080u));
+}
+
+// Store the scale of a group: fp32, or (ue8m0 = 2) its E8M0 byte -- the
+// biased exponent of the power-of-two scale, which is a positive normal.
+__device__ __forceinline__ void store_scale(const QuantParams& p, int64_t idx, float s) {
+  if (p.ue8m0 == 2) reinterpret_cast<uint8_t*>(p.s)[idx] = static_cast<uint8_t>(__float_as_uint(s) >> 23);
+  else p.s[idx] = s;
+}
+
+// 8 bf16 values -> 8 int8 codes: the same IEEE quotient fl32(y / s) as
+// quant_chunk, rounded to the nearest integer, ties to even (cvt.rni; |y/s|
+// <= 127 by the choice of s, NaN gives 0).
+__device__ __forceinline__ int32_t f32_to_i32_rni(float v) {
+  int32_t r;
+  asm("cvt.rni.s32.f32 %0, %1;" : "=r"(r) : "f"(v));
+  return r;
+}
+__device__ __forceinline__ uint2 quant_chunk_i8(const uint4& y, const QScale& qs) {
+  const uint32_t w[4] = {y.x, y.y, y.z, y.w};
+  uint32_t c[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint64_t f = bf2_to_f2(w[k]);
+    const uint64_t q0 = mul2(f, qs.rcp2);
+    const uint64_t r = fma2(q0, qs.neg2, f);
+    float a, b;
+    up2(fma2(r, qs.rcp2, q0), a, b);
+    c[k] = __byte_perm(static_cast<uint32_t>(f32_to_i32_rni(a)), static_cast<uint32_t>(f32_to_i32_rni(b)),
+                       0x0040);                          // low bytes of both -> bytes 0, 1
+  }
+  return make_uint2(__byte_perm(c[0], c[1], 0x5410), __byte_perm(c[2], c[3], 0x5410));
+}
+
+// Codes of a chunk in the format of the call.
+__device__ __forceinline__ uint2 codes_chunk(const QuantParams& p, const uint4& y, const QScale& qs) {
+  return p.i8 ? quant_chunk_i8(y, qs) : quant_chunk(y, qs);
 }
 
 // ---------------------------------------------------------------------------
@@ -479,10 +521,30 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
         if ((fix >> i) & 1u) y[i] = silu_chunk_fix(src.ld(off(i)), src.ld(p.L + off(i)), y[i]);
     }
     release();
-  } else {  // OP_RMS
+  } else {  // OP_RMS, OP_ADD_RMS
     uint4 xv[CH];
 #pragma unroll
     for (int i = 0; i < CH; ++i) xv[i] = valid[i] ? src.ld(off(i)) : make_uint4(0, 0, 0, 0);
+    if constexpr (OP == OP_ADD_RMS) {
+      // h = bf16(x + residual): the fp32 sum of two bf16 values is exact
+      // unless their exponents are more than 16 apart, and then it lies far
+      // from every bf16 rounding midpoint, so one RN to bf16 rounds the exact
+      // sum.  h replaces the residual and is what gets normalized.
+      uint16_t* rr = p.res + row * p.ldr;
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        if (valid[i]) {
+          const uint4 r = ld_stream(rr + off(i));
+          uint4 h;
+          h.x = f2_to_bf2_rn(add2(bf2_to_f2(xv[i].x), bf2_to_f2(r.x)));
+          h.y = f2_to_bf2_rn(add2(bf2_to_f2(xv[i].y), bf2_to_f2(r.y)));
+          h.z = f2_to_bf2_rn(add2(bf2_to_f2(xv[i].z), bf2_to_f2(r.z)));
+          h.w = f2_to_bf2_rn(add2(bf2_to_f2(xv[i].w), bf2_to_f2(r.w)));
+          *reinterpret_cast<uint4*>(rr + off(i)) = h;
+          xv[i] = h;
+        }
+      }
+    }
     release();
     // Sum of squares in fp64: squares of bf16 values are exact there (16
     // significant bits, exponents far inside the range).
@@ -530,11 +592,11 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
 #pragma unroll
     for (int i = 0; i < CH; ++i) m2 = chunk_absmax2(y[i], m2);
     const float amax = team_reduce(absmax2_to_f32(m2), MaxOp(), red_f, tid, T, bar_id);
-    const QScale qs = make_qscale(amax, p.ue8m0);
+    const QScale qs = make_qscale(amax, p.ue8m0, p.i8);
 #pragma unroll
     for (int i = 0; i < CH; ++i)
-      if (valid[i]) *reinterpret_cast<uint2*>(qr + off(i)) = quant_chunk(y[i], qs);
-    if (tid == 0) p.s[row * p.s_sm] = qs.s;
+      if (valid[i]) *reinterpret_cast<uint2*>(qr + off(i)) = codes_chunk(p, y[i], qs);
+    if (tid == 0) store_scale(p, row * p.s_sm, qs.s);
   } else {
     // 128-wide groups: the 16 threads tid & ~15 .. +15 own one group per i
     // (T is a multiple of 32 and L of 128, so whole half-warps are valid or not).
@@ -544,9 +606,9 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
       if (valid[i]) {
-        const QScale qs = make_qscale(a, p.ue8m0);
-        *reinterpret_cast<uint2*>(qr + off(i)) = quant_chunk(y[i], qs);
-        if ((tid & 15) == 0) p.s[row * p.s_sm + (off(i) >> 7) * p.s_sg] = qs.s;
+        const QScale qs = make_qscale(a, p.ue8m0, p.i8);
+        *reinterpret_cast<uint2*>(qr + off(i)) = codes_chunk(p, y[i], qs);
+        if ((tid & 15) == 0) store_scale(p, row * p.s_sm + (off(i) >> 7) * p.s_sg, qs.s);
       }
     }
   }
@@ -581,7 +643,7 @@ constexpr int kRingMaxBuf = 16;
 // CTA size cap of the ring kernel (it sets the register budget per thread):
 // SiLU needs more registers than the other ops, 8 chunks per thread more still.
 __host__ __device__ constexpr int ring_max_threads(int op, int ch) {
-  return ch == 8 ? 512 : (op == OP_SILU ? 800 : 1024);
+  return ch == 8 ? 512 : (op == OP_SILU ? 800 : (op == OP_ADD_RMS ? 768 : 1024));
 }
 
 template <int OP, bool PER_TOKEN, int CH>
@@ -655,7 +717,8 @@ inline int threads_for(int64_t nchunks, int ch) {
   return static_cast<int>(t < 32 ? 32 : t);
 }
 
-constexpr int kRingSmemMax = 200 * 1024;   // ring bytes per CTA (one CTA per SM)
+constexpr int kRingSmemMax = 216 * 1024;   // ring bytes per CTA (one CTA per SM; 2 slots of a
+                                           // 25600-wide SiLU row fit)
 
 // Ring geometry: as many teams as fit the CTA size cap (at most 8), and
 // the deepest ring (a multiple of the team count, >= 2 slots per team) that
@@ -732,11 +795,11 @@ fp8q_status check_common(const void* x, int64_t M, int64_t L, int64_t ldx, int64
   if (M < 0 || L <= 0 || L % 16 != 0) return FP8Q_ERR_INVALID_ARG;
   if (ldx < ld_in_min || ldx % 8 != 0 || ldq < L || ldq % 16 != 0) return FP8Q_ERR_INVALID_ARG;
   if (!(group == 128 && L % 128 == 0) && static_cast<int64_t>(group) != L) return FP8Q_ERR_INVALID_ARG;
-  if (ue8m0 != 0 && ue8m0 != 1) return FP8Q_ERR_INVALID_ARG;
+  if (ue8m0 < 0 || ue8m0 > 2) return FP8Q_ERR_INVALID_ARG;
   if (s_sm < 0 || s_sg < 0) return FP8Q_ERR_INVALID_ARG;
   if (M == 0) return FP8Q_OK;  // nothing is read or written: pointers may be null
   if (!x || !q || !s) return FP8Q_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 4)) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, ue8m0 == 2 ? 1 : 4)) return FP8Q_ERR_INVALID_ARG;
   return FP8Q_OK;
 }
 
@@ -781,5 +844,62 @@ extern "C" fp8q_status fp8q_silu_mul_quant(const void* x, int64_t M, int64_t I, 
   if (st != FP8Q_OK) return st;
   QuantParams p{static_cast<const uint16_t*>(x), nullptr, 0.0f, M, I, ldx, group_size, ue8m0,
                 static_cast<uint8_t*>(q), ldq, scales, s_stride_m, s_stride_g};
+  return launch_quant<OP_SILU>(p, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fp8q_status fp8q_add_rmsnorm_quant(const void* x, void* residual, const void* w, float eps,
+                                              int64_t M, int64_t H, int64_t ldx, int64_t ldr,
+                                              int group_size, int ue8m0, void* q, int64_t ldq,
+                                              float* scales, int64_t s_stride_m, int64_t s_stride_g,
+                                              void* stream) {
+  fp8q_status st = check_common(x, M, H, ldx, H, group_size, ue8m0, q, ldq, scales, s_stride_m,
+                                s_stride_g);
+  if (st != FP8Q_OK) return st;
+  if (!(eps >= 0.0f) || eps > 3.0e38f) return FP8Q_ERR_INVALID_ARG;
+  if (ldr < H || ldr % 8 != 0) return FP8Q_ERR_INVALID_ARG;
+  if (M > 0 && (!w || !aligned(w, 16) || !residual || !aligned(residual, 16))) return FP8Q_ERR_INVALID_ARG;
+  QuantParams p{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w), eps, M, H, ldx,
+                group_size, ue8m0, static_cast<uint8_t*>(q), ldq, scales, s_stride_m, s_stride_g,
+                static_cast<uint16_t*>(residual), ldr};
+  return launch_quant<OP_ADD_RMS>(p, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------- W8A8_INT8
+// The same three producers with int8 codes (scale amax / 127).
+extern "C" fp8q_status fp8q_group_quant_i8(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                           int group_size, void* q, int64_t ldq, float* scales,
+                                           int64_t s_stride_m, int64_t s_stride_g, void* stream) {
+  fp8q_status st = check_common(x, M, K, ldx, K, group_size, 0, q, ldq, scales, s_stride_m,
+                                s_stride_g);
+  if (st != FP8Q_OK) return st;
+  QuantParams p{static_cast<const uint16_t*>(x), nullptr, 0.0f, M, K, ldx, group_size, 0,
+                static_cast<uint8_t*>(q), ldq, scales, s_stride_m, s_stride_g, nullptr, 0, 1};
+  return launch_quant<OP_PLAIN>(p, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fp8q_status fp8q_rmsnorm_quant_i8(const void* x, const void* w, float eps, int64_t M,
+                                             int64_t H, int64_t ldx, int group_size, void* q,
+                                             int64_t ldq, float* scales, int64_t s_stride_m,
+                                             int64_t s_stride_g, void* stream) {
+  fp8q_status st = check_common(x, M, H, ldx, H, group_size, 0, q, ldq, scales, s_stride_m,
+                                s_stride_g);
+  if (st != FP8Q_OK) return st;
+  if (!(eps >= 0.0f) || eps > 3.0e38f) return FP8Q_ERR_INVALID_ARG;
+  if (M > 0 && (!w || !aligned(w, 16))) return FP8Q_ERR_INVALID_ARG;
+  QuantParams p{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w), eps, M, H, ldx,
+                group_size, 0, static_cast<uint8_t*>(q), ldq, scales, s_stride_m, s_stride_g, nullptr,
+                0, 1};
+  return launch_quant<OP_RMS>(p, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fp8q_status fp8q_silu_mul_quant_i8(const void* x, int64_t M, int64_t I, int64_t ldx,
+                                              int group_size, void* q, int64_t ldq, float* scales,
+                                              int64_t s_stride_m, int64_t s_stride_g, void* stream) {
+  if (I > (INT64_MAX / 4)) return FP8Q_ERR_INVALID_ARG;
+  fp8q_status st = check_common(x, M, I, ldx, 2 * I, group_size, 0, q, ldq, scales, s_stride_m,
+                                s_stride_g);
+  if (st != FP8Q_OK) return st;
+  QuantParams p{static_cast<const uint16_t*>(x), nullptr, 0.0f, M, I, ldx, group_size, 0,
+                static_cast<uint8_t*>(q), ldq, scales, s_stride_m, s_stride_g, nullptr, 0, 1};
   return launch_quant<OP_SILU>(p, static_cast<cudaStream_t>(stream));
 }

@@ -51,7 +51,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait until the phase of `bar` with the given parity has completed.  Gives
 // up (returns false) when *abort is set by another role, or after
 // kWaitLimitNs, in which case it sets *abort and records FP8Q_ERR_TIMEOUT.
+// A test-only build of the library (never the shipped one) may shorten the
+// limit with -DFP8Q_TEST_WAIT_LIMIT_NS=<ns>.
+#ifdef FP8Q_TEST_WAIT_LIMIT_NS
+constexpr uint64_t kWaitLimitNs = FP8Q_TEST_WAIT_LIMIT_NS;
+#else
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+#endif
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* status) {
@@ -271,6 +277,45 @@ __device__ __forceinline__ void tmem_ld_waited(uint32_t taddr, uint32_t* r) {
   }
 }
 
+// A 32x32b TMEM load of N columns without its wait (the registers are not
+// valid until tmem_wait_regs on the same array), and that wait: it names the
+// registers as in/out operands, so no use of them can be scheduled before it,
+// while other work (e.g. the arithmetic on an earlier chunk) can overlap the
+// load in flight.
+template <int N>
+__device__ __forceinline__ void tmem_ld_async(uint32_t taddr, uint32_t* r) {
+  static_assert(N == 8 || N == 16, "tcgen05.ld width");
+  if constexpr (N == 8) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
+        : "r"(taddr));
+  } else {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {"
+        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+  }
+}
+template <int N>
+__device__ __forceinline__ void tmem_wait_regs(uint32_t* r) {
+  static_assert(N == 8 || N == 16, "tcgen05.ld width");
+  if constexpr (N == 8) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]));
+  } else {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+  }
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -323,6 +368,85 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask) {
           smem_u32(bar)),
       "h"(mask)
       : "memory");
+}
+
+// ------------------------------------------------------------ block scaling
+// tcgen05.mma kind::mxf8f6f4.block_scale: the tensor core multiplies every
+// 32-deep K slice of A row r by the E8M0 scale SFA[r] and of B column c by
+// SFB[c] itself, so block-scaled products accumulate in TMEM with no register
+// promotion.  Scale factors live in TMEM: the scale of MMA row (or column) r
+// is in lane r % 32 of every lane quadrant, column (base + r / 32), and byte k
+// of that 32-bit column belongs to the k-th 32-deep K slice of a 128-deep
+// stage; the MMA picks the byte with the "scale factor id" (address bits
+// 30-31 and the instruction descriptor's id fields).
+
+// Make generic-proxy writes to shared memory visible to the async proxy
+// (tcgen05.cp, TMA) before they are signalled.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// One 512-byte scale-factor chunk -- 32 rows of 16 bytes in shared memory,
+// row l holding the scales of MMA rows l, l+32, l+64, l+96 (4 bytes each) --
+// into TMEM columns [taddr, taddr + 4) of all four lane quadrants
+// (tcgen05.cp 32x128b.warpx4).  Source descriptor: K-major, no swizzle, the
+// four 8-row core matrices 128 bytes apart (stride byte offset), version 1.
+__device__ __forceinline__ void tmem_cp_sf_chunk(uint32_t taddr, const void* src) {
+  const uint64_t desc = (static_cast<uint64_t>(smem_u32(src) & 0x3FFFF) >> 4) |
+                        (static_cast<uint64_t>(128 >> 4) << 32) | (1ull << 46);
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+               : "memory");
+}
+
+// D[tmem] (+)= (A * SFA) * (B * SFB)^T, e4m3 x e4m3 -> f32, E8M0 scale
+// factors at TMEM addresses sfa / sfb (byte id in bits 30-31), one CTA.
+__device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate, uint32_t sfa,
+                                             uint32_t sfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Instruction descriptor, kind::mxf8f6f4 with block scaling: A and B e4m3
+// (bits 7-9, 10-12 = 0), K-major, N >> 3 at bits 17-22, scale format E8M0
+// (bit 23), M >> 4 at bits 24-28, scale factor ids of B (bits 4-5) and A
+// (bits 29-30) = the K slice k.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, int k) {
+  return (static_cast<uint32_t>(k) << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(k) << 29);
+}
+
+// kind::i8 (W8A8_INT8): D[tmem] (+)= A * B^T with signed 8-bit operands and
+// exact s32 accumulation, one CTA or a CTA pair.
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor, kind::i8: D s32 (bits 4-5 = 2), A and B signed int8
+// (bits 7-9 and 10-12 = 1), K-major, N >> 3 at bits 17-22, M >> 4 at 24-28.
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {

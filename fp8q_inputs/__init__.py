@@ -91,3 +91,9 @@ def random_scales(seed: int, shape, lo: float = 1e-3, hi: float = 1e-1) -> np.nd
 def random_pow2_scales(seed: int, shape, lo_exp: int = -12, hi_exp: int = -2) -> np.ndarray:
     g = rng(seed)
     return np.ldexp(1.0, g.integers(lo_exp, hi_exp + 1, size=shape)).astype(np.float32)
+
+
+def random_e4m3_codes_u8(seed: int, shape) -> np.ndarray:
+    """Uniform random positive finite e4m3fn bytes 0..125, drawn directly as
+    uint8 (for large weight stand-ins where only the shape matters)."""
+    return rng(seed).integers(0, 126, size=shape, dtype=np.uint8)

@@ -10,7 +10,9 @@
  *
  *   scale      s = fl32(max(amax, 1e-10) / 448), amax = max |y| over the group
  *   UE8M0      (ue8m0 = 1) s is rounded up to the next power of two (a power of
- *              two is kept); the scale is still stored as fp32
+ *              two is kept); the scale is still stored as fp32.  (ue8m0 = 2)
+ *              the same power-of-two scale stored packed as one E8M0 byte:
+ *              its biased exponent b, s = 2^(b - 127)
  *   codes      q = e4m3fn(fl32(y / s)), IEEE fp32 division, round to nearest
  *              even, saturating to +-448; the sign of zero is kept
  *   groups     contiguous 1x128 chunks of a row (group_size = 128), or the
@@ -46,8 +48,8 @@
  *     second) stops, records FP8Q_ERR_TIMEOUT in a device status word and
  *     returns; read it with fp8q_last_device_status.  No C++ exception
  *     crosses this interface.
- *   - Pointers to bf16 / code tensors must be 16-byte aligned; scale pointers
- *     4-byte aligned.  With M = 0 a call validates its sizes and returns
+ *   - Pointers to bf16 / code tensors must be 16-byte aligned; fp32 scale
+ *     pointers 4-byte aligned (E8M0 byte arrays need no alignment).  With M = 0 a call validates its sizes and returns
  *     FP8Q_OK without touching memory; its pointers may then be NULL.
  */
 #ifndef FP8Q_H
@@ -87,9 +89,13 @@ typedef enum {
  *   x        bf16 [M, K], leading dimension ldx (>= K, multiple of 8)
  *   M, K     M >= 0 (M = 0 is a no-op), K > 0 and a multiple of 16
  *   group_size  128 (K must then be a multiple of 128) or K
- *   ue8m0    0 or 1 (round scales up to powers of two)
+ *   ue8m0    0: fp32 scales; 1: scales rounded up to powers of two, fp32;
+ *            2: the same power-of-two scales as packed E8M0 bytes -- `scales`
+ *            then points to uint8 storage (any alignment) and the strides
+ *            count bytes (the layout fp8q_scaled_mm_blockwise_e8m0 reads)
  *   q        e4m3 codes [M, K], leading dimension ldq (>= K, multiple of 16)
- *   scales   fp32, scale of group g of row m at scales[m*s_stride_m + g*s_stride_g]
+ *   scales   fp32 (or E8M0 bytes), scale of group g of row m at
+ *            scales[m*s_stride_m + g*s_stride_g]
  *            (row-major [M, K/group]: s_stride_m = K/group, s_stride_g = 1;
  *            group-major [K/group, M]: s_stride_m = 1, s_stride_g = M)
  */
@@ -113,6 +119,25 @@ FP8Q_API fp8q_status fp8q_rmsnorm_quant(const void* x, const void* w, float eps,
                                void* stream);
 
 /*
+ * fp8q_add_rmsnorm_quant -- residual add fused into the RMSNorm quant, the
+ * fusion "on either side of the path" that continues the pages' cut of the
+ * call count by fused ops ("Helion in vLLM", "Kernels integrated into vLLM").
+ *   h = bf16(x + residual)   (one rounding of the exact sum)
+ *   residual <- h            (the residual stream is updated in place)
+ *   q, scales = rmsnorm_quant(h)  exactly as fp8q_rmsnorm_quant
+ * This is what the unfused chain (bf16 add, then fp8q_rmsnorm_quant) gives.
+ *
+ *   x [M, H] bf16 (ldx), residual [M, H] bf16 (ldr >= H, multiple of 8,
+ *   16-byte aligned; read and written; must not overlap x, w, q or scales);
+ *   other arguments as in fp8q_rmsnorm_quant.
+ */
+FP8Q_API fp8q_status fp8q_add_rmsnorm_quant(const void* x, void* residual, const void* w, float eps,
+                                            int64_t M, int64_t H, int64_t ldx, int64_t ldr,
+                                            int group_size, int ue8m0, void* q, int64_t ldq,
+                                            float* scales, int64_t s_stride_m, int64_t s_stride_g,
+                                            void* stream);
+
+/*
  * fp8q_silu_mul_quant -- silu_and_mul_dynamic_per_token_quant (group_size = I)
  * and silu_and_mul_per_block_quant (group_size = 128) ("Helion in vLLM",
  * "Kernels integrated into vLLM", items 3 and 7).
@@ -125,6 +150,38 @@ FP8Q_API fp8q_status fp8q_rmsnorm_quant(const void* x, const void* w, float eps,
 FP8Q_API fp8q_status fp8q_silu_mul_quant(const void* x, int64_t M, int64_t I, int64_t ldx, int group_size,
                                 int ue8m0, void* q, int64_t ldq, float* scales,
                                 int64_t s_stride_m, int64_t s_stride_g, void* stream);
+
+/*
+ * fp8q_qk_norm_rope -- fused_qk_norm_rope ("Helion in vLLM" (24-ai.news),
+ * "Kernels integrated into vLLM", item 4; its arguments as the vllm PR #44010
+ * page lists them, section "Code analysis"), in place on the packed qkv
+ * output of the qkv projection.  The pages print no arithmetic; this library
+ * applies, to every q and k head of every token,
+ *   the RMSNorm of this header:  r = 1/sqrt(mean(x^2) + eps),
+ *                                y = bf16(bf16(x r) w)   (w = q or k weight)
+ *   then the rotary embedding at p = positions[t], cos = cache[p][i],
+ *   sin = cache[p][D/2 + i], on pairs (i, i + D/2) (is_neox = 1) or
+ *   (2i, 2i + 1) (is_neox = 0):
+ *                                a' = bf16(a cos - b sin), b' = bf16(b cos + a sin)
+ * v heads are not touched.  Arithmetic is fp32 (the norm's reciprocal root to
+ * about one fp32 ulp); results are the bf16 rounding of the definition
+ * except where an fp32 result lies within a few fp32 ulps of a bf16 rounding
+ * midpoint (then the neighbouring bf16 value).
+ *
+ *   qkv        bf16 [T, ld], row t = [q (hq heads) | k (hk) | v (hv)], head_dim D
+ *              each; ld >= (hq + hk + hv) D, multiple of 8; 16-byte aligned
+ *   head_dim   64, 128 or 256 (else FP8Q_ERR_UNSUPPORTED)
+ *   q_weight, k_weight  bf16 [D]
+ *   cos_sin_cache  fp32 [max_position, D]: D/2 cosines then D/2 sines per row
+ *   positions  int64 [T], each in [0, max_position); a position outside it
+ *              is not read: the token uses row 0 and the device status word
+ *              records FP8Q_ERR_INVALID_ARG (see fp8q_last_device_status)
+ */
+FP8Q_API fp8q_status fp8q_qk_norm_rope(void* qkv, int64_t T, int64_t ld, int num_heads_q,
+                                       int num_heads_k, int num_heads_v, int head_dim, float eps,
+                                       const void* q_weight, const void* k_weight,
+                                       const float* cos_sin_cache, int64_t max_position,
+                                       const int64_t* positions, int is_neox, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Scaled FP8 GEMMs                                                          */
@@ -178,6 +235,36 @@ FP8Q_API fp8q_status fp8q_scaled_mm_blockwise(const void* a_q, const void* b_q, 
                                      void* stream);
 
 /*
+ * fp8q_scaled_mm_blockwise_e8m0 -- scaled_mm_blockwise with power-of-two
+ * block scales stored as E8M0 bytes, the form the pages say DeepGEMM needs
+ * on B200 ("Helion in vLLM" (24-ai.news), section "Practical limits"; E8M0
+ * block scales on SM100 in the MXFP4 CUTLASS MoE page, vllm PR #37463).
+ *   y[m, n] = bf16_rn( sum_kb 2^(ea[m,kb]-127) 2^(eb[n/128,kb]-127) P_kb[m, n] )
+ * The tensor core applies the scales itself (tcgen05.mma
+ * kind::mxf8f6f4.block_scale, each 1x128 / 128x128 scale repeated over its
+ * four 32-deep K slices), so the fp32 accumulator stays in TMEM for the whole
+ * K range; the result equals fp8q_scaled_mm_blockwise on the decoded scales
+ * up to fp32 summation order.
+ *
+ *   a_sf     uint8 E8M0, one byte per 1x128 group of A: ea[m, kb] at
+ *            a_sf[m*as_stride_m + kb*as_stride_kb] (what fp8q_group_quant and
+ *            the fused quant ops write with ue8m0 = 2); the offset rule of
+ *            fp8q_scaled_mm_blockwise applies
+ *   b_sf     uint8 E8M0 [N/128, K/128] row-major, one byte per 128x128 block
+ *   A byte of 255 (E8M0 NaN) makes the affected outputs NaN.  N and K
+ *   multiples of 128; other arguments as in fp8q_scaled_mm_blockwise, with
+ *   fp8q_workspace_bytes(M, N, K, 2).  Variants: Swap-AB tiles (block_n
+ *   16..128), or 128-row tiles of block_n 128 or 224 (224 leaves TMEM room
+ *   for the scale factors next to two accumulator buffers); no CTA pairs.
+ */
+FP8Q_API fp8q_status fp8q_scaled_mm_blockwise_e8m0(const void* a_q, const void* b_q,
+                                                   const uint8_t* a_sf, int64_t as_stride_m,
+                                                   int64_t as_stride_kb, const uint8_t* b_sf,
+                                                   int64_t M, int64_t N, int64_t K, void* y,
+                                                   int64_t ldy, void* workspace, size_t ws_bytes,
+                                                   void* stream);
+
+/*
  * fp8q_scaled_mm_blockwise_noalloc -- the same GEMM as
  * fp8q_scaled_mm_blockwise, for callers that cannot hand the library any
  * device memory beyond their inputs and outputs.  (The pages have no
@@ -212,8 +299,43 @@ FP8Q_API fp8q_status fp8q_scaled_mm_blockwise_noalloc(const void* a_q, const voi
                                                       int64_t M, int64_t N, int64_t K, void* y,
                                                       int64_t ldy, void* stream);
 
-/* Bytes of scratch the GEMM of this shape needs (0 if none); blockwise = 0/1.
- * Depends only on the shape and the variant the library picks for it. */
+/* ------------------------------------------------------------------------ */
+/* W8A8_INT8                                                                 */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The W8A8_INT8 scheme ("Helion linear backend" (aihirek.info), section
+ * "Autotuning selects the variant": FP8_Dynamic, W8A8_INT8 and Block_FP8).
+ * The pages name the scheme only; this library reads it as the FP8 path with
+ * signed 8-bit integer codes:
+ *   scale  s = fl32(max(amax, 1e-10) / 127)   (IEEE fp32 division)
+ *   codes  q = int8(round-half-even(fl32(y / s))), saturated to [-128, 127]
+ *   GEMM   y[m, n] = bf16_rn( sa(m) sb(n) sum_k qa[m,k] qb[n,k] ), the sum
+ *          exact in 32-bit integers (tcgen05 kind::i8), converted to fp32
+ * The quant entry points take the arguments of their FP8 counterparts (no
+ * ue8m0); q holds int8 codes.  fp8q_scaled_mm_i8 takes those of
+ * fp8q_scaled_mm (int8 operands; K <= 133152 keeps every integer sum in
+ * range) with fp8q_workspace_bytes(M, N, K, 3).
+ */
+FP8Q_API fp8q_status fp8q_group_quant_i8(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                         int group_size, void* q, int64_t ldq, float* scales,
+                                         int64_t s_stride_m, int64_t s_stride_g, void* stream);
+FP8Q_API fp8q_status fp8q_rmsnorm_quant_i8(const void* x, const void* w, float eps, int64_t M,
+                                           int64_t H, int64_t ldx, int group_size, void* q,
+                                           int64_t ldq, float* scales, int64_t s_stride_m,
+                                           int64_t s_stride_g, void* stream);
+FP8Q_API fp8q_status fp8q_silu_mul_quant_i8(const void* x, int64_t M, int64_t I, int64_t ldx,
+                                            int group_size, void* q, int64_t ldq, float* scales,
+                                            int64_t s_stride_m, int64_t s_stride_g, void* stream);
+FP8Q_API fp8q_status fp8q_scaled_mm_i8(const void* a_q, const void* b_q, const float* a_scale,
+                                       int a_per_token, const float* b_scale, int b_per_channel,
+                                       int64_t M, int64_t N, int64_t K, void* y, int64_t ldy,
+                                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of scratch the GEMM of this shape needs (0 if none); blockwise = 0
+ * (fp8q_scaled_mm), 1 (fp8q_scaled_mm_blockwise), 2
+ * (fp8q_scaled_mm_blockwise_e8m0), 3 (fp8q_scaled_mm_i8).  Depends only on the shape and the variant
+ * the library picks for it. */
 FP8Q_API size_t fp8q_workspace_bytes(int64_t M, int64_t N, int64_t K, int blockwise);
 
 /* ------------------------------------------------------------------------ */
@@ -230,7 +352,7 @@ FP8Q_API size_t fp8q_workspace_bytes(int64_t M, int64_t N, int64_t K, int blockw
  * cta_pair = 1 runs each 256-row tile on a cluster of two CTAs (two SMs)
  * sharing one tcgen05 .cta_group::2 MMA, each SM staging half of the B tile
  * (only with swap_ab = 0 and split_k = 1; block_n 128, or 256 for the
- * per-token scheme). */
+ * per-token scheme).  block_n 224 is the E8M0 GEMM's wide tile (no swap). */
 typedef struct {
     int swap_ab;
     int split_k;
@@ -250,8 +372,9 @@ FP8Q_API fp8q_status fp8q_select_gemm_variant(int64_t M, int64_t N, int64_t K, i
 /* Force a variant for every following GEMM call in this process (testing and
  * tuning only; not thread-safe).  NULL restores automatic selection.  Returns
  * FP8Q_ERR_INVALID_ARG if the variant is malformed (block_n not one of
- * 16, 32, 64, 128, 256; split_k < 0 or > 64; cta_pair not 0 or 1, or set
- * with another combination than the one above). */
+ * 16, 32, 64, 128, 224, 256; split_k < 0 or > 64; cta_pair not 0 or 1, or
+ * set with another combination than the one above).  A GEMM call whose
+ * scheme cannot run the forced variant returns FP8Q_ERR_UNSUPPORTED. */
 FP8Q_API fp8q_status fp8q_force_gemm_variant(const fp8q_gemm_variant* v);
 
 /* ------------------------------------------------------------------------ */
@@ -259,8 +382,10 @@ FP8Q_API fp8q_status fp8q_force_gemm_variant(const fp8q_gemm_variant* v);
 /* ------------------------------------------------------------------------ */
 
 /* Synchronizes `stream`, then returns and clears the device status word of
- * the current device (FP8Q_OK, or FP8Q_ERR_TIMEOUT if a kernel gave up on a
- * wait since the last read).  FP8Q_ERR_CUDA if the synchronization failed. */
+ * the current device (FP8Q_OK; FP8Q_ERR_TIMEOUT if a kernel gave up on a
+ * wait since the last read; FP8Q_ERR_INVALID_ARG if fp8q_qk_norm_rope met a
+ * position outside its cache; the first error recorded wins).  FP8Q_ERR_CUDA
+ * if the synchronization failed. */
 FP8Q_API fp8q_status fp8q_last_device_status(void* stream);
 
 /* Static description of a status code (never NULL). */

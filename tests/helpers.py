@@ -77,6 +77,27 @@ def sample_rows(M: int, n: int, seed: int) -> np.ndarray:
     return np.array(sorted(rows), dtype=np.int64)
 
 
+def config_rows(M: int, seed: int, n: int = 256, tile: int = 256) -> np.ndarray:
+    """Rows for a config-size GEMM check (every column of each is compared):
+    n seeded rows spread over every `tile`-row tile, half of each tile's share
+    from its first 128 rows and half from its last 128 (the two CTAs of a
+    256-row CTA-pair tile), plus every row of the last tile and the first and
+    last rows.  M <= n: every row."""
+    if M <= n:
+        return np.arange(M, dtype=np.int64)
+    g = np.random.default_rng(seed)
+    ntiles = -(-M // tile)
+    per = max(2, n // ntiles)
+    rows = {0, M - 1}
+    for t in range(ntiles):
+        for lo, hi in ((t * tile, t * tile + tile // 2), (t * tile + tile // 2, (t + 1) * tile)):
+            lo, hi = min(lo, M), min(hi, M)
+            if hi > lo:
+                rows |= set(g.choice(np.arange(lo, hi), size=min(per // 2, hi - lo), replace=False).tolist())
+    rows |= set(range((ntiles - 1) * tile, M))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
 def quantized_weights(seed: int, N: int, K: int, blockwise: bool):
     """Seeded W ~ N(0, 0.02) quantized by the ORACLE: per output channel
     (codes, s[N]) or in 128x128 blocks (codes, s[N/128, K/128])."""

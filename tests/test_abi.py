@@ -14,7 +14,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def test_library_exports_every_declared_function():
     names = fq.header_functions()
-    assert len(names) == 12
+    assert len(names) == 19
     for n in names:
         assert hasattr(fq.lib, n), n
         assert callable(getattr(fq, n)), f"binding lacks {n}"
@@ -56,6 +56,40 @@ def test_invalid_arguments_rejected_before_launch():
                                       0, None) == fq.ERR_INVALID_ARG
     assert L.fp8q_scaled_mm_blockwise_noalloc(fake, fake, fake, 1, 1 << 29, fake, 4, 128, 256, fake,
                                               128, None) == fq.ERR_INVALID_ARG
+    # E8M0 GEMM: N or K not a multiple of 128, null scale bytes, misaligned y
+    e8 = L.fp8q_scaled_mm_blockwise_e8m0
+    assert e8(fake, fake, fake, 2, 1, fake, 4, 192, 256, fake, 192, None, 0, None) == fq.ERR_INVALID_ARG
+    assert e8(fake, fake, fake, 2, 1, fake, 4, 128, 200, fake, 128, None, 0, None) == fq.ERR_INVALID_ARG
+    assert e8(fake, fake, None, 2, 1, fake, 4, 128, 256, fake, 128, None, 0, None) == fq.ERR_INVALID_ARG
+    assert e8(fake, fake, fake, 2, 1, fake, 4, 128, 256, fake + 8, 128, None, 0, None) == fq.ERR_INVALID_ARG
+    # residual add: residual leading dimension below H, null residual
+    ar = L.fp8q_add_rmsnorm_quant
+    assert ar(fake, fake, fake, ctypes.c_float(1e-6), 4, 256, 256, 128, 128, 0, fake, 256, fake, 2, 1,
+              None) == fq.ERR_INVALID_ARG
+    assert ar(fake, None, fake, ctypes.c_float(1e-6), 4, 256, 256, 256, 128, 0, fake, 256, fake, 2, 1,
+              None) == fq.ERR_INVALID_ARG
+    assert ar(None, None, None, ctypes.c_float(1e-6), 0, 256, 256, 256, 128, 0, None, 256, None, 2, 1,
+              None) == fq.OK
+    # qk norm + rope: unsupported head size, ld too small, bad is_neox, zero tokens
+    qr = L.fp8q_qk_norm_rope
+    assert qr(fake, 4, 1280, 8, 1, 1, 96, ctypes.c_float(1e-6), fake, fake, fake, 16, fake, 1,
+              None) == fq.ERR_UNSUPPORTED
+    assert qr(fake, 4, 1000, 8, 1, 1, 128, ctypes.c_float(1e-6), fake, fake, fake, 16, fake, 1,
+              None) == fq.ERR_INVALID_ARG
+    assert qr(fake, 4, 1280, 8, 1, 1, 128, ctypes.c_float(1e-6), fake, fake, fake, 16, fake, 2,
+              None) == fq.ERR_INVALID_ARG
+    assert qr(None, 0, 1280, 8, 1, 1, 128, ctypes.c_float(1e-6), None, None, None, 16, None, 1,
+              None) == fq.OK
+    # int8: K beyond the exact-sum range, group size, null scales
+    assert L.fp8q_scaled_mm_i8(fake, fake, fake, 1, fake, 1, 4, 128, 133152 + 16, fake, 128, None, 0,
+                               None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_group_quant_i8(fake, 4, 256, 256, 64, fake, 256, fake, 2, 1, None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_rmsnorm_quant_i8(fake, fake, ctypes.c_float(1e-6), 4, 256, 256, 128, fake, 256, None,
+                                   2, 1, None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_silu_mul_quant_i8(fake, 4, 256, 256, 128, fake, 256, fake, 2, 1, None) == fq.ERR_INVALID_ARG
+    # packed E8M0 quant scales need no alignment; ue8m0 beyond 2 is rejected
+    assert L.fp8q_group_quant(fake, 4, 256, 256, 128, 3, fake, 256, fake + 1, 2, 1, None) == fq.ERR_INVALID_ARG
+    assert L.fp8q_group_quant(fake, 4, 256, 256, 128, 1, fake, 256, fake + 1, 2, 1, None) == fq.ERR_INVALID_ARG
 
 
 def test_zero_rows_is_a_noop_without_pointers():
@@ -64,6 +98,8 @@ def test_zero_rows_is_a_noop_without_pointers():
     assert L.fp8q_scaled_mm(None, None, None, 1, None, 1, 0, 256, 256, None, 256, None, 0, None) == fq.OK
     assert L.fp8q_scaled_mm_blockwise(None, None, None, 2, 1, None, 0, 256, 256, None, 256, None, 0,
                                       None) == fq.OK
+    assert L.fp8q_scaled_mm_blockwise_e8m0(None, None, None, 2, 1, None, 0, 256, 256, None, 256, None,
+                                           0, None) == fq.OK
 
 
 def _variant_table():
@@ -133,3 +169,24 @@ def test_variant_selection_host_logic():
     fq.fp8q_force_gemm_variant()
     with pytest.raises(fq.Fp8qError):
         fq.fp8q_force_gemm_variant(0, 1, 48)
+
+
+def test_e8m0_variant_selection_host_logic():
+    # The E8M0 GEMM follows the per-token scheme's choice, single CTAs only,
+    # 224-column tiles where that scheme takes 256-column ones.
+    for M, N, K in [(8192, 51200, 5120), (2048, 24576, 4096), (4096, 6144, 4096)]:
+        v = fq.fp8q_select_gemm_variant(M, N, K, 2)
+        assert v["cta_pair"] == 0 and v["swap_ab"] == 0 and v["block_n"] in (128, 224), v
+    for M in (1, 16, 32, 64):
+        v = fq.fp8q_select_gemm_variant(M, 10240, 5120, 2)
+        pt = fq.fp8q_select_gemm_variant(M, 10240, 5120, False)
+        assert v == pt, (M, v, pt)
+    assert fq.fp8q_workspace_bytes(8192, 51200, 5120, 2) == 0
+    assert fq.fp8q_workspace_bytes(8192, 51200, 5120, 3) == 0
+    # forcing: 224 is accepted (the E8M0 tile), an unsupported combination for
+    # the scheme is reported by the GEMM call itself
+    fq.fp8q_force_gemm_variant(0, 3, 224)
+    assert fq.fp8q_select_gemm_variant(4096, 6144, 4096, 2) == \
+        {"swap_ab": 0, "split_k": 3, "block_n": 224, "cta_pair": 0}
+    assert fq.fp8q_workspace_bytes(4096, 6144, 4096, 2) > 0
+    fq.fp8q_force_gemm_variant()

@@ -40,13 +40,13 @@ def test_reference_line_has_the_driver_keys(reference_line):
                         "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
-    assert "2 of 2048 tokens" in cb["sample"]
+    assert f"2 of 8192 tokens" in cb["sample"]
 
 
 def test_reference_arm_times_the_gpu_arms_workload(reference_line):
     sys.path.insert(0, ROOT)
     import bench
-    assert reference_line["config"] == bench.workload_config(2048, 1)
+    assert reference_line["config"] == bench.workload_config(bench.DEFAULT_M, 1)
     assert reference_line["metric"] == bench.METRIC
 
 

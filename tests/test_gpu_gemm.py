@@ -5,8 +5,9 @@ with y_ref the fp64 sum of the dequantized operands.  Every GEMM variant
 (tile width, Swap-AB, Split-K) is forced in turn on shapes that span several
 tiles and ragged M / N / K tails and checked in full; the config shapes
 (Qwen3-8B / 32B linears, decode and prefill M) run through the automatic
-variant choice and are checked on sampled rows (every row of the last partial
-tile included).
+variant choice and are checked on every column of 256 stratified rows (every
+256-row tile and both of its 128-row halves) plus every row of the last
+256-row tile; decode batches (M <= 256) in full.
 """
 import numpy as np
 import pytest
@@ -14,7 +15,7 @@ import torch
 
 import fp8q_inputs as inp
 import oracle
-from helpers import (bf16_to_np, gemm_tolerance_check, quantized_weights, sample_rows,
+from helpers import (bf16_to_np, config_rows, gemm_tolerance_check, quantized_weights,
                      to_dev_bf16, to_dev_codes)
 
 pytestmark = pytest.mark.gpu
@@ -226,14 +227,16 @@ def test_abi_rejects_bad_arguments():
     # quant: bad group size, bad ue8m0
     x = torch.zeros((4, 256), dtype=torch.bfloat16, device="cuda")
     assert L.fp8q_group_quant(p(x), 4, 256, 256, 64, 0, p(a), 256, p(s), 1, 1, st) == fq.ERR_INVALID_ARG
-    assert L.fp8q_group_quant(p(x), 4, 256, 256, 128, 2, p(a), 256, p(s), 2, 1, st) == fq.ERR_INVALID_ARG
+    assert L.fp8q_group_quant(p(x), 4, 256, 256, 128, 3, p(a), 256, p(s), 2, 1, st) == fq.ERR_INVALID_ARG
     torch.cuda.synchronize()
 
 
 # ------------------------------------------------------------ config shapes
-def _check_config_gemm(M, N, K, blockwise, seed, nrows=12, act="normal"):
+def _check_config_gemm(M, N, K, blockwise, seed, act="normal"):
     """Activations quantized by the oracle (1x128 groups or per token), weights
-    W ~ N(0, 0.02) quantized by the oracle (128x128 blocks or per channel)."""
+    W ~ N(0, 0.02) quantized by the oracle (128x128 blocks or per channel).
+    Checked: every column of 256 stratified rows (every 256-row tile, both
+    128-row halves) and of every row of the last 256-row tile."""
     if act == "heavy":
         x = inp.heavy_tailed_bf16(seed, M, K)
     else:
@@ -245,7 +248,7 @@ def _check_config_gemm(M, N, K, blockwise, seed, nrows=12, act="normal"):
         a, sa = oracle.group_quant(x, K)
         sa = sa.reshape(-1)
         sb = sb.reshape(-1)
-    rows = sample_rows(M, nrows, seed + 2)
+    rows = config_rows(M, seed + 2)
     if blockwise:
         y = _run_bw(a, b, sa, sb, M, N, K)
         y_ref, ad = oracle.scaled_mm_blockwise(a, b, sa, sb, rows)
@@ -283,21 +286,21 @@ def test_config_qwen3_8b_per_token_mlp(M, layer):
 @pytest.mark.parametrize("layer", ["qkv", "o", "gate_up", "down"])
 def test_config_qwen3_8b_blockwise(M, layer):
     K, N = QWEN8[layer]
-    _check_config_gemm(M, N, K, True, 800 + M, nrows=8)
+    _check_config_gemm(M, N, K, True, 800 + M)
 
 
 @pytest.mark.parametrize("M", [1, 2, 4, 8, 16, 32, 64])
 @pytest.mark.parametrize("layer", ["qkv", "o", "gate_up", "down"])
 def test_config_qwen3_32b_decode_blockwise(M, layer):
     K, N = QWEN32[layer]
-    _check_config_gemm(M, N, K, True, 900 + M, nrows=6)
+    _check_config_gemm(M, N, K, True, 900 + M)
 
 
 @pytest.mark.parametrize("blockwise", [False, True])
 @pytest.mark.parametrize("layer", ["qkv", "o", "gate_up", "down"])
 def test_config_qwen3_32b_prefill(layer, blockwise):
     K, N = QWEN32[layer]
-    _check_config_gemm(8192, N, K, blockwise, 1000, nrows=4, act="heavy")
+    _check_config_gemm(8192, N, K, blockwise, 1000, act="heavy")
 
 
 def test_config_tiny_per_token_linear_chain():

@@ -186,3 +186,44 @@ def test_group_scale_for_every_bf16_amax(ue8m0):
     torch.cuda.synchronize()
     np.testing.assert_array_equal(s.cpu().numpy(), s_ref)
     np.testing.assert_array_equal(codes_np(q), q_ref)
+
+
+@pytest.mark.parametrize("ue8m0", [False, True, "packed"])
+@pytest.mark.parametrize("per_token", [False, True])
+@pytest.mark.parametrize("M,H", [(16, 2048), (33, 4096), (129, 5120), (3, 20480)])
+def test_add_rmsnorm_quant(M, H, per_token, ue8m0):
+    # residual add + RMSNorm quant: the updated residual is bit-exact (one
+    # bf16 rounding of the sum), codes and scales meet the fused tolerance;
+    # H = 20480 takes the shared-memory ring kernel.
+    x = inp.heavy_tailed_bf16(7000 + M + H, M, H)
+    r = inp.normal_bf16(7100 + M + H, (M, H), std=2.0)
+    w = inp.rms_weight_bf16(7200 + H, H)
+    g = H if per_token else 128
+    q_ref, s_ref, r_ref = oracle.add_rmsnorm_quant(x, r, w, 1e-6, g, ue8m0)
+    rd = to_dev_bf16(r, ld=H + 64)                   # padded residual rows
+    q, s = fq.fp8q_add_rmsnorm_quant(to_dev_bf16(x), rd, to_dev_bf16(w[None, :])[0], 1e-6, g, ue8m0)
+    torch.cuda.synchronize()
+    got_r = rd.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(got_r, r_ref)
+    if ue8m0 == "packed":
+        np.testing.assert_array_equal(s.cpu().numpy(), s_ref)
+        assert_fused_quant_close(codes_np(q), np.zeros(1), q_ref, np.zeros(1), "add+rms packed")
+    else:
+        n = assert_fused_quant_close(codes_np(q), s.cpu().numpy(), q_ref, s_ref, "add+rms")
+        print(f"add+rms M={M} H={H} g={g} ue8m0={ue8m0}: {n} differing codes")
+
+
+def test_add_rmsnorm_quant_full_size_qwen3_32b():
+    # Qwen3-32B prefill: M = 8192 tokens, H = 5120; every row checked
+    M, H = 8192, 5120
+    x = inp.heavy_tailed_bf16(7301, M, H)
+    r = inp.heavy_tailed_bf16(7302, M, H)
+    w = inp.rms_weight_bf16(7303, H)
+    for g in (H, 128):
+        q_ref, s_ref, r_ref = oracle.add_rmsnorm_quant(x, r, w, 1e-6, g)
+        rd = to_dev_bf16(r)
+        q, s = fq.fp8q_add_rmsnorm_quant(to_dev_bf16(x), rd, to_dev_bf16(w[None, :])[0], 1e-6, g)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(rd.view(torch.int16).cpu().numpy().view(np.uint16), r_ref)
+        n = assert_fused_quant_close(codes_np(q), s.cpu().numpy(), q_ref, s_ref, "add+rms full")
+        print(f"add+rms full g={g}: {n} differing codes of {q_ref.size}")

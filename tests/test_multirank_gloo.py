@@ -63,8 +63,9 @@ def test_two_ranks_time_the_slowest_rank_and_count_every_ranks_flops():
     sys.path.insert(0, ROOT)
     import bench
     flops = bench.gemm_flops(2048)
-    # Qwen3-8B MLP block, two chains: 2 x (gate_up + down) = 4 x 2 M H I x 2
-    assert flops == 2 * (2 * 2048 * 4096 * 2 * 12288 + 2 * 2048 * 12288 * 4096)
+    # Qwen3-32B block linears, two schemes: 2 x (qkv + o + gate_up + down), 2 M N K each
+    H, I = 5120, 25600
+    assert flops == 2 * 2 * 2048 * (H * 10240 + 8192 * H + H * 2 * I + I * H)
     for rank in (0, 1):
         total_ms, e2e_ms, tflops = got[rank]
         assert total_ms == 11.0 and e2e_ms == 20.0
