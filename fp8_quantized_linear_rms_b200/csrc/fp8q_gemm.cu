@@ -92,12 +92,13 @@ struct Cfg {
   static_assert(!(BW && MX) && !(I8 && (BW || MX)), "one scale scheme");
   static constexpr int B_BYTES = BN * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;           // TMA bytes per stage
-  // Scale factors per stage (MX): one 512-byte chunk for the 128 MMA rows,
-  // one per 128 MMA columns; in TMEM 4 columns per chunk, double-buffered.
+  // Scale factors (MX): per pipeline stage a TMEM slot of 4 columns for the
+  // 128 MMA rows and 4 per 128 MMA columns, written by SF_WARPS warps (one
+  // per TMEM lane quadrant) with tcgen05.st.
   static constexpr int SFB_CHUNKS = (BN + 127) / 128;
-  static constexpr int SF_BYTES = MX ? 512 * (1 + SFB_CHUNKS) : 0;
   static constexpr int SF_COLS = 4 * (1 + SFB_CHUNKS);
-  static constexpr int STAGES_RAW = kSmemBudget / (STAGE_BYTES + SF_BYTES);
+  static constexpr int SF_WARPS = MX ? 4 : 0;
+  static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int EPI_WARPS = (BW && BN >= 128) ? 8 : 4;
   static constexpr int COL_GROUPS = EPI_WARPS / 4;        // column slices per TMEM lane quadrant
@@ -109,12 +110,12 @@ struct Cfg {
   static constexpr int CHUNK = BW ? (CPT >= 128 ? 8 : 16) : (CPT < 32 ? 16 : 32);
   static constexpr int NBUF = (BW && BN < 256) ? 4 : 2;    // TMEM accumulator buffers
   static constexpr int SF_COL0 = NBUF * BN;                 // first scale-factor column (MX)
-  static constexpr int TMEM_NEED = NBUF * BN + (MX ? 2 * SF_COLS : 0);
+  static constexpr int TMEM_NEED = NBUF * BN + (MX ? STAGES * SF_COLS : 0);
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                  : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int THREADS = 64 + 32 * (EPI_WARPS + SF_WARPS);
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * NBUF + 1) + 16;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * (STAGE_BYTES + SF_BYTES) + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
   static_assert(STAGES >= 2, "pipeline too shallow");
   static_assert(TMEM_NEED <= 512, "accumulators exceed TMEM");
   static_assert(CPT % CHUNK == 0 && (CHUNK == 8 || CHUNK == 16 || CHUNK == 32), "chunking");
@@ -214,8 +215,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * A_BYTES;
-  uint8_t* sSF = sB + S * C::B_BYTES;                      // MX: scale factors per stage
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSF + S * C::SF_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * C::B_BYTES);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + NB;
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&full[i], 1);
+      mbar_init(&full[i], 1 + C::SF_WARPS);     // TMA bytes (+ the SF warps' stores)
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < NB; ++i) {
@@ -267,7 +267,6 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
   griddep_launch_dependents();
 
   if (warp == 0) {
-   if constexpr (!MX) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !kTestStallProducer) {
       int it = 0;
@@ -291,16 +290,85 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
       }
     }
     __syncwarp();
-   } else {
-    // ------------------------------------------------------------ producer (MX, whole warp)
-    // Per stage, lane l writes the E8M0 scale factors of MMA rows l + 32 j
-    // (chunk 0) and MMA columns 128 h + l + 32 j (chunk 1 + h), each byte
-    // repeated over the four 32-deep K slices of the stage, at byte
-    // l * 16 + j * 4 of its chunk; then lane 0 arms the stage and issues its
-    // TMA loads.  Rows or columns outside the problem take the scale 1 (byte
-    // 127): their operands are zero-filled by TMA.  The scale bytes of a
-    // stage are loaded SFD stages ahead (a register ring), so their global
-    // latency hides behind the MMAs of the stages before it.
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = I8 ? idesc_s8_s32(BM, BN) : idesc_e4m3_f32(BM, BN);
+      int it = 0, t = 0, pc = 0;
+      bool ok = true;
+      SegIter si(p);
+      Seg g;
+      while (ok && si.next(p, g)) {
+        const int kb0 = g.kb0, kb1 = g.kb1;
+        uint32_t d = tmem_base;
+        int buf = 0;
+        if (!BW) {
+          buf = t & 1;
+          if (!mbar_wait(&tempty[buf], ((t >> 1) & 1) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          d = tmem_base + buf * BN;
+        }
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int st = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!mbar_wait(&full[st], ph, abort_flag, p.status)) { ok = false; break; }
+          int pb = 0;
+          if (BW) {
+            pb = pc % NB;
+            if (!mbar_wait(&tempty[pb], ((pc / NB) & 1) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+            d = tmem_base + pb * BN;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_kmajor_sw128(sA + st * A_BYTES);
+          const uint64_t bdesc = smem_desc_kmajor_sw128(sB + st * C::B_BYTES);
+          if constexpr (MX) {
+            // the four block-scaled MMAs of the stage, with the scale
+            // factors the SF warps stored in the stage's TMEM slot
+            const uint32_t sf = tmem_base + C::SF_COL0 + st * C::SF_COLS;
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              const uint32_t acc = (kb > kb0 || k > 0);
+              const uint32_t kid = static_cast<uint32_t>(k) << 30;
+              mma_mxf8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc_mx_e4m3(BM, BN, k), acc, sf | kid,
+                           (sf + 4) | kid);
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              const uint32_t acc = BW ? (k > 0) : (kb > kb0 || k > 0);
+              if constexpr (I8) mma_i8(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
+              else mma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);  // +32 bytes of K
+            }
+          }
+          mma_commit(&empty[st]);
+          if (BW) {
+            mma_commit(&tfull[pb]);
+            ++pc;
+          }
+        }
+        if (!ok) break;
+        if (!BW) {
+          mma_commit(&tfull[buf]);
+          ++t;
+        }
+      }
+      // Every MMA issued so far has completed once `drain` flips.
+      mma_commit(drain);
+      drain_wait(drain, 0);
+    }
+    __syncwarp();
+  } else if (MX && warp >= 2 + C::EPI_WARPS) {
+    // ------------------------------------------------------------ scale factors (MX)
+    // Four warps, one per TMEM lane quadrant.  For every stage each writes
+    // the E8M0 scale factors into its quadrant of the stage's TMEM slot --
+    // lane l, column c of the SFA chunk: MMA row 32 c + l; of SFB chunk h:
+    // MMA column 128 h + 32 c + l; each byte repeated over the stage's four
+    // 32-deep K slices -- waits for its stores and arrives on the stage's
+    // full barrier.  A slot is rewritten only after the empty barrier of its
+    // stage, so the MMAs that read it have completed.  Rows or columns
+    // outside the problem take the scale 1 (byte 127): their operands are
+    // zero-filled by TMA.  The scale bytes of a stage are loaded SFD stages
+    // ahead (a register ring) so their global latency stays off the path:
     //   no swap: raw[0..3] = A bytes of rows l + 32 j, raw[4..6] = the B
     //            bytes of the (at most three) 128-row weight blocks the
     //            tile's columns fall in;
@@ -309,9 +377,9 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
     constexpr int SFD = 4;
     constexpr int NRAW = SWAP ? 1 + 4 * C::SFB_CHUNKS : 7;
     constexpr uint32_t kOneByte = 127u;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int nb_rows = p.N >> 7;                    // weight block rows
     uint32_t raw[SFD][NRAW];
-    // iterator SFD stages ahead of the one being armed
     SegIter sai(p);
     Seg ga;
     bool amore = sai.next(p, ga);
@@ -354,7 +422,20 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
     bool ok = true;
     SegIter si(p);
     Seg g;
+    int tb_cur = -1;
+    uint32_t sel[C::SFB_CHUNKS][4];                  // no swap: which raw[4..6] each SFB word takes
     while (ok && si.next(p, g)) {
+      if (!SWAP && g.tb != tb_cur) {
+        tb_cur = g.tb;
+        const int nb0 = (g.tb * BN) >> 7;
+#pragma unroll
+        for (int h = 0; h < C::SFB_CHUNKS; ++h)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = 128 * h + lane + 32 * j;
+            sel[h][j] = c < BN ? static_cast<uint32_t>(((g.tb * BN + c) >> 7) - nb0) : 3u;
+          }
+      }
       for (int kb = g.kb0; kb < g.kb1; ++kb, ++it) {
         const int st = it % S;
         const uint32_t ph = (it / S) & 1;
@@ -366,22 +447,16 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
 #pragma unroll
           for (int i = 0; i < NRAW; ++i) raw[d][i] = raw[d + 1][i];
         load_ahead(raw[SFD - 1]);
-        int w_ok = 1;
-        if (lane == 0) w_ok = mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status);
-        if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) { ok = false; break; }
         uint32_t wa[4], wb[C::SFB_CHUNKS][4];
         if (!SWAP) {
-          const int nb0 = (g.tb * BN) >> 7;
 #pragma unroll
           for (int j = 0; j < 4; ++j) wa[j] = cur[j] * 0x01010101u;
 #pragma unroll
           for (int h = 0; h < C::SFB_CHUNKS; ++h)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const int c = 128 * h + lane + 32 * j;
-              const int rel = ((g.tb * BN + c) >> 7) - nb0;        // 0, 1 or 2
-              const uint32_t b = rel == 0 ? cur[4] : (rel == 1 ? cur[5] : cur[6]);
-              wb[h][j] = (c < BN ? b : kOneByte) * 0x01010101u;
+              const uint32_t k = sel[h][j];
+              wb[h][j] = (k == 0 ? cur[4] : k == 1 ? cur[5] : k == 2 ? cur[6] : kOneByte) * 0x01010101u;
             }
         } else {
 #pragma unroll
@@ -391,97 +466,20 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) wb[h][j] = cur[1 + 4 * h + j] * 0x01010101u;
         }
-        uint32_t* sf = reinterpret_cast<uint32_t*>(sSF + st * C::SF_BYTES);
-        *reinterpret_cast<uint4*>(sf + lane * 4) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        int w_ok = 1;
+        if (lane == 0) w_ok = mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status);
+        if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sfa = tmem_base + lane_addr + C::SF_COL0 + st * C::SF_COLS;
+        tmem_st_32x32b_x4(sfa, wa[0], wa[1], wa[2], wa[3]);
 #pragma unroll
         for (int h = 0; h < C::SFB_CHUNKS; ++h)
-          *reinterpret_cast<uint4*>(sf + 128 * (1 + h) + lane * 4) =
-              make_uint4(wb[h][0], wb[h][1], wb[h][2], wb[h][3]);
-        fence_proxy_async_smem();
+          tmem_st_32x32b_x4(sfa + 4 + 4 * h, wb[h][0], wb[h][1], wb[h][2], wb[h][3]);
+        tmem_st_wait();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
-          tma_load_2d(sA + st * A_BYTES, &tmA, &full[st], kb * BK, g.ta * BM);
-          tma_load_2d(sB + st * C::B_BYTES, &tmB, &full[st], kb * BK, g.tb * BN);
-        }
+        if (lane == 0) mbar_arrive(&full[st]);
       }
-    }
-    if (!ok && lane == 0) {
-      const int first = it - S > 0 ? it - S : 0;
-      for (int j = first; j < it; ++j) drain_wait(&full[j % S], (j / S) & 1);
-    }
-    __syncwarp();
-   }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = I8 ? idesc_s8_s32(BM, BN) : idesc_e4m3_f32(BM, BN);
-      int it = 0, t = 0, pc = 0;
-      bool ok = true;
-      SegIter si(p);
-      Seg g;
-      while (ok && si.next(p, g)) {
-        const int kb0 = g.kb0, kb1 = g.kb1;
-        uint32_t d = tmem_base;
-        int buf = 0;
-        if (!BW) {
-          buf = t & 1;
-          if (!mbar_wait(&tempty[buf], ((t >> 1) & 1) ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after();
-          d = tmem_base + buf * BN;
-        }
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int st = it % S;
-          const uint32_t ph = (it / S) & 1;
-          if (!mbar_wait(&full[st], ph, abort_flag, p.status)) { ok = false; break; }
-          int pb = 0;
-          if (BW) {
-            pb = pc % NB;
-            if (!mbar_wait(&tempty[pb], ((pc / NB) & 1) ^ 1u, abort_flag, p.status)) { ok = false; break; }
-            d = tmem_base + pb * BN;
-          }
-          tc_fence_after();
-          const uint64_t adesc = smem_desc_kmajor_sw128(sA + st * A_BYTES);
-          const uint64_t bdesc = smem_desc_kmajor_sw128(sB + st * C::B_BYTES);
-          if constexpr (MX) {
-            // this stage's scale factors into TMEM (slot alternates per
-            // stage), then the four block-scaled MMAs of the stage; tcgen05
-            // ops of one thread run in issue order.
-            const uint32_t sf = tmem_base + C::SF_COL0 + (it & 1) * C::SF_COLS;
-            const uint8_t* ssf = sSF + st * C::SF_BYTES;
-            tmem_cp_sf_chunk(sf, ssf);
-#pragma unroll
-            for (int h = 0; h < C::SFB_CHUNKS; ++h) tmem_cp_sf_chunk(sf + 4 + 4 * h, ssf + 512 * (1 + h));
-#pragma unroll
-            for (int k = 0; k < BK / UMMA_K; ++k) {
-              const uint32_t acc = (kb > kb0 || k > 0);
-              const uint32_t kid = static_cast<uint32_t>(k) << 30;
-              mma_mxf8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc_mx_e4m3(BM, BN, k), acc, sf | kid,
-                           (sf + 4) | kid);
-            }
-          } else {
-#pragma unroll
-            for (int k = 0; k < BK / UMMA_K; ++k) {
-              const uint32_t acc = BW ? (k > 0) : (kb > kb0 || k > 0);
-              if constexpr (I8) mma_i8(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
-              else mma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, acc);  // +32 bytes of K
-            }
-          }
-          mma_commit(&empty[st]);
-          if (BW) {
-            mma_commit(&tfull[pb]);
-            ++pc;
-          }
-        }
-        if (!ok) break;
-        if (!BW) {
-          mma_commit(&tfull[buf]);
-          ++t;
-        }
-      }
-      // Every MMA issued so far has completed once `drain` flips.
-      mma_commit(drain);
-      drain_wait(drain, 0);
     }
     __syncwarp();
   } else {

@@ -15,9 +15,15 @@
 // groups read consecutive heads of a token (coalesced); the group reduces the
 // sum of squares with shuffles, exchanges NeoX partners with one shuffle
 // (GPT-J pairs sit inside a thread) and each thread keeps several heads in
-// flight.  Arithmetic is fp32: r from rsqrtf refined by one Newton step,
-// the rotation by one FMA on a rounded product, each output rounded to bf16
-// once.
+// flight.  The norm is exact, as in the quant kernels: the sum of squares in
+// fp64 (squares of bf16 values are exact there), r = 1/sqrt(ss/D + eps) in
+// fp64, and n = bf16(x r) from the two ends rz(x r_lo) and rz(x r_hi) + 1 ulp
+// of fp32 values r_lo <= r <= r_hi; the rare elements whose ends round
+// differently are rounded from fp64 once.  y = bf16(n w) is one exactly
+// rounded bf16 product.  The rotation is fp32: a cos - b sin as
+// fma(a, cos, -p) - e with p = fl(b sin) and e its exact FMA residual, so the
+// difference keeps its accuracy when the two products nearly cancel; each
+// output is rounded to bf16 once.
 #include <cuda_bf16.h>
 
 #include <atomic>
@@ -49,6 +55,31 @@ __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
+// u v + s w (s = +-1) with the product w-term split exactly: p = fl(s w),
+// e = the rounding error of p (an FMA residual), result fma(u, v, p) + e.
+__device__ __forceinline__ float rot(float u, float v, float s, float w) {
+  const float pr = s * w;
+  const float e = fmaf(s, w, -pr);
+  return fmaf(u, v, pr) + e;
+}
+
+// bf16 (nearest even) of a double with one rounding: round to odd at fp32
+// (24 bits, two more than bf16 needs), then nearest-even to bf16.
+__device__ __noinline__ uint32_t f64_to_bf16_rn(double v) {
+  float f = __double2float_rz(v);
+  if (static_cast<double>(f) != v) f = __uint_as_float(__float_as_uint(f) | 1u);
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
+}
+
+// n = bf16(x r) exactly: the ends of |x r| from r_lo <= r <= r_hi decide the
+// rounding when they agree; otherwise x r is rounded from fp64.
+__device__ __forceinline__ uint32_t norm_bf16(float x, float r_lo, float r_hi, double r) {
+  const uint32_t a = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rz(x, r_lo))));
+  const uint32_t b = static_cast<uint32_t>(__bfloat16_as_ushort(
+      __float2bfloat16_rn(__uint_as_float(__float_as_uint(__fmul_rz(x, r_hi)) + 1u))));
+  return a == b ? a : f64_to_bf16_rn(static_cast<double>(x) * r);
+}
+
 __device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b) {   // one rounding
   const __nv_bfloat162 y = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&a),
                                    *reinterpret_cast<const __nv_bfloat162*>(&b));
@@ -88,20 +119,25 @@ __global__ void __launch_bounds__(kRopeThreads) qk_norm_rope_kernel(const RopePa
 #pragma unroll
     for (int u = 0; u < kRopeItems; ++u) {
       const uint32_t xw[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-      float ss = 0.0f;
+      double ss = 0.0;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) ss = fmaf(bf_lo(xw[k]), bf_lo(xw[k]), fmaf(bf_hi(xw[k]), bf_hi(xw[k]), ss));
+      for (int k = 0; k < 4; ++k) {
+        const double lo = bf_lo(xw[k]), hi = bf_hi(xw[k]);
+        ss = __fma_rn(lo, lo, __fma_rn(hi, hi, ss));
+      }
 #pragma unroll
       for (int o = G / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-      const float m = ss * (1.0f / D) + p.eps;
-      float r = rsqrtf(m);
-      r = fmaf(0.5f * r, fmaf(-m * r, r, 1.0f), r);          // one Newton step
+      const double r = 1.0 / sqrt(ss / static_cast<double>(D) + static_cast<double>(p.eps));
+      const float r_lo = __double2float_rd(r * (1.0 - 0x1p-40));
+      const float r_hi = __double2float_ru(r * (1.0 + 0x1p-40));
       const uint4 w = h[u] < p.hq ? wq : wk;
       const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
       float y[8];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const uint32_t yw = bf2_mul(pack_bf2(bf_lo(xw[k]) * r, bf_hi(xw[k]) * r), ww[k]);
+        const uint32_t nw = norm_bf16(bf_lo(xw[k]), r_lo, r_hi, r) |
+                            (norm_bf16(bf_hi(xw[k]), r_lo, r_hi, r) << 16);
+        const uint32_t yw = bf2_mul(nw, ww[k]);
         y[2 * k] = bf_lo(yw);
         y[2 * k + 1] = bf_hi(yw);
       }
@@ -127,8 +163,7 @@ __global__ void __launch_bounds__(kRopeThreads) qk_norm_rope_kernel(const RopePa
         const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
         const bool first = g < G / 2;          // this thread holds the a's
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          out[j] = first ? fmaf(y[j], c[j], -(z[j] * sn[j])) : fmaf(y[j], c[j], z[j] * sn[j]);
+        for (int j = 0; j < 8; ++j) out[j] = rot(y[j], c[j], first ? -z[j] : z[j], sn[j]);
       } else {
         const float4 c0 = __ldg(reinterpret_cast<const float4*>(cs + 4 * g));
         const float4 s0 = __ldg(reinterpret_cast<const float4*>(cs + D / 2 + 4 * g));
@@ -136,8 +171,8 @@ __global__ void __launch_bounds__(kRopeThreads) qk_norm_rope_kernel(const RopePa
         const float sn[4] = {s0.x, s0.y, s0.z, s0.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          out[2 * j] = fmaf(y[2 * j], c[j], -(y[2 * j + 1] * sn[j]));
-          out[2 * j + 1] = fmaf(y[2 * j + 1], c[j], y[2 * j] * sn[j]);
+          out[2 * j] = rot(y[2 * j], c[j], -y[2 * j + 1], sn[j]);
+          out[2 * j + 1] = rot(y[2 * j + 1], c[j], y[2 * j], sn[j]);
         }
       }
       if (ok[u])

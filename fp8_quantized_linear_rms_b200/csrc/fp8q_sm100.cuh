@@ -375,28 +375,11 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask) {
 // 32-deep K slice of A row r by the E8M0 scale SFA[r] and of B column c by
 // SFB[c] itself, so block-scaled products accumulate in TMEM with no register
 // promotion.  Scale factors live in TMEM: the scale of MMA row (or column) r
-// is in lane r % 32 of every lane quadrant, column (base + r / 32), and byte k
-// of that 32-bit column belongs to the k-th 32-deep K slice of a 128-deep
-// stage; the MMA picks the byte with the "scale factor id" (address bits
-// 30-31 and the instruction descriptor's id fields).
-
-// Make generic-proxy writes to shared memory visible to the async proxy
-// (tcgen05.cp, TMA) before they are signalled.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// One 512-byte scale-factor chunk -- 32 rows of 16 bytes in shared memory,
-// row l holding the scales of MMA rows l, l+32, l+64, l+96 (4 bytes each) --
-// into TMEM columns [taddr, taddr + 4) of all four lane quadrants
-// (tcgen05.cp 32x128b.warpx4).  Source descriptor: K-major, no swizzle, the
-// four 8-row core matrices 128 bytes apart (stride byte offset), version 1.
-__device__ __forceinline__ void tmem_cp_sf_chunk(uint32_t taddr, const void* src) {
-  const uint64_t desc = (static_cast<uint64_t>(smem_u32(src) & 0x3FFFF) >> 4) |
-                        (static_cast<uint64_t>(128 >> 4) << 32) | (1ull << 46);
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
-               : "memory");
-}
+// is in lane r % 32 of every lane quadrant (the same data in all four),
+// column (base + r / 32), and byte k of that 32-bit column belongs to the
+// k-th 32-deep K slice of a 128-deep stage; the MMA picks the byte with the
+// "scale factor id" (address bits 30-31 and the instruction descriptor's id
+// fields).
 
 // D[tmem] (+)= (A * SFA) * (B * SFB)^T, e4m3 x e4m3 -> f32, E8M0 scale
 // factors at TMEM addresses sfa / sfb (byte id in bits 30-31), one CTA.
@@ -410,6 +393,19 @@ __device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, u
           d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
+}
+
+// 32 lanes x 4 consecutive 32-bit columns from registers into TMEM (lane =
+// thread of the warp; the warp's lane quadrant is in taddr's lane field),
+// and the wait for this thread's TMEM stores.
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2,
+                                                  uint32_t r3) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r0),
+               "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // Instruction descriptor, kind::mxf8f6f4 with block scaling: A and B e4m3
