@@ -758,11 +758,88 @@ fp8q_status launch_ring(const QuantParams& p, int T, int nteams, int nbuf, int s
                        1, p, nbuf, nteams, T, stride, device_status_ptr());
 }
 
+// Group kernel: 1x128 groups of the SiLU*mul quant, which need no row-wide
+// value, as independent items.  Item i = (row i / G, group
+// i % G); a team of 16 consecutive threads owns one item, 8 elements (one
+// 16-byte chunk of x, or of gate and of up) per thread, so a warp reads two
+// groups' 256 contiguous bytes per load; every thread keeps kGroupItems items
+// in flight (all loads issued before any arithmetic).  The group amax is four
+// shuffles inside the team; codes and scales are exactly those of the row
+// kernels (same helpers, same exactness).  No block barriers.
+constexpr int kGroupThreads = 256;
+constexpr int kGroupItems = 4;
+
+template <int OP>
+__global__ void __launch_bounds__(kGroupThreads) quant_groups_kernel(const QuantParams p) {
+  constexpr int TEAMS = kGroupThreads / 16;
+  const int t = threadIdx.x & 15;
+  const int team = threadIdx.x >> 4;
+  const int64_t G = p.L >> 7;
+  const int64_t items = p.M * G;
+  griddep_wait();                 // x may come from the previous kernel
+  griddep_launch_dependents();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * TEAMS * kGroupItems;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * TEAMS * kGroupItems; base < items;
+       base += stride) {
+    int64_t row[kGroupItems], col[kGroupItems];
+    bool ok[kGroupItems];
+    uint4 a[kGroupItems], b[kGroupItems];
+#pragma unroll
+    for (int u = 0; u < kGroupItems; ++u) {
+      const int64_t it = base + team + static_cast<int64_t>(u) * TEAMS;
+      ok[u] = it < items;
+      row[u] = ok[u] ? it / G : 0;
+      col[u] = ok[u] ? (it - row[u] * G) * 128 + 8 * t : 0;      // element offset in the row
+      const uint16_t* xr = p.x + row[u] * p.ldx;
+      a[u] = ok[u] ? ld_stream(xr + col[u]) : make_uint4(0, 0, 0, 0);
+      if constexpr (OP == OP_SILU) b[u] = ok[u] ? ld_stream(xr + p.L + col[u]) : make_uint4(0, 0, 0, 0);
+      else b[u] = make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kGroupItems; ++u) {
+      uint4 y;
+      if constexpr (OP == OP_SILU) {
+        uint32_t d = 0;
+        bool bad = false;
+        y.x = silu_pair(a[u].x, b[u].x, d, bad);
+        y.y = silu_pair(a[u].y, b[u].y, d, bad);
+        y.z = silu_pair(a[u].z, b[u].z, d, bad);
+        y.w = silu_pair(a[u].w, b[u].w, d, bad);
+        if (d != 0 || bad) y = silu_chunk_fix(a[u], b[u], y);   // rare: exact recomputation
+      } else {
+        y = a[u];
+      }
+      float am = absmax2_to_f32(chunk_absmax2(y, 0u));
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+      const QScale qs = make_qscale(am, p.ue8m0, p.i8);
+      if (ok[u]) {
+        *reinterpret_cast<uint2*>(p.q + row[u] * p.ldq + col[u]) = codes_chunk(p, y, qs);
+        if (t == 0) store_scale(p, row[u] * p.s_sm + (col[u] >> 7) * p.s_sg, qs.s);
+      }
+    }
+  }
+}
+
 template <int OP>
 fp8q_status launch_quant(const QuantParams& p, cudaStream_t stream) {
   if (p.M == 0) return FP8Q_OK;
   const int64_t nchunks = p.L / 8;
   const bool per_token = p.group == p.L;
+  if constexpr (OP == OP_SILU) {
+    if (!per_token) {
+      // 1x128 groups: independent items, no row-wide reduction (measured:
+      // faster than the row kernels for SiLU*mul; for the plain quant the
+      // row kernel is faster)
+      constexpr int64_t per_block = (kGroupThreads / 16) * kGroupItems;
+      const int64_t items = p.M * (p.L >> 7);
+      int64_t blocks = (items + per_block - 1) / per_block;
+      const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
+      if (blocks > cap) blocks = cap;
+      return launch_kernel(quant_groups_kernel<OP>, dim3(static_cast<unsigned>(blocks)),
+                           dim3(kGroupThreads), 0, stream, 1, p);
+    }
+  }
   // 4 chunks (32 elements) per thread while that needs <= 512 threads, else 8.
   const int ch = nchunks > 4 * kMaxThreads ? 8 : 4;
   const int T = threads_for(nchunks, ch);
