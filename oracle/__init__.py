@@ -364,3 +364,16 @@ def qk_norm_rope(qkv_bits, hq: int, hk: int, hv: int, head_dim: int, eps: float,
     _load().oracle_qk_norm_rope(_ptr(x), T, L, hq, hk, D, ctypes.c_float(eps), _ptr(qw), _ptr(kw),
                                 _ptr(cs), _ptr(pos), int(bool(is_neox)))
     return x
+
+
+# ----------------------------------------------- gate_up GEMM + SiLU*mul quant (fused)
+def gate_up_silu_quant(a_q, b_q, sa, sb, group_size: int = 128, ue8m0=False, rows=None):
+    """The fused op's definition, written as the chain it replaces: the blockwise
+    gate_up GEMM (rows of A; W = [gate (I rows) | up (I rows)], block scales),
+    each output rounded to bf16 as the GEMM emits it, then SiLU*mul quant of
+    h = [h_gate | h_up].  Returns (q, s, h_bits) for the listed rows."""
+    y, _ = scaled_mm_blockwise(a_q, b_q, sa, sb, rows)
+    h = bf16_round(y)
+    h_bits = (h.view(np.uint32) >> 16).astype(np.uint16)
+    res = silu_mul_quant(h_bits, group_size, ue8m0)
+    return res + (h_bits,)

@@ -112,3 +112,22 @@ def test_scaled_mm_blockwise_e8m0_exact_rationals(M, N, K):
     y, ad = oracle.scaled_mm_blockwise_e8m0(a, b, sa, sb)
     dec = lambda t: t.view(ml_dtypes.float8_e8m0fnu).astype(np.float32)
     _close_to_exact(y, ad, exact.scaled_mm_blockwise_exact(a, b, dec(sa), dec(sb)))
+
+
+def test_gate_up_silu_quant_is_the_chain_on_the_exact_gemm():
+    # h = bf16 of the blockwise GEMM, compared with bf16 of the exact-rational
+    # GEMM (an independent computation); then the SiLU*mul quant of that h
+    M, I, K = 3, 128, 256
+    a = inp.random_e4m3_codes(71, (M, K))
+    b = inp.random_e4m3_codes(72, (2 * I, K))
+    sa = inp.random_scales(73, (M, K // 128))
+    sb = inp.random_scales(74, (2 * I // 128, K // 128))
+    q, s, h = oracle.gate_up_silu_quant(a, b, sa, sb, 128)
+    ex = exact.scaled_mm_blockwise_exact(a, b, sa, sb)
+    hx = np.array([[float(v) for v in row] for row in ex])
+    # the exact values, rounded to bf16 once by the (separately pinned) bf16 rounding
+    want = np.array([[np.float32(oracle.bf16_round(np.array([v]))[0]) for v in row] for row in hx])
+    np.testing.assert_array_equal(inp.bf16_bits_to_f32(h), want)
+    q2, s2 = oracle.silu_mul_quant(h, 128)
+    np.testing.assert_array_equal(q, q2)
+    np.testing.assert_array_equal(s, s2)
