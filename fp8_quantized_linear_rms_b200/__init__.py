@@ -10,8 +10,8 @@ package fails loudly if ``libfp8q.so`` is missing (build it with
 The names match the C ABI:
   fp8q_group_quant, fp8q_rmsnorm_quant, fp8q_add_rmsnorm_quant, fp8q_silu_mul_quant
                                                                 (activation quant)
-  fp8q_scaled_mm, fp8q_scaled_mm_blockwise, fp8q_scaled_mm_blockwise_e8m0
-                                                                (scaled FP8 GEMMs)
+  fp8q_scaled_mm, fp8q_scaled_mm_blockwise, fp8q_scaled_mm_blockwise_e8m0,
+  fp8q_scaled_mm_blockwise_silu_quant                           (scaled FP8 GEMMs)
   fp8q_workspace_bytes, fp8q_select_gemm_variant, fp8q_force_gemm_variant,
   fp8q_last_device_status, fp8q_status_string, fp8q_version
 """
@@ -62,6 +62,8 @@ _SIGS = {
                               ctypes.c_size_t, _P]),
     "fp8q_scaled_mm_blockwise": (_INT, [_P, _P, _P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I64,
                                         _P, ctypes.c_size_t, _P]),
+    "fp8q_scaled_mm_blockwise_silu_quant": (_INT, [_P, _P, _P, _I64, _I64, _P, _I64, _I64, _I64, _INT,
+                                                   _P, _I64, _P, _I64, _I64, _P]),
     "fp8q_scaled_mm_blockwise_e8m0": (_INT, [_P, _P, _P, _I64, _I64, _P, _I64, _I64, _I64, _P,
                                              _I64, _P, ctypes.c_size_t, _P]),
     "fp8q_scaled_mm_blockwise_noalloc": (_INT, [_P, _P, _P, _I64, _I64, _P, _I64, _I64, _I64, _P,
@@ -332,6 +334,48 @@ def fp8q_scaled_mm_blockwise_e8m0(a_q: torch.Tensor, b_q: torch.Tensor, a_sf: to
                                            _rowmajor(y, "y"), wp, wn, _stream(stream))
     _check("fp8q_scaled_mm_blockwise_e8m0", st)
     return y
+
+
+def interleave_gate_up(t: torch.Tensor, block: int = 128) -> torch.Tensor:
+    """Rows of a gate_up tensor [2I, ...] = [gate (I rows) | up (I rows)] reordered
+    into 128-row blocks [gate block 0 | up block 0 | gate block 1 | ...], the
+    weight layout fp8q_scaled_mm_blockwise_silu_quant reads (a setup-time
+    permutation of the weights; use block=1 for their [2I/128, K/128] scales)."""
+    n2 = t.shape[0]
+    if n2 % (2 * block):
+        raise ValueError(f"rows ({n2}) must be a multiple of {2 * block}")
+    nb = n2 // (2 * block)
+    rest = t.shape[1:]
+    g = t[: n2 // 2].reshape(nb, block, *rest)
+    u = t[n2 // 2:].reshape(nb, block, *rest)
+    return torch.stack([g, u], dim=1).reshape(n2, *rest).contiguous()
+
+
+def fp8q_scaled_mm_blockwise_silu_quant(a_q: torch.Tensor, b_q: torch.Tensor, a_scale: torch.Tensor,
+                                        b_scale: torch.Tensor, a_scale_layout: str = "row_major",
+                                        ue8m0=False, q=None, scales=None,
+                                        scale_layout: str = "row_major", stream=None):
+    """gate_up blockwise GEMM with the SiLU*mul 1x128 quant fused into its epilogue.
+    b_q [2I, K] and b_scale [2I/128, K/128] in the interleaved layout of
+    interleave_gate_up.  Returns (q e4m3 [M, I], scales [M, I/128] or [I/128, M])."""
+    for t, n in ((a_q, "a_q"), (b_q, "b_q")):
+        _need(t, torch.float8_e4m3fn, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _need(a_scale, torch.float32, "a_scale")
+    _need(b_scale, torch.float32, "b_scale")
+    M, K = a_q.shape
+    N2 = b_q.shape[0]
+    I = N2 // 2
+    sm, skb = (1, M) if a_scale_layout == "group_major" else (K // 128, 1)
+    mode = _ue8m0_mode(ue8m0)
+    if q is None:
+        q = torch.empty((M, I), dtype=torch.float8_e4m3fn, device=a_q.device)
+    scales, ssm, ssg = _scales_out(M, I, 128, scale_layout, a_q.device, scales, mode)
+    _check("fp8q_scaled_mm_blockwise_silu_quant", lib.fp8q_scaled_mm_blockwise_silu_quant(
+        a_q.data_ptr(), b_q.data_ptr(), a_scale.data_ptr(), sm, skb, b_scale.data_ptr(), M, N2, K, mode,
+        q.data_ptr(), _rowmajor(q, "q"), scales.data_ptr(), ssm, ssg, _stream(stream)))
+    return q, scales
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

@@ -36,6 +36,7 @@
 #include <unordered_map>
 
 #include "fp8q_common.cuh"
+#include "fp8q_quant_math.cuh"
 #include "fp8q_sm100.cuh"
 
 namespace fp8q {
@@ -48,6 +49,22 @@ constexpr int BK = 128;       // K bytes (e4m3 elements) per pipeline stage
 constexpr int UMMA_K = 32;    // K per tcgen05.mma for 8-bit operands
 constexpr int A_BYTES = BM * BK;
 constexpr int kSmemBudget = 200 * 1024;
+
+// Register split of the blockwise 128x256 kernel (setmaxnreg): its 8
+// epilogue warps hold 128 fp32 accumulators a thread, which leaves no room for
+// wide TMEM loads at the 168 registers a thread of a 10-warp CTA.  With the
+// split the CTA has 12 warps -- epilogue warps 0-7 (two warpgroups), the TMA
+// producer warp 8, the MMA warp 9, two idle -- and after setup the third
+// warpgroup drops to kRegLow registers while the epilogue warpgroups rise
+// to kRegHigh.  The sum 256 kRegHigh + 128 kRegLow = 60416 stays below the
+// CTA's allocation at launch even at 160 registers a thread (61440), so the
+// raise never waits.
+#ifndef FP8Q_REGSPLIT
+#define FP8Q_REGSPLIT 0
+#endif
+constexpr bool kRegSplit = FP8Q_REGSPLIT != 0;
+constexpr int kRegLow = 40, kRegHigh = 216;
+static_assert(256 * kRegHigh + 128 * kRegLow <= 384 * 160, "register split exceeds the launch allocation");
 
 // Test-only build switch (-DFP8Q_TEST_STALL_PRODUCER=1, never in the shipped
 // library): the GEMM's TMA producer issues nothing, so the MMA thread's first
@@ -81,6 +98,14 @@ struct GemmArgs {
   int64_t sfa_sm, sfa_skb;
   const uint8_t* sfb;
   int64_t sfb_snb;
+  // SiLU*mul quant fused into the epilogue (gate_up): codes q[m*sq_ldq + o],
+  // scale of group (m, o/128) at sq_s[m*sq_s_sm + (o/128)*sq_s_sg] (fp32, or
+  // an E8M0 byte when sq_ue8m0 = 2)
+  uint8_t* sq_q;
+  int64_t sq_ldq;
+  float* sq_s;
+  int64_t sq_s_sm, sq_s_sg;
+  int sq_ue8m0;
 };
 
 // MX: E8M0 block scales applied by the tensor core (kind::mxf8f6f4.block_scale);
@@ -107,13 +132,19 @@ struct Cfg {
   // flight (the next one loads while the current one is scaled); its
   // 256-column tile holds 128 fp32 accumulators per thread (8 epilogue warps,
   // 10 in all: 168 registers a thread), so it reads 8 columns at a time.
-  static constexpr int CHUNK = BW ? (CPT >= 128 ? 8 : 16) : (CPT < 32 ? 16 : 32);
+  static constexpr int CHUNK = BW ? (CPT >= 128 ? (kRegSplit && BN == 256 && !SWAP ? 32 : 8) : 16)
+                                  : (CPT < 32 ? 16 : 32);
   static constexpr int NBUF = (BW && BN < 256) ? 4 : 2;    // TMEM accumulator buffers
   static constexpr int SF_COL0 = NBUF * BN;                 // first scale-factor column (MX)
   static constexpr int TMEM_NEED = NBUF * BN + (MX ? STAGES * SF_COLS : 0);
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                  : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
-  static constexpr int THREADS = 64 + 32 * (EPI_WARPS + SF_WARPS);
+  // register split: see kRegSplit (blockwise 128x256 tiles only)
+  static constexpr bool REGSPLIT = kRegSplit && BW && BN == 256 && !SWAP;
+  static constexpr int W_PROD = REGSPLIT ? EPI_WARPS : 0;       // TMA producer warp
+  static constexpr int W_MMA = REGSPLIT ? EPI_WARPS + 1 : 1;    // TMEM allocator and MMA warp
+  static constexpr int EPI_BASE = REGSPLIT ? 0 : 2;             // first epilogue warp
+  static constexpr int THREADS = REGSPLIT ? 384 : 64 + 32 * (EPI_WARPS + SF_WARPS);
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * NBUF + 1) + 16;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
   static_assert(STAGES >= 2, "pipeline too shallow");
@@ -203,11 +234,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int BN, bool SWAP, bool BW, bool MX, bool I8>
+// SQ (blockwise, 128x256 tiles, no swap, whole K): the gate_up GEMM with the
+// SiLU*mul quant in its epilogue.  The weight rows come interleaved in
+// 128-row blocks, [gate block j | up block j] for j = 0, 1, ..., so tile tb
+// holds gate outputs [128 tb, 128 tb + 128) in columns 0-127 and the matching
+// up outputs in columns 128-255.  Each epilogue thread owns 64 gate and the
+// matching 64 up columns of its row; after the K loop it rounds both to bf16
+// as the GEMM emits them, applies the exact SiLU*mul of the quant kernels,
+// takes the 1x128 group amax with its partner thread (the other column
+// slice, same row) through shared memory and writes e4m3 codes and the
+// group's scale.  The 2I-wide bf16 intermediate is never written.
+template <int BN, bool SWAP, bool BW, bool MX, bool I8, bool SQ>
 __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs p) {
   using C = Cfg<BN, SWAP, BW, MX, I8>;
+  static_assert(!SQ || (BW && !SWAP && BN == 256 && C::EPI_WARPS == 8 && 64 % C::CHUNK == 0),
+                "the fused SiLU*mul quant epilogue runs on 128x256 blockwise tiles");
+  // SQ: per-slice partial group amax, double-buffered by tile parity, and the
+  // mbarrier (one arrival per epilogue warp and tile) that orders the exchange
+  __shared__ float sq_red[SQ ? 2 : 1][2][SQ ? BM : 1];
+  __shared__ uint64_t sq_bar;
   constexpr int S = C::STAGES;
   constexpr int NB = C::NBUF;
   extern __shared__ uint8_t smem_raw[];
@@ -235,14 +282,15 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
       mbar_init(&tempty[i], C::EPI_WARPS);
     }
     mbar_init(drain, 1);
+    if (SQ) mbar_init(&sq_bar, C::EPI_WARPS);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == C::W_PROD && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
-  if (warp == 1) {
+  if (warp == C::W_MMA) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -250,7 +298,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  if (warp == 0 && lane == 0) {
+  if (warp == C::W_PROD && lane == 0) {
     // The first weight tiles of this CTA into L2 while the previous kernel
     // finishes (weights: the MMA's A operand under Swap-AB, else B).
     SegIter si(p);
@@ -266,7 +314,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
   griddep_wait();
   griddep_launch_dependents();
 
-  if (warp == 0) {
+  auto role_producer = [&]() {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !kTestStallProducer) {
       int it = 0;
@@ -290,7 +338,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  };
+  auto role_mma = [&]() {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = I8 ? idesc_s8_s32(BM, BN) : idesc_e4m3_f32(BM, BN);
@@ -357,7 +406,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
       drain_wait(drain, 0);
     }
     __syncwarp();
-  } else if (MX && warp >= 2 + C::EPI_WARPS) {
+  };
+  auto role_sf = [&]() {
     // ------------------------------------------------------------ scale factors (MX)
     // Four warps, one per TMEM lane quadrant.  For every stage each writes
     // the E8M0 scale factors into its quadrant of the stage's TMEM slot --
@@ -482,15 +532,16 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
       }
     }
     __syncwarp();
-  } else {
+  };
+  auto role_epilogue = [&]() {
     // ------------------------------------------------------------ epilogue
-    const int e = warp - 2;
+    const int e = warp - C::EPI_BASE;
     const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
     const int cg = e >> 2;                     // column slice
     const int row = quad * 32 + lane;          // MMA-A row within the tile
     const int col0 = cg * C::CPT;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    int t = 0, pc = 0;
+    int t = 0, pc = 0, sq_t = 0;
     bool ok = true;
 
     SegIter si(p);
@@ -663,9 +714,11 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
         // problem reads the scales of row/column 0 instead: its output is never
         // written.  Weight block row: the whole tile (Swap-AB) or this warp's
         // 128-column slice (a slice never straddles a block row).
-        const int nb = SWAP ? ta : (tb * BN + col0) / 128;
+        // (SQ: the slice spans the tile's gate block row 2 tb and up block row 2 tb + 1)
+        const int nb = SWAP ? ta : (SQ ? 2 * tb : (tb * BN + col0) / 128);
         const bool slice_valid = SWAP || (tb * BN + col0) < p.N;
         int sb_o = static_cast<int>((slice_valid ? nb : 0) * p.sb_snb + kb0 * p.sb_skb);
+        int sb_o2 = SQ ? static_cast<int>((nb + 1) * p.sb_snb + kb0 * p.sb_skb) : 0;
         int sa_o[SWAP ? NCH : 1];
         if (!SWAP) {
           sa_o[0] = static_cast<int>((a_valid ? a_idx : 0) * p.sa_sm + kb0 * p.sa_skb);
@@ -676,15 +729,24 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
             sa_o[j] = static_cast<int>((m < p.M ? m : 0) * p.sa_sm + kb0 * p.sa_skb);
           }
         }
-        float sq[SD][SWAP ? NCH : 1];                  // non-swap: sa * sb of the row
+        constexpr int NSC = SWAP ? NCH : (SQ ? 2 : 1);  // scales per K block per thread
+        float sq[SD][NSC];                             // non-swap: sa * sb of the row (SQ: gate, up)
         int kl = kb0;                                  // next K block to load scales of
         auto load_scales = [&](float* out) {
           const bool in = kl < kb1;
           const float sbk = in ? __ldg(p.sb + sb_o) : 0.0f;
+          if constexpr (SQ) {
+            const float sa_k = in ? __ldg(p.sa + sa_o[0]) : 0.0f;
+            out[0] = sa_k * sbk;
+            out[1] = in ? sa_k * __ldg(p.sb + sb_o2) : 0.0f;
+            sa_o[0] += static_cast<int>(p.sa_skb);
+            sb_o2 += static_cast<int>(p.sb_skb);
+          } else {
 #pragma unroll
-          for (int j = 0; j < (SWAP ? NCH : 1); ++j) {
-            out[j] = in ? __ldg(p.sa + sa_o[j]) * sbk : 0.0f;
-            sa_o[j] += static_cast<int>(p.sa_skb);
+            for (int j = 0; j < (SWAP ? NCH : 1); ++j) {
+              out[j] = in ? __ldg(p.sa + sa_o[j]) * sbk : 0.0f;
+              sa_o[j] += static_cast<int>(p.sa_skb);
+            }
           }
           sb_o += static_cast<int>(p.sb_skb);
           ++kl;
@@ -694,15 +756,16 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
         int pb = pc % NB;
         uint32_t ph = (pc / NB) & 1;
         for (int kb = kb0; kb < kb1; ++kb) {
-          float sc0[SWAP ? NCH : 1];
+          float sc0[NSC];
 #pragma unroll
-          for (int j = 0; j < (SWAP ? NCH : 1); ++j) sc0[j] = sq[0][j];
+          for (int j = 0; j < NSC; ++j) sc0[j] = sq[0][j];
 #pragma unroll
           for (int q = 0; q + 1 < SD; ++q)
 #pragma unroll
-            for (int j = 0; j < (SWAP ? NCH : 1); ++j) sq[q][j] = sq[q + 1][j];
+            for (int j = 0; j < NSC; ++j) sq[q][j] = sq[q + 1][j];
           load_scales(sq[SD - 1]);
           const uint64_t srow2 = pair_f32(sc0[0], sc0[0]);
+          const uint64_t srow2u = pair_f32(sc0[NSC - 1], sc0[NSC - 1]);   // SQ: up half
           if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[pb], ph, abort_flag, p.status))) {
             ok = false;
             break;
@@ -711,15 +774,21 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
           // Chunk j + 1 is loaded while chunk j is scaled into the
           // accumulators; the buffer is handed back to the MMA as soon as the
           // last chunk has landed, before its FMAs.
-          const uint32_t tbuf = tmem_base + lane_addr + pb * BN + col0;
+          // (SQ: chunk j < NCH/2 is gate column 64 cg + 8 j of the tile,
+          // chunk j >= NCH/2 the matching up column 128 + 64 cg + 8 (j - NCH/2))
+          const uint32_t tbuf = tmem_base + lane_addr + pb * BN + (SQ ? 0 : col0);
+          auto ccol = [&](int j) {
+            return SQ ? (j < NCH / 2 ? 64 * cg + j * C::CHUNK : 128 + 64 * cg + (j - NCH / 2) * C::CHUNK)
+                      : j * C::CHUNK;
+          };
           uint32_t r[2][C::CHUNK];
-          tmem_ld_async<C::CHUNK>(tbuf, r[0]);
+          tmem_ld_async<C::CHUNK>(tbuf + ccol(0), r[0]);
 #pragma unroll
           for (int j = 0; j < NCH; ++j) {
             uint32_t* rc = r[j & 1];
             tmem_wait_regs<C::CHUNK>(rc);
             if (j + 1 < NCH) {
-              tmem_ld_async<C::CHUNK>(tbuf + (j + 1) * C::CHUNK, r[(j + 1) & 1]);
+              tmem_ld_async<C::CHUNK>(tbuf + ccol(j + 1), r[(j + 1) & 1]);
             } else {
               tc_fence_before();
               __syncwarp();
@@ -729,7 +798,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
             for (int i = 0; i < C::CHUNK; i += 2) {
               const uint64_t sc = SWAP ? pair_f32(__shfl_sync(0xFFFFFFFFu, sc0[SWAP ? j : 0], i),
                                                   __shfl_sync(0xFFFFFFFFu, sc0[SWAP ? j : 0], i + 1))
-                                       : srow2;
+                                       : ((SQ && j >= NCH / 2) ? srow2u : srow2);
               ffma2_acc(acc[(j * C::CHUNK + i) / 2], rc[i], rc[i + 1], sc);
             }
           }
@@ -740,23 +809,98 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
           ++pc;
         }
         if (!ok) break;
+        if constexpr (SQ) {
+          // gate values in acc[0, 32), up values in acc[32, 64) (pairs);
+          // h = bf16 of each, as the GEMM emits y; y = bf16(silu(h_gate) h_up)
+          uint4 yv[8];
+          uint32_t m2 = 0;
 #pragma unroll
-        for (int c = 0; c < C::CPT; c += C::CHUNK) {
-          float v[C::CHUNK];
+          for (int c = 0; c < 8; ++c) {
+            uint32_t gw[4], uw[4];
 #pragma unroll
-          for (int i = 0; i < C::CHUNK; i += 2) unpair_f32(acc[(c + i) / 2], v[i], v[i + 1]);
-          if (g.ncontrib == 1) emit(col0 + c, v);
-          else stash(col0 + c, v);
+            for (int k = 0; k < 4; ++k) {
+              float a0, a1, b0, b1;
+              unpair_f32(acc[4 * c + k], a0, a1);
+              unpair_f32(acc[32 + 4 * c + k], b0, b1);
+              gw[k] = pack_bf16x2(a0, a1);
+              uw[k] = pack_bf16x2(b0, b1);
+            }
+            uint32_t d = 0;
+            bool bad = false;
+            uint4 y;
+            y.x = silu_pair(gw[0], uw[0], d, bad);
+            y.y = silu_pair(gw[1], uw[1], d, bad);
+            y.z = silu_pair(gw[2], uw[2], d, bad);
+            y.w = silu_pair(gw[3], uw[3], d, bad);
+            if (d != 0 || bad)
+              y = silu_chunk_fix(make_uint4(gw[0], gw[1], gw[2], gw[3]), make_uint4(uw[0], uw[1], uw[2], uw[3]), y);
+            yv[c] = y;
+            m2 = chunk_absmax2(y, m2);
+          }
+          // group amax over the two column slices of the row: write this
+          // slice's partial, one arrival per warp, bounded wait for all 8
+          // warps of the tile, read the partner's.  The slot of tile t is
+          // written again at tile t + 2, after every warp has arrived for
+          // tile t + 1 and so has read it.
+          float am = absmax2_to_f32(m2);
+          const int par = sq_t & 1;
+          sq_red[par][cg][row] = am;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sq_bar);
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sq_bar, static_cast<uint32_t>(par), abort_flag, p.status))) {
+            ok = false;
+            break;
+          }
+          am = fmaxf(am, sq_red[par][cg ^ 1][row]);
+          ++sq_t;
+          const QScale qs = make_qscale(am, p.sq_ue8m0);
+          if (a_valid) {
+            uint8_t* qr = p.sq_q + static_cast<int64_t>(a_idx) * p.sq_ldq + tb * 128 + 64 * cg;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint2*>(qr + 8 * c) = quant_chunk(yv[c], qs);
+            if (cg == 0) {
+              const int64_t si = static_cast<int64_t>(a_idx) * p.sq_s_sm + static_cast<int64_t>(tb) * p.sq_s_sg;
+              if (p.sq_ue8m0 == 2) reinterpret_cast<uint8_t*>(p.sq_s)[si] = static_cast<uint8_t>(__float_as_uint(qs.s) >> 23);
+              else p.sq_s[si] = qs.s;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < C::CPT; c += C::CHUNK) {
+            float v[C::CHUNK];
+#pragma unroll
+            for (int i = 0; i < C::CHUNK; i += 2) unpair_f32(acc[(c + i) / 2], v[i], v[i + 1]);
+            if (g.ncontrib == 1) emit(col0 + c, v);
+            else stash(col0 + c, v);
+          }
+          if (g.ncontrib > 1) finish_split();
         }
-        if (g.ncontrib > 1) finish_split();
       }
     }
+  };
+  if constexpr (C::REGSPLIT) {
+    // the third warpgroup (producer, MMA, two idle warps) gives up registers,
+    // the two epilogue warpgroups take them; each role body sits inside its
+    // warpgroup's branch so its code is allocated under the new limit
+    if (warp >= 8) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegLow));
+      if (warp == C::W_PROD) role_producer();
+      else if (warp == C::W_MMA) role_mma();
+    } else {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegHigh));
+      role_epilogue();
+    }
+  } else {
+    if (warp == C::W_PROD) role_producer();
+    else if (warp == C::W_MMA) role_mma();
+    else if (MX && warp >= 2 + C::EPI_WARPS) role_sf();   // (MX kernels have no register split)
+    else if (warp >= C::EPI_BASE && warp < C::EPI_BASE + C::EPI_WARPS) role_epilogue();
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+  if (warp == C::W_MMA) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------ CTA pairs
@@ -1135,7 +1279,7 @@ bool tensor_map(const void* ptr, int64_t rows, int64_t k, int box_rows, CUtensor
   return true;
 }
 
-template <int BN, bool SWAP, bool BW, bool MX = false, bool I8 = false>
+template <int BN, bool SWAP, bool BW, bool MX = false, bool I8 = false, bool SQ = false>
 fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
                         cudaStream_t stream) {
   using C = Cfg<BN, SWAP, BW, MX, I8>;
@@ -1146,7 +1290,7 @@ fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev].load(std::memory_order_relaxed)) {
-    if (cudaFuncSetAttribute(gemm_kernel<BN, SWAP, BW, MX, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gemm_kernel<BN, SWAP, BW, MX, I8, SQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess)
       return FP8Q_ERR_CUDA;
     attr_done[dev].store(1, std::memory_order_relaxed);
@@ -1154,7 +1298,7 @@ fp8q_status launch_gemm(const void* a_op, const void* b_op, const GemmArgs& p,
   int grid;
   if (p.streamk) grid = (p.total_iters + p.seg_len - 1) / p.seg_len;
   else grid = p.units < num_sms() ? p.units : num_sms();
-  return launch_kernel(gemm_kernel<BN, SWAP, BW, MX, I8>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES,
+  return launch_kernel(gemm_kernel<BN, SWAP, BW, MX, I8, SQ>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES,
                        stream, 1, ma, mb, p);
 }
 
@@ -1639,6 +1783,54 @@ extern "C" fp8q_status fp8q_scaled_mm_blockwise_e8m0(const void* a_q, const void
   p.y = static_cast<uint16_t*>(y);
   p.ldy = ldy;
   return run_gemm<false, true>(a_q, b_q, p, pl, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" fp8q_status fp8q_scaled_mm_blockwise_silu_quant(
+    const void* a_q, const void* b_q, const float* a_scale, int64_t as_stride_m, int64_t as_stride_kb,
+    const float* b_scale, int64_t M, int64_t N2, int64_t K, int ue8m0, void* q, int64_t ldq,
+    float* scales, int64_t s_stride_m, int64_t s_stride_g, void* stream) {
+  if (M < 0 || N2 <= 0 || K <= 0 || M > kMaxDim || N2 > kMaxDim || K > kMaxDim) return FP8Q_ERR_INVALID_ARG;
+  if (N2 % 256 != 0 || K % 128 != 0 || as_stride_m < 0 || as_stride_kb < 0) return FP8Q_ERR_INVALID_ARG;
+  if (ue8m0 < 0 || ue8m0 > 2 || s_stride_m < 0 || s_stride_g < 0 || ldq < N2 / 2 || ldq % 16 != 0)
+    return FP8Q_ERR_INVALID_ARG;
+  if (M == 0) return FP8Q_OK;
+  if (!a_q || !b_q || !a_scale || !b_scale || !q || !scales) return FP8Q_ERR_INVALID_ARG;
+  if (!aligned(a_q, 16) || !aligned(b_q, 16) || !aligned(q, 16) || !aligned(a_scale, 4) ||
+      !aligned(b_scale, 4) || !aligned(scales, ue8m0 == 2 ? 1 : 4))
+    return FP8Q_ERR_INVALID_ARG;
+  if (!scale_offsets_fit(M, K, as_stride_m, as_stride_kb)) return FP8Q_ERR_INVALID_ARG;
+  // 128x256 single-CTA tiles over the whole K range (the epilogue needs the
+  // finished sums); a forced variant does not apply here.
+  const fp8q_gemm_variant v{0, 1, 256, 0};
+  const Plan pl = make_plan(M, N2, K, 1, v);
+  GemmArgs p{};
+  p.K = static_cast<int>(K);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N2);
+  p.sa = a_scale;
+  p.sa_sm = as_stride_m;
+  p.sa_skb = as_stride_kb;
+  p.sb = b_scale;
+  p.sb_sn = 0;
+  p.sb_snb = K / 128;
+  p.sb_skb = 1;
+  p.sq_q = static_cast<uint8_t*>(q);
+  p.sq_ldq = ldq;
+  p.sq_s = scales;
+  p.sq_s_sm = s_stride_m;
+  p.sq_s_sg = s_stride_g;
+  p.sq_ue8m0 = ue8m0;
+  p.tiles_a = pl.tiles_a;
+  p.tiles_b = pl.tiles_b;
+  p.kblocks = pl.kblocks;
+  p.split = 1;
+  p.kb_per_split = pl.kblocks;
+  p.units = pl.units;
+  p.max_contrib = 1;
+  p.status = device_status_ptr();
+  p.rows_a = p.M;
+  p.rows_b = p.N;
+  return launch_gemm<256, false, true, false, false, true>(a_q, b_q, p, static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------ no-allocation path

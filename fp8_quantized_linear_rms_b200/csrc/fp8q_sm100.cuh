@@ -284,8 +284,10 @@ __device__ __forceinline__ void tmem_ld_waited(uint32_t taddr, uint32_t* r) {
 // load in flight.
 template <int N>
 __device__ __forceinline__ void tmem_ld_async(uint32_t taddr, uint32_t* r) {
-  static_assert(N == 8 || N == 16, "tcgen05.ld width");
-  if constexpr (N == 8) {
+  static_assert(N == 8 || N == 16 || N == 32, "tcgen05.ld width");
+  if constexpr (N == 32) {
+    tmem_ld_32x32b_x32_raw(taddr, r);
+  } else if constexpr (N == 8) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
@@ -303,8 +305,16 @@ __device__ __forceinline__ void tmem_ld_async(uint32_t taddr, uint32_t* r) {
 }
 template <int N>
 __device__ __forceinline__ void tmem_wait_regs(uint32_t* r) {
-  static_assert(N == 8 || N == 16, "tcgen05.ld width");
-  if constexpr (N == 8) {
+  static_assert(N == 8 || N == 16 || N == 32, "tcgen05.ld width");
+  if constexpr (N == 32) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31]));
+  } else if constexpr (N == 8) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
                    "+r"(r[6]), "+r"(r[7]));

@@ -235,6 +235,32 @@ FP8Q_API fp8q_status fp8q_scaled_mm_blockwise(const void* a_q, const void* b_q, 
                                      void* stream);
 
 /*
+ * fp8q_scaled_mm_blockwise_silu_quant -- the gate_up projection with the
+ * SiLU*mul quant fused into its epilogue: one of the fusions "on either side
+ * of the path" that continue the pages' cut of the call count ("Helion in
+ * vLLM", "Kernels integrated into vLLM": fused ops replace chains of calls).
+ * Equal to, and bit-identical with,
+ *   h = fp8q_scaled_mm_blockwise(a, W)          (bf16 [M, 2I] = [gate | up])
+ *   q, scales = fp8q_silu_mul_quant(h, group_size = 128, ue8m0)
+ * run with the same 128x256 whole-K GEMM variant, without ever writing h.
+ *
+ *   b_q, b_scale  the gate_up weight [2I, K] and its [2I/128, K/128] block
+ *            scales with the rows interleaved in 128-row blocks:
+ *            [gate rows 0-127 | up rows 0-127 | gate 128-255 | up 128-255 | ...]
+ *            (block row 2j = gate block j, 2j + 1 = up block j)
+ *   N2       2I, a multiple of 256
+ *   a_q, a_scale, as_stride_m, as_stride_kb, M, K   as in fp8q_scaled_mm_blockwise
+ *   ue8m0, q [M, I] (ldq >= I, multiple of 16), scales, s_stride_m,
+ *   s_stride_g   as in fp8q_silu_mul_quant with group_size 128
+ * Runs 128x256 single-CTA tiles over the whole K range (no split-K and no
+ * workspace; fp8q_force_gemm_variant does not apply).
+ */
+FP8Q_API fp8q_status fp8q_scaled_mm_blockwise_silu_quant(
+    const void* a_q, const void* b_q, const float* a_scale, int64_t as_stride_m,
+    int64_t as_stride_kb, const float* b_scale, int64_t M, int64_t N2, int64_t K, int ue8m0,
+    void* q, int64_t ldq, float* scales, int64_t s_stride_m, int64_t s_stride_g, void* stream);
+
+/*
  * fp8q_scaled_mm_blockwise_e8m0 -- scaled_mm_blockwise with power-of-two
  * block scales stored as E8M0 bytes, the form the pages say DeepGEMM needs
  * on B200 ("Helion in vLLM" (24-ai.news), section "Practical limits"; E8M0

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def test_library_exports_every_declared_function():
     names = fq.header_functions()
-    assert len(names) == 19
+    assert len(names) == 20
     for n in names:
         assert hasattr(fq.lib, n), n
         assert callable(getattr(fq, n)), f"binding lacks {n}"
@@ -80,6 +80,12 @@ def test_invalid_arguments_rejected_before_launch():
               None) == fq.ERR_INVALID_ARG
     assert qr(None, 0, 1280, 8, 1, 1, 128, ctypes.c_float(1e-6), None, None, None, 16, None, 1,
               None) == fq.OK
+    # fused gate_up + SiLU quant: 2I not a multiple of 256, ldq < I, bad ue8m0
+    fs = L.fp8q_scaled_mm_blockwise_silu_quant
+    assert fs(fake, fake, fake, 2, 1, fake, 4, 384, 256, 0, fake, 192, fake, 2, 1, None) == fq.ERR_INVALID_ARG
+    assert fs(fake, fake, fake, 2, 1, fake, 4, 512, 256, 0, fake, 128, fake, 2, 1, None) == fq.ERR_INVALID_ARG
+    assert fs(fake, fake, fake, 2, 1, fake, 4, 512, 256, 3, fake, 256, fake, 2, 1, None) == fq.ERR_INVALID_ARG
+    assert fs(None, None, None, 2, 1, None, 0, 512, 256, 0, None, 256, None, 2, 1, None) == fq.OK
     # int8: K beyond the exact-sum range, group size, null scales
     assert L.fp8q_scaled_mm_i8(fake, fake, fake, 1, fake, 1, 4, 128, 133152 + 16, fake, 128, None, 0,
                                None) == fq.ERR_INVALID_ARG
@@ -190,3 +196,16 @@ def test_e8m0_variant_selection_host_logic():
         {"swap_ab": 0, "split_k": 3, "block_n": 224, "cta_pair": 0}
     assert fq.fp8q_workspace_bytes(4096, 6144, 4096, 2) > 0
     fq.fp8q_force_gemm_variant()
+
+
+def test_interleave_gate_up_layout():
+    import torch
+    I, K = 256, 4
+    w = torch.arange(2 * I * K, dtype=torch.float32).reshape(2 * I, K)
+    wi = fq.interleave_gate_up(w)
+    # block row 2j = gate rows [128 j, 128 j + 128), 2j + 1 = up rows [I + 128 j, ...)
+    assert torch.equal(wi[0:128], w[0:128]) and torch.equal(wi[128:256], w[I:I + 128])
+    assert torch.equal(wi[256:384], w[128:256]) and torch.equal(wi[384:512], w[I + 128:I + 256])
+    s = torch.arange(2 * I // 128, dtype=torch.float32)[:, None].repeat(1, 3)
+    si = fq.interleave_gate_up(s, block=1)
+    assert si[:, 0].tolist() == [0.0, 2.0, 1.0, 3.0]
