@@ -71,6 +71,8 @@ def parse():
                     help="per-op timing instead of the step: quant, gemm8b, decode32b, prefill32b, "
                          "e8m0, all (GPU), or oracle (the CPU oracle, all host cores and one core)")
     ap.add_argument("--reps", type=int, default=50)
+    ap.add_argument("--sweep-m", default=None,
+                    help="comma-separated token counts replacing each sweep's own list of M")
     return ap.parse_args()
 
 
@@ -744,6 +746,9 @@ def run_sweep(args):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    def sweep_ms(default):
+        return tuple(int(v) for v in args.sweep_m.split(",")) if args.sweep_m else default
+
     def timeit(fn):
         fn()
         torch.cuda.synchronize()
@@ -805,7 +810,7 @@ def run_sweep(args):
     which = args.sweep
     if which in ("quant", "all"):
         w = {h: bf16_rand((h,), 1, False) * 0.1 + 1.0 for h in (4096, 5120)}
-        for M in (16, 128, 2048, 8192):
+        for M in sweep_ms((16, 128, 2048, 8192)):
             cases = [("group_quant", 4096), ("rmsnorm_quant", 4096), ("rmsnorm_quant", 5120),
                      ("silu_mul_quant", 12288), ("silu_mul_quant", 25600)]
             for op, L in cases:
@@ -884,17 +889,17 @@ def run_sweep(args):
 
     if which in ("gemm8b", "all"):
         sh = inp.linear_shapes(inp.QWEN3_8B)
-        for M in (1, 16, 128, 2048):
+        for M in sweep_ms((1, 16, 128, 2048)):
             for layer in ("gate_up", "down"):
                 K, N = sh[layer]
                 gemm_case(f"qwen3-8b {layer}", M, N, K, False)
-        for M in (1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096):
+        for M in sweep_ms((1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096)):
             for layer in ("qkv", "o", "gate_up", "down"):
                 K, N = sh[layer]
                 gemm_case(f"qwen3-8b {layer}", M, N, K, True)
     if which in ("decode32b", "all"):
         sh = inp.linear_shapes(inp.QWEN3_32B)
-        for M in (1, 2, 4, 8, 16, 32, 64):
+        for M in sweep_ms((1, 2, 4, 8, 16, 32, 64)):
             for layer in ("qkv", "o", "gate_up", "down"):
                 K, N = sh[layer]
                 gemm_case(f"qwen3-32b {layer}", M, N, K, True)
@@ -906,7 +911,7 @@ def run_sweep(args):
                 gemm_case(f"qwen3-32b {layer}", 8192, N, K, bw)
     if which in ("e8m0", "all"):
         sh8, sh32 = inp.linear_shapes(inp.QWEN3_8B), inp.linear_shapes(inp.QWEN3_32B)
-        for M in (1, 16, 64, 256, 1024, 4096):
+        for M in sweep_ms((1, 16, 64, 256, 1024, 4096)):
             for layer in ("qkv", "o", "gate_up", "down"):
                 K, N = sh8[layer]
                 gemm_case(f"qwen3-8b {layer}", M, N, K, "e8m0")

@@ -418,6 +418,164 @@ fp8q_status launch_ring(const QuantParams& p, int T, int nteams, int nbuf, int s
                        1, p, nbuf, nteams, T, stride, device_status_ptr());
 }
 
+// Staged SiLU*mul kernel (long rows): persistent CTAs, one row at a time per
+// CTA.  Warp 0 (one lane) streams whole [gate | up] rows into NBUF slots of
+// shared memory with cp.async.bulk, as in the ring kernel; the other T threads
+// all work on the same row (chunk c to thread c mod T).  Per token: phase 1
+// turns each chunk of gate and up into y = bf16(silu(g) u), stores y over the
+// chunk's gate bytes and keeps the thread's amax; one CTA-wide reduction gives
+// the row's scale; phase 2 reads the y chunks back and writes the codes.  With
+// 1x128 groups the 16 threads of a group (one half-warp, T being a multiple of
+// 32) reduce its amax by shuffles and write the codes at once.  y never stays
+// in registers across the row reduction, so a row of 25600 values is worked on
+// by up to 992 threads instead of the ~400 that a register-resident row fits.
+// Slots go back to the producer after a proxy fence (the y stores are generic
+// writes to bytes the next bulk copy overwrites).  Waits are bounded as in the
+// ring kernel.
+constexpr int kStagedMaxThreads = 1024;
+
+template <bool PER_TOKEN>
+__global__ void __launch_bounds__(kStagedMaxThreads, 1)
+    silu_staged_kernel(const QuantParams p, int nbuf, int T, int row_stride_bytes, int* status) {
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint64_t full[kRingMaxBuf], empty[kRingMaxBuf];
+  __shared__ float red_f[32];
+  __shared__ volatile int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t copy_bytes = static_cast<uint32_t>(4 * p.L);
+  const int64_t nchunks = p.L >> 3;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nbuf; ++i) {
+      sm100::mbar_init(&full[i], 1);
+      sm100::mbar_init(&empty[i], T / 32);
+    }
+    abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();                 // x may come from the previous kernel
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int i = 0;
+      bool ok = true;
+      for (int64_t row = blockIdx.x; row < p.M; row += gridDim.x, ++i) {
+        const int slot = i % nbuf;
+        if (!sm100::mbar_wait(&empty[slot], ((i / nbuf) & 1) ^ 1u, &abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        sm100::mbar_arrive_expect_tx(&full[slot], copy_bytes);
+        sm100::bulk_load(ring + static_cast<size_t>(slot) * row_stride_bytes, p.x + row * p.ldx,
+                         copy_bytes, &full[slot]);
+      }
+      if (!ok) {
+        const int first = i - nbuf > 0 ? i - nbuf : 0;
+        for (int j = first; j < i; ++j) sm100::drain_wait(&full[j % nbuf], (j / nbuf) & 1);
+      }
+    }
+    return;
+  }
+
+  const int tid = threadIdx.x - 32;
+  constexpr int bar = 1;
+  int i = 0;
+  for (int64_t row = blockIdx.x; row < p.M; row += gridDim.x, ++i) {
+    const int slot = i % nbuf;
+    const bool ok = sm100::mbar_wait(&full[slot], (i / nbuf) & 1, &abort_flag, status);
+    if (sm100::team_any(!ok, bar, T)) break;
+    uint8_t* base = ring + static_cast<size_t>(slot) * row_stride_bytes;
+    uint8_t* qr = p.q + row * p.ldq;
+    auto silu_chunk = [&](int64_t c) {
+      const uint4 g = *reinterpret_cast<const uint4*>(base + 16 * c);
+      const uint4 u = *reinterpret_cast<const uint4*>(base + 2 * p.L + 16 * c);
+      uint32_t d = 0;
+      bool bad = false;
+      uint4 y;
+      y.x = silu_pair(g.x, u.x, d, bad);
+      y.y = silu_pair(g.y, u.y, d, bad);
+      y.z = silu_pair(g.z, u.z, d, bad);
+      y.w = silu_pair(g.w, u.w, d, bad);
+      if (d != 0 || bad) y = silu_chunk_fix(g, u, y);   // rare: exact recomputation
+      return y;
+    };
+    if constexpr (PER_TOKEN) {
+      uint32_t m2 = 0;
+#pragma unroll 2
+      for (int64_t c = tid; c < nchunks; c += T) {
+        const uint4 y = silu_chunk(c);
+        m2 = chunk_absmax2(y, m2);
+        *reinterpret_cast<uint4*>(base + 16 * c) = y;
+      }
+      const float amax = team_reduce(absmax2_to_f32(m2), MaxOp(), red_f, tid, T, bar);
+      const QScale qs = make_qscale(amax, p.ue8m0, p.i8);
+#pragma unroll 4
+      for (int64_t c = tid; c < nchunks; c += T)
+        *reinterpret_cast<uint2*>(qr + 8 * c) = codes_chunk(p, *reinterpret_cast<const uint4*>(base + 16 * c), qs);
+      if (tid == 0) store_scale(p, row * p.s_sm, qs.s);
+    } else {
+      // nchunks is a multiple of 16 and T of 32: a group's 16 chunks belong to
+      // one half-warp in the same pass, and a pass covers whole half-warps
+      // (the two halves of a warp may leave the loop one pass apart, so the
+      // shuffles name only the own half)
+      const uint32_t half = 0xFFFFu << (lane & 16);
+#pragma unroll 2
+      for (int64_t c0 = tid - (tid & 15); c0 < nchunks; c0 += T) {
+        const int64_t c = c0 + (tid & 15);
+        const uint4 y = silu_chunk(c);
+        float a = absmax2_to_f32(chunk_absmax2(y, 0u));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(half, a, o));
+        const QScale qs = make_qscale(a, p.ue8m0, p.i8);
+        *reinterpret_cast<uint2*>(qr + 8 * c) = codes_chunk(p, y, qs);
+        if ((tid & 15) == 0) store_scale(p, row * p.s_sm + (c >> 4) * p.s_sg, qs.s);
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) sm100::mbar_arrive(&empty[slot]);
+  }
+}
+
+// Staged-kernel geometry for a row of L values: T = the fewest threads (a
+// multiple of 32, at most 992) that cover the row's chunks in the fewest
+// passes, and as many row slots (at most 16) as fit the shared memory.  False
+// when fewer than two slots fit.
+bool staged_geometry(int64_t L, int* T, int* nbuf, int* stride) {
+  const int64_t nchunks = L >> 3;
+  const int64_t tmax = kStagedMaxThreads - 32;
+  const int64_t passes = (nchunks + tmax - 1) / tmax;
+  const int64_t t = ((nchunks + passes - 1) / passes + 31) / 32 * 32;
+  const int64_t st = (4 * L + 127) / 128 * 128;
+  if (st * 2 > kRingSmemMax) return false;
+  int64_t nb = kRingSmemMax / st;
+  if (nb > kRingMaxBuf) nb = kRingMaxBuf;
+  *T = static_cast<int>(t);
+  *nbuf = static_cast<int>(nb);
+  *stride = static_cast<int>(st);
+  return true;
+}
+
+template <bool PER_TOKEN>
+fp8q_status launch_staged(const QuantParams& p, int T, int nbuf, int stride, cudaStream_t stream) {
+  auto kern = silu_staged_kernel<PER_TOKEN>;
+  static std::atomic<int> attr_done[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return FP8Q_ERR_CUDA;
+  if (!attr_done[dev].load(std::memory_order_relaxed)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemMax) != cudaSuccess)
+      return FP8Q_ERR_CUDA;
+    attr_done[dev].store(1, std::memory_order_relaxed);
+  }
+  int64_t grid = num_sms();
+  if (grid > p.M) grid = p.M;
+  return launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(32 + T), nbuf * stride, stream, 1, p,
+                       nbuf, T, stride, device_status_ptr());
+}
+
 // Group kernel: 1x128 groups of the SiLU*mul quant, which need no row-wide
 // value, as independent items.  Item i = (row i / G, group
 // i % G); a team of 16 consecutive threads owns one item, 8 elements (one
@@ -487,6 +645,11 @@ fp8q_status launch_quant(const QuantParams& p, cudaStream_t stream) {
   const int64_t nchunks = p.L / 8;
   const bool per_token = p.group == p.L;
   if constexpr (OP == OP_SILU) {
+    // Long per-token rows: the staged kernel (measured faster than the ring
+    // and register kernels from 8192 values on).
+    int T = 0, nbuf = 0, stride = 0;
+    if (per_token && nchunks >= 1024 && staged_geometry(p.L, &T, &nbuf, &stride))
+      return launch_staged<true>(p, T, nbuf, stride, stream);
     if (!per_token) {
       // 1x128 groups: independent items, no row-wide reduction (measured:
       // faster than the row kernels for SiLU*mul; for the plain quant the
