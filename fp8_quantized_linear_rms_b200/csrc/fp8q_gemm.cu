@@ -699,13 +699,15 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
         if (g.ncontrib > 1) finish_split();
       } else {
         // -------- blockwise scales: promote each K-block partial into registers.
-        // The scales of the next SD K blocks are kept in flight in a register
-        // ring (stage 0 = the block being promoted), so the global-load
-        // latency of a block's scales overlaps the promotion of the blocks
-        // before it.  Swap-AB: the scale varies per column (token); lane l
+        // The raw scales of the next SD K blocks are kept in flight in a
+        // register ring (stage 0 = the block being promoted), so the
+        // global-load latency of a block's scales overlaps the promotion of
+        // the blocks before it; the product sa * sb is formed only when the
+        // block is consumed (forming it at load time would wait for the load
+        // right there).  Swap-AB: the scale varies per column (token); lane l
         // holds that of column c + l of every chunk.
         constexpr int NCH = C::CPT / C::CHUNK;
-        constexpr int SD = 4;
+        constexpr int SD = 3;
         uint64_t acc[C::CPT / 2];                      // fp32 pairs, columns 2i, 2i+1
 #pragma unroll
         for (int i = 0; i < C::CPT / 2; ++i) acc[i] = 0ull;
@@ -730,40 +732,41 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
           }
         }
         constexpr int NSC = SWAP ? NCH : (SQ ? 2 : 1);  // scales per K block per thread
-        float sq[SD][NSC];                             // non-swap: sa * sb of the row (SQ: gate, up)
+        constexpr int NA = SWAP ? NCH : 1;             // activation scales per K block
+        constexpr int NW = SQ ? 2 : 1;                 // weight scales per K block (SQ: gate, up)
+        float ra[SD][NA], rw[SD][NW];
         int kl = kb0;                                  // next K block to load scales of
-        auto load_scales = [&](float* out) {
+        auto load_scales = [&](float* a_out, float* w_out) {
           const bool in = kl < kb1;
-          const float sbk = in ? __ldg(p.sb + sb_o) : 0.0f;
+          w_out[0] = in ? __ldg(p.sb + sb_o) : 0.0f;
           if constexpr (SQ) {
-            const float sa_k = in ? __ldg(p.sa + sa_o[0]) : 0.0f;
-            out[0] = sa_k * sbk;
-            out[1] = in ? sa_k * __ldg(p.sb + sb_o2) : 0.0f;
-            sa_o[0] += static_cast<int>(p.sa_skb);
+            w_out[NW - 1] = in ? __ldg(p.sb + sb_o2) : 0.0f;
             sb_o2 += static_cast<int>(p.sb_skb);
-          } else {
+          }
 #pragma unroll
-            for (int j = 0; j < (SWAP ? NCH : 1); ++j) {
-              out[j] = in ? __ldg(p.sa + sa_o[j]) * sbk : 0.0f;
-              sa_o[j] += static_cast<int>(p.sa_skb);
-            }
+          for (int j = 0; j < NA; ++j) {
+            a_out[j] = in ? __ldg(p.sa + sa_o[j]) : 0.0f;
+            sa_o[j] += static_cast<int>(p.sa_skb);
           }
           sb_o += static_cast<int>(p.sb_skb);
           ++kl;
         };
 #pragma unroll
-        for (int q = 0; q < SD; ++q) load_scales(sq[q]);
+        for (int q = 0; q < SD; ++q) load_scales(ra[q], rw[q]);
         int pb = pc % NB;
         uint32_t ph = (pc / NB) & 1;
         for (int kb = kb0; kb < kb1; ++kb) {
-          float sc0[NSC];
+          float sc0[NSC];                              // sa * sb (SQ: gate, up)
 #pragma unroll
-          for (int j = 0; j < NSC; ++j) sc0[j] = sq[0][j];
+          for (int j = 0; j < NSC; ++j) sc0[j] = ra[0][SWAP ? j : 0] * rw[0][SQ ? j : 0];
 #pragma unroll
-          for (int q = 0; q + 1 < SD; ++q)
+          for (int q = 0; q + 1 < SD; ++q) {
 #pragma unroll
-            for (int j = 0; j < NSC; ++j) sq[q][j] = sq[q + 1][j];
-          load_scales(sq[SD - 1]);
+            for (int j = 0; j < NA; ++j) ra[q][j] = ra[q + 1][j];
+#pragma unroll
+            for (int j = 0; j < NW; ++j) rw[q][j] = rw[q + 1][j];
+          }
+          load_scales(ra[SD - 1], rw[SD - 1]);
           const uint64_t srow2 = pair_f32(sc0[0], sc0[0]);
           const uint64_t srow2u = pair_f32(sc0[NSC - 1], sc0[NSC - 1]);   // SQ: up half
           if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[pb], ph, abort_flag, p.status))) {
@@ -1149,20 +1152,26 @@ __global__ void __launch_bounds__(Cfg2<BN, BW>::THREADS, 1)
         for (int i = 0; i < C::CPT / 2; ++i) acc[i] = 0ull;
         const int nb = (tb * BN + col0) / 128;
         const bool slice_valid = (tb * BN + col0) < p.N;
+        // raw scales of the next SD K blocks in flight; sa * sb formed on use
         constexpr int SD = 4;
-        float srow_q[SD];
-        auto load_scale = [&](int kb) {
-          if (kb >= p.kblocks || !slice_valid || !m_valid) return 0.0f;
-          return __ldg(p.sa + m * p.sa_sm + kb * p.sa_skb) * __ldg(p.sb + nb * p.sb_snb + kb * p.sb_skb);
+        float ra[SD], rw[SD];
+        auto load_scale = [&](int kb, float& a, float& w) {
+          const bool in = kb < p.kblocks && slice_valid && m_valid;
+          a = in ? __ldg(p.sa + m * p.sa_sm + kb * p.sa_skb) : 0.0f;
+          w = in ? __ldg(p.sb + nb * p.sb_snb + kb * p.sb_skb) : 0.0f;
         };
 #pragma unroll
-        for (int q = 0; q < SD; ++q) srow_q[q] = load_scale(q);
+        for (int q = 0; q < SD; ++q) load_scale(q, ra[q], rw[q]);
         for (int kb = 0; kb < p.kblocks; ++kb) {
           const int pb = pc % NB;
-          const uint64_t srow2 = pair_f32(srow_q[0], srow_q[0]);
+          const float s0 = ra[0] * rw[0];
+          const uint64_t srow2 = pair_f32(s0, s0);
 #pragma unroll
-          for (int q = 0; q + 1 < SD; ++q) srow_q[q] = srow_q[q + 1];
-          srow_q[SD - 1] = load_scale(kb + SD);
+          for (int q = 0; q + 1 < SD; ++q) {
+            ra[q] = ra[q + 1];
+            rw[q] = rw[q + 1];
+          }
+          load_scale(kb + SD, ra[SD - 1], rw[SD - 1]);
           if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[pb], (pc / NB) & 1, abort_flag, p.status))) {
             ok = false;
             break;
