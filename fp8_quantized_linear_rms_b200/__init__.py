@@ -58,6 +58,8 @@ _SIGS = {
                                    _P]),
     "fp8q_add_rmsnorm_quant": (_INT, [_P, _P, _P, ctypes.c_float, _I64, _I64, _I64, _I64, _INT, _INT,
                                       _P, _I64, _P, _I64, _I64, _P]),
+    "fp8q_set_fused_quant_exact": (_INT, [_INT]),
+    "fp8q_get_fused_quant_exact": (_INT, []),
     "fp8q_scaled_mm": (_INT, [_P, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P, _I64, _P,
                               ctypes.c_size_t, _P]),
     "fp8q_scaled_mm_blockwise": (_INT, [_P, _P, _P, _I64, _I64, _P, _I64, _I64, _I64, _P, _I64,
@@ -518,6 +520,17 @@ def fp8q_force_gemm_variant(swap_ab: int | None = None, split_k: int = 1, block_
         return
     v = GemmVariant(int(swap_ab), int(split_k), int(block_n), int(cta_pair))
     _check("fp8q_force_gemm_variant", lib.fp8q_force_gemm_variant(ctypes.byref(v)))
+
+
+def fp8q_set_fused_quant_exact(exact: bool) -> None:
+    """Arithmetic of the producer-fused quant ops for the calls that follow
+    (process-wide): False (default) = fast y within the fused tolerance with
+    exact scales, True = bit-exact codes and scales."""
+    _check("fp8q_set_fused_quant_exact", lib.fp8q_set_fused_quant_exact(1 if exact else 0))
+
+
+def fp8q_get_fused_quant_exact() -> bool:
+    return bool(lib.fp8q_get_fused_quant_exact())
 
 
 def fp8q_last_device_status(stream=None) -> int:

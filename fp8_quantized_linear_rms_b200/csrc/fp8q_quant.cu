@@ -124,11 +124,22 @@ struct SmemRow {
   }
 };
 
+// Candidate margin of the fast fused ops: a fast y lies within 2 bf16 steps of
+// its definition (RMSNorm: n within one step, then one more rounding of n w;
+// SiLU*mul: within one step), so the exact amax of a group is the exact value
+// of an element whose fast value is within 2 steps of the fast amax, and no
+// element more than 4 steps below it can reach that.
+constexpr uint32_t kCandSteps = 4;
+
 // Quantize one row with a team of T threads (T a multiple of 32, CH chunks
 // of 8 elements per thread; chunk c of the row belongs to thread c mod T, so
 // every warp access is 512 contiguous bytes).  `release()` is called once the
 // row's input has been read into registers.
-template <int OP, bool PER_TOKEN, int CH, typename Src, typename Release>
+// FAST (RMSNorm and SiLU*mul): y from the fast arithmetic of the quant math
+// header, then the elements within kCandSteps of their group's fast amax
+// recomputed exactly before the scales are taken, so scales are exact and
+// codes differ from the definition only where a fast y does.
+template <int OP, bool PER_TOKEN, int CH, bool FAST, typename Src, typename Release>
 __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, const Src& src,
                                             int tid, int T, int bar_id, double* red_d,
                                             float* red_f, Release release) {
@@ -138,6 +149,32 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
 #pragma unroll
   for (int i = 0; i < CH; ++i) valid[i] = (tid + static_cast<int64_t>(i) * T) < nchunks;
   auto off = [&](int i) { return (tid + static_cast<int64_t>(i) * T) * 8; };
+  // FAST: bit i set when chunk i holds an element whose fast |y| is within
+  // kCandSteps bf16 steps of its group's fast amax (a team reduction per
+  // token, four shuffles per 128-group).
+  auto candidates = [&](const uint4* yy) {
+    uint32_t cand = 0;
+    if constexpr (PER_TOKEN) {
+      uint32_t m2 = 0;
+#pragma unroll
+      for (int i = 0; i < CH; ++i) m2 = chunk_absmax2(yy[i], m2);
+      const float thr =
+          bf16_steps_below(team_reduce(absmax2_to_f32(m2), MaxOp(), red_f, tid, T, bar_id), kCandSteps);
+#pragma unroll
+      for (int i = 0; i < CH; ++i)
+        cand |= static_cast<uint32_t>(valid[i] && absmax2_to_f32(chunk_absmax2(yy[i], 0u)) >= thr) << i;
+    } else {
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        const float a = absmax2_to_f32(chunk_absmax2(yy[i], 0u));
+        float am = a;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+        cand |= static_cast<uint32_t>(valid[i] && a >= bf16_steps_below(am, kCandSteps)) << i;
+      }
+    }
+    return cand;
+  };
 
   // Hot loops compute every value on the fast path and only flag the rare
   // chunks with a pair whose rounding the fast path cannot decide; the exact
@@ -162,7 +199,12 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
       }
 #pragma unroll
       for (int i = 0; i < SB; ++i) {
-        if (valid[i0 + i]) {
+        if (valid[i0 + i] && FAST && chunk_min_gate(g[i]) >= -85.0f) {
+          y[i0 + i].x = silu_pair_fast(g[i].x, u[i].x);
+          y[i0 + i].y = silu_pair_fast(g[i].y, u[i].y);
+          y[i0 + i].z = silu_pair_fast(g[i].z, u[i].z);
+          y[i0 + i].w = silu_pair_fast(g[i].w, u[i].w);
+        } else if (valid[i0 + i]) {
           uint32_t d = 0;
           bool bad = false;
           y[i0 + i].x = silu_pair(g[i].x, u[i].x, d, bad);
@@ -206,6 +248,65 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
       }
     }
     release();
+    bool exact_route = !FAST;
+    double r1 = 0.0;                // FAST: r from the fp32 sum of squares
+    if constexpr (FAST) {
+      // fp32 sum of squares in four packed accumulators (one per word of a
+      // chunk): each fp32 lane adds at most CH <= 8 squares, which are exact
+      // in fp32, so the relative error is <= 7 2^-24 < 2^-21.1; the eight
+      // lanes are added in fp64.  Rows whose sum leaves [2^-100, 2^120] (a
+      // square that overflows, or underflowed squares that could matter) take
+      // the exact route; the decision is the team's (ss is).
+      uint64_t s2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        uint64_t f = bf2_to_f2(xv[i].x);
+        s2[0] = fma2(f, f, s2[0]);
+        f = bf2_to_f2(xv[i].y);
+        s2[1] = fma2(f, f, s2[1]);
+        f = bf2_to_f2(xv[i].z);
+        s2[2] = fma2(f, f, s2[2]);
+        f = bf2_to_f2(xv[i].w);
+        s2[3] = fma2(f, f, s2[3]);
+      }
+      double part = 0.0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float lo, hi;
+        up2(s2[k], lo, hi);
+        part += static_cast<double>(lo) + static_cast<double>(hi);
+      }
+      const double ssf = team_reduce(part, SumOp(), red_d, tid, T, bar_id);
+      exact_route = !(ssf >= 0x1p-100 && ssf <= 0x1p120);
+      if (!exact_route) {
+        r1 = rms_r1(__fma_rn(ssf, 1.0 / static_cast<double>(p.L), static_cast<double>(p.eps)));
+        const uint64_t rf2 = dup2(__double2float_rn(r1));
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+          if (valid[i]) {
+            const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.w + off(i)));
+            y[i].x = bf2_mul(rms_n_pair_fast(xv[i].x, rf2), wv.x);
+            y[i].y = bf2_mul(rms_n_pair_fast(xv[i].y, rf2), wv.y);
+            y[i].z = bf2_mul(rms_n_pair_fast(xv[i].z, rf2), wv.z);
+            y[i].w = bf2_mul(rms_n_pair_fast(xv[i].w, rf2), wv.w);
+          } else {
+            y[i] = make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+    }
+    // FAST: the rare exact paths read the row's chunks again from global
+    // memory (x, or h as written back to the residual), so xv need not stay
+    // live past the fast y
+    auto reload = [&](int i) {
+      const uint16_t* src_row = OP == OP_ADD_RMS ? p.res + row * p.ldr : p.x + row * p.ldx;
+      return valid[i] ? ld_stream(src_row + off(i)) : make_uint4(0, 0, 0, 0);
+    };
+    if (exact_route) {
+    if constexpr (FAST) {
+#pragma unroll
+      for (int i = 0; i < CH; ++i) xv[i] = reload(i);
+    }
     // Sum of squares in fp64: squares of bf16 values are exact there (16
     // significant bits, exponents far inside the range).
     double a0 = 0.0, a1 = 0.0;
@@ -244,6 +345,83 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
           y[i] = rms_chunk_fix(xv[i], __ldg(reinterpret_cast<const uint4*>(p.w + off(i))), y[i], rlo2,
                                rhi2, ss, p.L, p.eps);
     }
+    }  // exact route
+    if constexpr (FAST) {
+      if (!exact_route) {
+        // The elements that can decide an amax, exactly: first with the
+        // bracket r1 (1 -+ 2^-21) around the fast r (its relative error is
+        // below 2^-22.1: half the sum's), and where that leaves a rounding
+        // open, with the exact sum of squares (the whole team, rarely).
+        const uint32_t cand = candidates(y);
+        float wlo, whi;
+        rms_bracket_of(r1, 0x1p-21, wlo, whi);
+        const uint64_t wlo2 = dup2(wlo), whi2 = dup2(whi);
+        bool open = false;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+          if ((cand >> i) & 1u) {
+            const uint4 xc = reload(i);
+            const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.w + off(i)));
+            uint32_t d = 0;
+            y[i].x = bf2_mul(rms_n_pair(xc.x, wlo2, whi2, d), wv.x);
+            y[i].y = bf2_mul(rms_n_pair(xc.y, wlo2, whi2, d), wv.y);
+            y[i].z = bf2_mul(rms_n_pair(xc.z, wlo2, whi2, d), wv.z);
+            y[i].w = bf2_mul(rms_n_pair(xc.w, wlo2, whi2, d), wv.w);
+            open |= d != 0;
+          }
+        }
+        if (sm100::team_any(open, bar_id, T)) {
+          double a0 = 0.0, a1 = 0.0;
+#pragma unroll
+          for (int i = 0; i < CH; ++i) {
+            const uint4 xc = reload(i);
+            const uint32_t xw[4] = {xc.x, xc.y, xc.z, xc.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const double lo = __uint_as_float(xw[k] << 16), hi = __uint_as_float(xw[k] & 0xFFFF0000u);
+              a0 = __fma_rn(lo, lo, a0);
+              a1 = __fma_rn(hi, hi, a1);
+            }
+          }
+          const double ss = team_reduce(a0 + a1, SumOp(), red_d, tid, T, bar_id);
+          float r_lo, r_hi;
+          rms_bracket(__fma_rn(ss, 1.0 / static_cast<double>(p.L), static_cast<double>(p.eps)), r_lo, r_hi);
+          const uint64_t rlo2 = dup2(r_lo), rhi2 = dup2(r_hi);
+#pragma unroll
+          for (int i = 0; i < CH; ++i) {
+            if ((cand >> i) & 1u) {
+              const uint4 xc = reload(i);
+              const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.w + off(i)));
+              uint32_t d = 0;
+              y[i].x = bf2_mul(rms_n_pair(xc.x, rlo2, rhi2, d), wv.x);
+              y[i].y = bf2_mul(rms_n_pair(xc.y, rlo2, rhi2, d), wv.y);
+              y[i].z = bf2_mul(rms_n_pair(xc.z, rlo2, rhi2, d), wv.z);
+              y[i].w = bf2_mul(rms_n_pair(xc.w, rlo2, rhi2, d), wv.w);
+              if (d != 0) y[i] = rms_chunk_fix(xc, wv, y[i], rlo2, rhi2, ss, p.L, p.eps);
+            }
+          }
+        }
+      }
+    }
+  }
+  if constexpr (FAST && OP == OP_SILU) {
+    // The elements that can decide an amax, exactly (their gate and up
+    // chunks read again from global memory).
+    const uint32_t cand = candidates(y);
+    const uint16_t* xr = p.x + row * p.ldx;
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+      if ((cand >> i) & 1u) {
+        const uint4 g = ld_stream(xr + off(i)), u = ld_stream(xr + p.L + off(i));
+        uint32_t d = 0;
+        bool bad = false;
+        y[i].x = silu_pair(g.x, u.x, d, bad);
+        y[i].y = silu_pair(g.y, u.y, d, bad);
+        y[i].z = silu_pair(g.z, u.z, d, bad);
+        y[i].w = silu_pair(g.w, u.w, d, bad);
+        if (d != 0 || bad) y[i] = silu_chunk_fix(g, u, y[i]);
+      }
+    }
   }
 
   uint8_t* qr = p.q + row * p.ldq;
@@ -279,14 +457,14 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
 // MAXT/MINB set the register budget (measured): 64 registers for 4 chunks
 // per thread (plain and RMSNorm: the occupancy beats the few spills), 80 for
 // SiLU rows of up to 384 threads, 128 for 8 chunks per thread.
-template <int OP, bool PER_TOKEN, int CH, int MAXT, int MINB>
+template <int OP, bool PER_TOKEN, int CH, int MAXT, int MINB, bool FAST>
 __global__ void __launch_bounds__(MAXT, MINB) quant_rows_kernel(const QuantParams p) {
   __shared__ double red_d[32];
   __shared__ float red_f[32];
   griddep_wait();                 // x (and w) may come from the previous kernel
   griddep_launch_dependents();
   for (int64_t row = blockIdx.x; row < p.M; row += gridDim.x)
-    process_row<OP, PER_TOKEN, CH>(p, row, GlobalRow{p.x + row * p.ldx}, threadIdx.x, blockDim.x,
+    process_row<OP, PER_TOKEN, CH, FAST>(p, row, GlobalRow{p.x + row * p.ldx}, threadIdx.x, blockDim.x,
                                    0, red_d, red_f, [] {});
 }
 
@@ -306,7 +484,7 @@ __host__ __device__ constexpr int ring_max_threads(int op, int ch) {
   return ch == 8 ? 512 : (op == OP_SILU ? 800 : (op == OP_ADD_RMS ? 768 : 1024));
 }
 
-template <int OP, bool PER_TOKEN, int CH>
+template <int OP, bool PER_TOKEN, int CH, bool FAST>
 __global__ void __launch_bounds__(ring_max_threads(OP, CH), 1)
     quant_ring_kernel(const QuantParams p, int nbuf, int nteams, int T, int row_stride_bytes,
                       int* status) {
@@ -362,7 +540,7 @@ __global__ void __launch_bounds__(ring_max_threads(OP, CH), 1)
     const bool ok = sm100::mbar_wait(&full[slot], (i / nbuf) & 1, &abort_flag, status);
     if (sm100::team_any(!ok, bar, T)) break;
     const uint16_t* src = reinterpret_cast<const uint16_t*>(ring + static_cast<size_t>(slot) * row_stride_bytes);
-    process_row<OP, PER_TOKEN, CH>(p, row, SmemRow{src}, tid, T, bar, red_d[team], red_f[team], [&] {
+    process_row<OP, PER_TOKEN, CH, FAST>(p, row, SmemRow{src}, tid, T, bar, red_d[team], red_f[team], [&] {
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&empty[slot]);
     });
@@ -398,11 +576,11 @@ bool ring_geometry(int64_t row_bytes, int T, int max_threads, int* nteams, int* 
   return true;
 }
 
-template <int OP, bool PER_TOKEN, int CH>
+template <int OP, bool PER_TOKEN, int CH, bool FAST>
 fp8q_status launch_ring(const QuantParams& p, int T, int nteams, int nbuf, int stride,
                         cudaStream_t stream) {
   const int smem = nbuf * stride;
-  auto kern = quant_ring_kernel<OP, PER_TOKEN, CH>;
+  auto kern = quant_ring_kernel<OP, PER_TOKEN, CH, FAST>;
   static std::atomic<int> attr_done[64];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -418,23 +596,32 @@ fp8q_status launch_ring(const QuantParams& p, int T, int nteams, int nbuf, int s
                        1, p, nbuf, nteams, T, stride, device_status_ptr());
 }
 
-// Staged SiLU*mul kernel (long rows): persistent CTAs, one row at a time per
-// CTA.  Warp 0 (one lane) streams whole [gate | up] rows into NBUF slots of
-// shared memory with cp.async.bulk, as in the ring kernel; the other T threads
-// all work on the same row (chunk c to thread c mod T).  Per token: phase 1
-// turns each chunk of gate and up into y = bf16(silu(g) u), stores y over the
-// chunk's gate bytes and keeps the thread's amax; one CTA-wide reduction gives
-// the row's scale; phase 2 reads the y chunks back and writes the codes.  With
-// 1x128 groups the 16 threads of a group (one half-warp, T being a multiple of
-// 32) reduce its amax by shuffles and write the codes at once.  y never stays
-// in registers across the row reduction, so a row of 25600 values is worked on
-// by up to 992 threads instead of the ~400 that a register-resident row fits.
-// Slots go back to the producer after a proxy fence (the y stores are generic
-// writes to bytes the next bulk copy overwrites).  Waits are bounded as in the
-// ring kernel.
+// Staged SiLU*mul per-token kernel (long rows): persistent CTAs, one row at
+// a time per CTA.  Warp 0 (one lane) streams whole [gate | up] rows into NBUF
+// slots of shared memory with cp.async.bulk, as in the ring kernel; the other T
+// threads all work on the same row (chunk c to thread c mod T, at most
+// kStagedPasses chunks a thread).  Phase 1 turns each chunk of gate and up into
+// y = bf16(silu(g) u), stores y over the chunk's gate bytes and keeps the
+// thread's amax; one CTA-wide reduction gives the row's scale; phase 2 reads
+// the y chunks back and writes the codes.  y never stays in registers across
+// the row reduction, so a row of 25600 values is worked on by up to 992
+// threads instead of the ~400 that a register-resident row fits.  FAST: the
+// chunks holding an element within kCandSteps of the fast amax are recomputed
+// exactly (gate and up read again from global memory) and the amax reduced
+// again.  Slots go back to the producer after a proxy fence (the y stores are
+// generic writes to bytes the next bulk copy overwrites).  Waits are bounded
+// as in the ring kernel.
 constexpr int kStagedMaxThreads = 1024;
+constexpr int kStagedPasses = 4;
 
-template <bool PER_TOKEN>
+// max of two packed pairs of bf16 magnitudes
+__device__ __forceinline__ uint32_t absmax2_merge(uint32_t a, uint32_t b) {
+  const __nv_bfloat162 m = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                   *reinterpret_cast<const __nv_bfloat162*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&m);
+}
+
+template <bool FAST>
 __global__ void __launch_bounds__(kStagedMaxThreads, 1)
     silu_staged_kernel(const QuantParams p, int nbuf, int T, int row_stride_bytes, int* status) {
   extern __shared__ __align__(128) uint8_t ring[];
@@ -488,9 +675,7 @@ __global__ void __launch_bounds__(kStagedMaxThreads, 1)
     if (sm100::team_any(!ok, bar, T)) break;
     uint8_t* base = ring + static_cast<size_t>(slot) * row_stride_bytes;
     uint8_t* qr = p.q + row * p.ldq;
-    auto silu_chunk = [&](int64_t c) {
-      const uint4 g = *reinterpret_cast<const uint4*>(base + 16 * c);
-      const uint4 u = *reinterpret_cast<const uint4*>(base + 2 * p.L + 16 * c);
+    auto exact_chunk = [](const uint4& g, const uint4& u) {
       uint32_t d = 0;
       bool bad = false;
       uint4 y;
@@ -501,38 +686,54 @@ __global__ void __launch_bounds__(kStagedMaxThreads, 1)
       if (d != 0 || bad) y = silu_chunk_fix(g, u, y);   // rare: exact recomputation
       return y;
     };
-    if constexpr (PER_TOKEN) {
-      uint32_t m2 = 0;
-#pragma unroll 2
-      for (int64_t c = tid; c < nchunks; c += T) {
-        const uint4 y = silu_chunk(c);
-        m2 = chunk_absmax2(y, m2);
+    uint32_t cm[kStagedPasses];      // packed absmax of each of this thread's chunks
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int k = 0; k < kStagedPasses; ++k) {
+      const int64_t c = tid + static_cast<int64_t>(k) * T;
+      cm[k] = 0;
+      if (c < nchunks) {
+        const uint4 g = *reinterpret_cast<const uint4*>(base + 16 * c);
+        const uint4 u = *reinterpret_cast<const uint4*>(base + 2 * p.L + 16 * c);
+        uint4 y;
+        if (FAST && chunk_min_gate(g) >= -85.0f) {
+          y.x = silu_pair_fast(g.x, u.x);
+          y.y = silu_pair_fast(g.y, u.y);
+          y.z = silu_pair_fast(g.z, u.z);
+          y.w = silu_pair_fast(g.w, u.w);
+        } else {
+          y = exact_chunk(g, u);
+        }
+        cm[k] = chunk_absmax2(y, 0u);
+        m2 = absmax2_merge(m2, cm[k]);
         *reinterpret_cast<uint4*>(base + 16 * c) = y;
       }
-      const float amax = team_reduce(absmax2_to_f32(m2), MaxOp(), red_f, tid, T, bar);
-      const QScale qs = make_qscale(amax, p.ue8m0, p.i8);
-#pragma unroll 4
-      for (int64_t c = tid; c < nchunks; c += T)
-        *reinterpret_cast<uint2*>(qr + 8 * c) = codes_chunk(p, *reinterpret_cast<const uint4*>(base + 16 * c), qs);
-      if (tid == 0) store_scale(p, row * p.s_sm, qs.s);
-    } else {
-      // nchunks is a multiple of 16 and T of 32: a group's 16 chunks belong to
-      // one half-warp in the same pass, and a pass covers whole half-warps
-      // (the two halves of a warp may leave the loop one pass apart, so the
-      // shuffles name only the own half)
-      const uint32_t half = 0xFFFFu << (lane & 16);
-#pragma unroll 2
-      for (int64_t c0 = tid - (tid & 15); c0 < nchunks; c0 += T) {
-        const int64_t c = c0 + (tid & 15);
-        const uint4 y = silu_chunk(c);
-        float a = absmax2_to_f32(chunk_absmax2(y, 0u));
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(half, a, o));
-        const QScale qs = make_qscale(a, p.ue8m0, p.i8);
-        *reinterpret_cast<uint2*>(qr + 8 * c) = codes_chunk(p, y, qs);
-        if ((tid & 15) == 0) store_scale(p, row * p.s_sm + (c >> 4) * p.s_sg, qs.s);
-      }
     }
+    float amax = team_reduce(absmax2_to_f32(m2), MaxOp(), red_f, tid, T, bar);
+    if constexpr (FAST) {
+      const float thr = bf16_steps_below(amax, kCandSteps);
+      const uint16_t* xr = p.x + row * p.ldx;
+      m2 = 0;
+#pragma unroll
+      for (int k = 0; k < kStagedPasses; ++k) {
+        const int64_t c = tid + static_cast<int64_t>(k) * T;
+        if (c < nchunks && absmax2_to_f32(cm[k]) >= thr) {
+          const uint4 y = exact_chunk(ld_stream(xr + 8 * c), ld_stream(xr + p.L + 8 * c));
+          cm[k] = chunk_absmax2(y, 0u);
+          *reinterpret_cast<uint4*>(base + 16 * c) = y;
+        }
+        m2 = absmax2_merge(m2, cm[k]);
+      }
+      amax = team_reduce(absmax2_to_f32(m2), MaxOp(), red_f, tid, T, bar);
+    }
+    const QScale qs = make_qscale(amax, p.ue8m0, p.i8);
+#pragma unroll
+    for (int k = 0; k < kStagedPasses; ++k) {
+      const int64_t c = tid + static_cast<int64_t>(k) * T;
+      if (c < nchunks)
+        *reinterpret_cast<uint2*>(qr + 8 * c) = codes_chunk(p, *reinterpret_cast<const uint4*>(base + 16 * c), qs);
+    }
+    if (tid == 0) store_scale(p, row * p.s_sm, qs.s);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
     if (lane == 0) sm100::mbar_arrive(&empty[slot]);
@@ -547,6 +748,7 @@ bool staged_geometry(int64_t L, int* T, int* nbuf, int* stride) {
   const int64_t nchunks = L >> 3;
   const int64_t tmax = kStagedMaxThreads - 32;
   const int64_t passes = (nchunks + tmax - 1) / tmax;
+  if (passes > kStagedPasses) return false;
   const int64_t t = ((nchunks + passes - 1) / passes + 31) / 32 * 32;
   const int64_t st = (4 * L + 127) / 128 * 128;
   if (st * 2 > kRingSmemMax) return false;
@@ -558,9 +760,9 @@ bool staged_geometry(int64_t L, int* T, int* nbuf, int* stride) {
   return true;
 }
 
-template <bool PER_TOKEN>
+template <bool FAST>
 fp8q_status launch_staged(const QuantParams& p, int T, int nbuf, int stride, cudaStream_t stream) {
-  auto kern = silu_staged_kernel<PER_TOKEN>;
+  auto kern = silu_staged_kernel<FAST>;
   static std::atomic<int> attr_done[64];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -587,7 +789,7 @@ fp8q_status launch_staged(const QuantParams& p, int T, int nbuf, int stride, cud
 constexpr int kGroupThreads = 256;
 constexpr int kGroupItems = 4;
 
-template <int OP>
+template <int OP, bool FAST>
 __global__ void __launch_bounds__(kGroupThreads) quant_groups_kernel(const QuantParams p) {
   constexpr int TEAMS = kGroupThreads / 16;
   const int t = threadIdx.x & 15;
@@ -597,6 +799,9 @@ __global__ void __launch_bounds__(kGroupThreads) quant_groups_kernel(const Quant
   griddep_wait();                 // x may come from the previous kernel
   griddep_launch_dependents();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * TEAMS * kGroupItems;
+  // item -> row: a 32-bit division whenever the item count allows it (a
+  // 64-bit one is a long software sequence, paid once per 8 elements)
+  const bool narrow = items <= 0xFFFFFFFFll;
   for (int64_t base = static_cast<int64_t>(blockIdx.x) * TEAMS * kGroupItems; base < items;
        base += stride) {
     int64_t row[kGroupItems], col[kGroupItems];
@@ -606,7 +811,9 @@ __global__ void __launch_bounds__(kGroupThreads) quant_groups_kernel(const Quant
     for (int u = 0; u < kGroupItems; ++u) {
       const int64_t it = base + team + static_cast<int64_t>(u) * TEAMS;
       ok[u] = it < items;
-      row[u] = ok[u] ? it / G : 0;
+      row[u] = !ok[u] ? 0
+               : narrow ? static_cast<int64_t>(static_cast<uint32_t>(it) / static_cast<uint32_t>(G))
+                        : it / G;
       col[u] = ok[u] ? (it - row[u] * G) * 128 + 8 * t : 0;      // element offset in the row
       const uint16_t* xr = p.x + row[u] * p.ldx;
       a[u] = ok[u] ? ld_stream(xr + col[u]) : make_uint4(0, 0, 0, 0);
@@ -616,7 +823,7 @@ __global__ void __launch_bounds__(kGroupThreads) quant_groups_kernel(const Quant
 #pragma unroll
     for (int u = 0; u < kGroupItems; ++u) {
       uint4 y;
-      if constexpr (OP == OP_SILU) {
+      auto exact_chunk = [&]() {
         uint32_t d = 0;
         bool bad = false;
         y.x = silu_pair(a[u].x, b[u].x, d, bad);
@@ -624,12 +831,30 @@ __global__ void __launch_bounds__(kGroupThreads) quant_groups_kernel(const Quant
         y.z = silu_pair(a[u].z, b[u].z, d, bad);
         y.w = silu_pair(a[u].w, b[u].w, d, bad);
         if (d != 0 || bad) y = silu_chunk_fix(a[u], b[u], y);   // rare: exact recomputation
+      };
+      if constexpr (OP == OP_SILU) {
+        if (FAST && chunk_min_gate(a[u]) >= -85.0f) {
+          y.x = silu_pair_fast(a[u].x, b[u].x);
+          y.y = silu_pair_fast(a[u].y, b[u].y);
+          y.z = silu_pair_fast(a[u].z, b[u].z);
+          y.w = silu_pair_fast(a[u].w, b[u].w);
+        } else {
+          exact_chunk();
+        }
       } else {
         y = a[u];
       }
       float am = absmax2_to_f32(chunk_absmax2(y, 0u));
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+      if constexpr (FAST && OP == OP_SILU) {
+        // the chunks that can decide the group's amax, exactly; amax again
+        const float mine = absmax2_to_f32(chunk_absmax2(y, 0u));
+        if (mine >= bf16_steps_below(am, kCandSteps)) exact_chunk();
+        am = absmax2_to_f32(chunk_absmax2(y, 0u));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+      }
       const QScale qs = make_qscale(am, p.ue8m0, p.i8);
       if (ok[u]) {
         *reinterpret_cast<uint2*>(p.q + row[u] * p.ldq + col[u]) = codes_chunk(p, y, qs);
@@ -639,17 +864,18 @@ __global__ void __launch_bounds__(kGroupThreads) quant_groups_kernel(const Quant
   }
 }
 
-template <int OP>
-fp8q_status launch_quant(const QuantParams& p, cudaStream_t stream) {
+template <int OP, bool FAST>
+fp8q_status launch_quant_mode(const QuantParams& p, cudaStream_t stream) {
   if (p.M == 0) return FP8Q_OK;
   const int64_t nchunks = p.L / 8;
   const bool per_token = p.group == p.L;
   if constexpr (OP == OP_SILU) {
-    // Long per-token rows: the staged kernel (measured faster than the ring
-    // and register kernels from 8192 values on).
+    // Long per-token rows (more than 2048 chunks): the staged kernel
+    // (measured at I = 25600: 399 us against 514 for the ring kernel; at
+    // I = 12288 the register kernel stays faster, 190 against 274 us).
     int T = 0, nbuf = 0, stride = 0;
-    if (per_token && nchunks >= 1024 && staged_geometry(p.L, &T, &nbuf, &stride))
-      return launch_staged<true>(p, T, nbuf, stride, stream);
+    if (per_token && nchunks > 2048 && staged_geometry(p.L, &T, &nbuf, &stride))
+      return launch_staged<FAST>(p, T, nbuf, stride, stream);
     if (!per_token) {
       // 1x128 groups: independent items, no row-wide reduction (measured:
       // faster than the row kernels for SiLU*mul; for the plain quant the
@@ -659,7 +885,7 @@ fp8q_status launch_quant(const QuantParams& p, cudaStream_t stream) {
       int64_t blocks = (items + per_block - 1) / per_block;
       const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
       if (blocks > cap) blocks = cap;
-      return launch_kernel(quant_groups_kernel<OP>, dim3(static_cast<unsigned>(blocks)),
+      return launch_kernel(quant_groups_kernel<OP, FAST>, dim3(static_cast<unsigned>(blocks)),
                            dim3(kGroupThreads), 0, stream, 1, p);
     }
   }
@@ -674,18 +900,32 @@ fp8q_status launch_quant(const QuantParams& p, cudaStream_t stream) {
   // (Measured: for rows of <= 2048 chunks the register kernel, with many
   // CTAs per SM, is faster than the ring.)
   if (ch == 8 && ring_geometry(row_bytes, T, ring_max_threads(OP, ch), &nteams, &nbuf, &stride))
-    return per_token ? launch_ring<OP, true, 8>(p, T, nteams, nbuf, stride, stream)
-                     : launch_ring<OP, false, 8>(p, T, nteams, nbuf, stride, stream);
+    return per_token ? launch_ring<OP, true, 8, FAST>(p, T, nteams, nbuf, stride, stream)
+                     : launch_ring<OP, false, 8, FAST>(p, T, nteams, nbuf, stride, stream);
   const int64_t grid = p.M < (1LL << 30) ? p.M : (1LL << 30);
   const dim3 g(static_cast<unsigned>(grid)), b(T);
   auto go = [&](auto kern) { return launch_kernel(kern, g, b, 0, stream, 1, p); };
   if (ch == 8)
-    return per_token ? go(quant_rows_kernel<OP, true, 8, 512, 1>) : go(quant_rows_kernel<OP, false, 8, 512, 1>);
+    return per_token ? go(quant_rows_kernel<OP, true, 8, 512, 1, FAST>) : go(quant_rows_kernel<OP, false, 8, 512, 1, FAST>);
   if (OP == OP_SILU && T <= 256)
-    return per_token ? go(quant_rows_kernel<OP, true, 4, 256, 3>) : go(quant_rows_kernel<OP, false, 4, 256, 3>);
+    return per_token ? go(quant_rows_kernel<OP, true, 4, 256, 3, FAST>) : go(quant_rows_kernel<OP, false, 4, 256, 3, FAST>);
   if (OP == OP_SILU && T <= 384)
-    return per_token ? go(quant_rows_kernel<OP, true, 4, 384, 2>) : go(quant_rows_kernel<OP, false, 4, 384, 2>);
-  return per_token ? go(quant_rows_kernel<OP, true, 4, 512, 2>) : go(quant_rows_kernel<OP, false, 4, 512, 2>);
+    return per_token ? go(quant_rows_kernel<OP, true, 4, 384, 2, FAST>) : go(quant_rows_kernel<OP, false, 4, 384, 2, FAST>);
+  return per_token ? go(quant_rows_kernel<OP, true, 4, 512, 2, FAST>) : go(quant_rows_kernel<OP, false, 4, 512, 2, FAST>);
+}
+
+// The fused ops (RMSNorm, SiLU*mul) run their fast y unless the exact mode is
+// set (fp8q_set_fused_quant_exact); the plain quant is always exact.
+std::atomic<int> g_fused_exact{0};
+
+template <int OP>
+fp8q_status launch_quant(const QuantParams& p, cudaStream_t stream) {
+  if constexpr (OP == OP_PLAIN) {
+    return launch_quant_mode<OP, false>(p, stream);
+  } else {
+    return g_fused_exact.load(std::memory_order_relaxed) ? launch_quant_mode<OP, false>(p, stream)
+                                                         : launch_quant_mode<OP, true>(p, stream);
+  }
 }
 
 // Host-side validation shared by the three ops (row length L of y).
@@ -803,3 +1043,11 @@ extern "C" fp8q_status fp8q_silu_mul_quant_i8(const void* x, int64_t M, int64_t 
                 static_cast<uint8_t*>(q), ldq, scales, s_stride_m, s_stride_g, nullptr, 0, 1};
   return launch_quant<OP_SILU>(p, static_cast<cudaStream_t>(stream));
 }
+
+extern "C" fp8q_status fp8q_set_fused_quant_exact(int exact) {
+  if (exact != 0 && exact != 1) return FP8Q_ERR_INVALID_ARG;
+  g_fused_exact.store(exact, std::memory_order_relaxed);
+  return FP8Q_OK;
+}
+
+extern "C" int fp8q_get_fused_quant_exact(void) { return g_fused_exact.load(std::memory_order_relaxed); }

@@ -248,20 +248,26 @@ __device__ __noinline__ uint4 rms_chunk_fix(const uint4 xv, const uint4 wv, uint
   return make_uint4(yw[0], yw[1], yw[2], yw[3]);
 }
 
-// Fast bracket of r = 1/sqrt(m): rsqrtf, one Newton step in fp64 (error
-// <= 1.5 e^2 + fp64 roundings, e <= 2^-21 the rsqrtf error: below 2^-40),
-// then the fp32 values just below and above r (1 -+ 2^-30).
-__device__ __forceinline__ void rms_bracket(double m, float& r_lo, float& r_hi) {
-  double r1;
+// r = 1/sqrt(m) in fp64: rsqrtf, one Newton step in fp64 (error
+// <= 1.5 e^2 + fp64 roundings, e <= 2^-21 the rsqrtf error: below 2^-40).
+__device__ __forceinline__ double rms_r1(double m) {
   if (m >= 0x1p-120 && m <= 0x1p120) {
     const double r0 = static_cast<double>(rsqrtf(static_cast<float>(m)));
     const double h = __fma_rn(-m * r0, r0, 1.0);          // 1 - m r0^2
-    r1 = __fma_rn(0.5 * r0, h, r0);
-  } else {
-    r1 = 1.0 / sqrt(m);
+    return __fma_rn(0.5 * r0, h, r0);
   }
-  r_lo = __double2float_rd(r1 * (1.0 - 0x1p-30));
-  r_hi = __double2float_ru(r1 * (1.0 + 0x1p-30));
+  return 1.0 / sqrt(m);
+}
+
+// fp32 bracket of r = r1 (1 +- rel): the fp32 values just below and above.
+__device__ __forceinline__ void rms_bracket_of(double r1, double rel, float& r_lo, float& r_hi) {
+  r_lo = __double2float_rd(r1 * (1.0 - rel));
+  r_hi = __double2float_ru(r1 * (1.0 + rel));
+}
+
+// Fast bracket of r = 1/sqrt(m) for an exact m: 1 -+ 2^-30 around rms_r1.
+__device__ __forceinline__ void rms_bracket(double m, float& r_lo, float& r_hi) {
+  rms_bracket_of(rms_r1(m), 0x1p-30, r_lo, r_hi);
 }
 
 // ---------------------------------------------------------------------------
@@ -307,7 +313,9 @@ __device__ __forceinline__ uint64_t silu_p2(uint64_t g2, uint64_t u2) {
 }
 
 // bf16 rounding of the low bracket end of a pair; `d` collects its XOR with
-// the high end; `bad` is set for tiny values and gates below -85.
+// the high end; `bad` is set for tiny values, tiny gates (g (1/(1+e^-g)) would
+// be an fp32 subnormal short of bits, which a large up value can lift back into
+// range) and gates below -85.
 __device__ __forceinline__ uint32_t silu_pair(uint32_t gw, uint32_t uw, uint32_t& d, bool& bad) {
   const uint64_t g2 = bf2_to_f2(gw);
   const uint64_t p = silu_p2(g2, bf2_to_f2(uw));
@@ -316,7 +324,7 @@ __device__ __forceinline__ uint32_t silu_pair(uint32_t gw, uint32_t uw, uint32_t
   float p0, p1, g0, g1;
   up2(p, p0, p1);
   up2(g2, g0, g1);
-  bad |= fminf(fabsf(p0), fabsf(p1)) < kTiny || fminf(g0, g1) < -85.0f;
+  bad |= fminf(fminf(fabsf(p0), fabsf(p1)), fminf(fabsf(g0), fabsf(g1))) < kTiny || fminf(g0, g1) < -85.0f;
   return na;
 }
 
@@ -334,7 +342,7 @@ __device__ __noinline__ uint32_t silu_pair_f64(uint32_t gw, uint32_t uw) {
 
 // Cold path of a flagged SiLU chunk: each element whose fast value is not
 // proven is recomputed exactly.  A zero gate or up value makes the fast
-// value an exact (signed) zero, so those tiny results are kept.
+// value an exact (signed) zero, so those results are kept.
 __device__ __noinline__ uint4 silu_chunk_fix(const uint4 g, const uint4 u, uint4 y) {
   const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, uw[4] = {u.x, u.y, u.z, u.w};
   uint32_t yw[4] = {y.x, y.y, y.z, y.w};
@@ -348,10 +356,59 @@ __device__ __noinline__ uint4 silu_chunk_fix(const uint4 g, const uint4 u, uint4
     up2(u2, uf[0], uf[1]);
     bool need = open != 0;
     for (int h = 0; h < 2; ++h)
-      need |= gf[h] < -85.0f || (fabsf(pf[h]) < kTiny && gf[h] != 0.0f && uf[h] != 0.0f);
+      need |= gf[h] < -85.0f ||
+              ((fabsf(pf[h]) < kTiny || fabsf(gf[h]) < kTiny) && gf[h] != 0.0f && uf[h] != 0.0f);
     if (need) yw[k] = silu_pair_f64(gw[k], uw[k]);
   }
   return make_uint4(yw[0], yw[1], yw[2], yw[3]);
+}
+
+// ---------------------------------------------------------------------------
+// Fast y (the fused ops' default mode).  y comes within one bf16 step of its
+// definition (differing only when the real value lies closer to a bf16
+// rounding midpoint than the fast value's error); the quant kernels recompute
+// exactly the elements that can decide a group's amax, so scales stay exact
+// and codes (from the exact IEEE quotient of y) differ only where y does.
+
+// bf16(x rf) of a pair, rf = fl32(r): one product, one rounding.
+__device__ __forceinline__ uint32_t rms_n_pair_fast(uint32_t xw, uint64_t rf2) {
+  return f2_to_bf2_rn(mul2(bf2_to_f2(xw), rf2));
+}
+
+// Fast bf16(silu(g) u) of a pair: (g u) / (1 + 2^(-g log2 e)) with ex2.approx
+// and rcp.approx.  For gates >= -85: the product g u is exact unless it
+// under- or overflows; the rounding of the exponent argument costs a relative
+// error of at most |g| 2^-23.5 ln 2 in 2^(.) (<= 2^-17.3), ex2.approx
+// 2^-22.7, 1 + e one rounding, rcp.approx 2^-23.3, the last product one
+// rounding: |error| <= 2^-17 relative, far below a bf16 step (2^-8); a tiny
+// or overflowing g u gives a value within a step of the rounded real one or
+// the flagged infinity.  Gates below -85 (2^(.) overflowing) are the caller's
+// to send to the exact path.
+__device__ __forceinline__ uint32_t silu_pair_fast(uint32_t gw, uint32_t uw) {
+  const float NL2E = -1.44269502f;          // -fl32(log2 e)
+  const uint64_t g2 = bf2_to_f2(gw);
+  float a0, a1;
+  up2(mul2(g2, dup2(NL2E)), a0, a1);
+  float d0, d1;
+  up2(add2(dup2(1.0f), pk2(ex2_approx(a0), ex2_approx(a1))), d0, d1);
+  return f2_to_bf2_rn(mul2(mul2(g2, bf2_to_f2(uw)), pk2(rcp_approx(d0), rcp_approx(d1))));
+}
+
+// Lowest gate of a chunk (packed bf16 minimum of its eight gate values; a NaN
+// gate is ignored, as the exact path's < -85 test ignores it).
+__device__ __forceinline__ float chunk_min_gate(const uint4& g) {
+  __nv_bfloat162 m = *reinterpret_cast<const __nv_bfloat162*>(&g.x);
+  m = __hmin2(m, *reinterpret_cast<const __nv_bfloat162*>(&g.y));
+  m = __hmin2(m, *reinterpret_cast<const __nv_bfloat162*>(&g.z));
+  m = __hmin2(m, *reinterpret_cast<const __nv_bfloat162*>(&g.w));
+  return fminf(__low2float(m), __high2float(m));
+}
+
+// The bf16 magnitude `steps` below a (a bf16 value as fp32, >= 0; 0 stays 0):
+// consecutive bf16 magnitudes are consecutive integers.
+__device__ __forceinline__ float bf16_steps_below(float a, uint32_t steps) {
+  const uint32_t b = __float_as_uint(a) >> 16;
+  return __uint_as_float((b > steps ? b - steps : 0u) << 16);
 }
 
 }  // namespace

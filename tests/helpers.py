@@ -2,6 +2,8 @@
 compare against the oracle with the stated tolerances."""
 from __future__ import annotations
 
+import contextlib
+
 import ml_dtypes
 import numpy as np
 import torch
@@ -112,3 +114,15 @@ def quantized_weights(seed: int, N: int, K: int, blockwise: bool):
     t = (wf / s[:, None, :, None]).astype(np.float32)
     q = oracle.e4m3_encode(t).reshape(N, K)
     return q, s
+
+
+@contextlib.contextmanager
+def fused_quant_exact(exact=True):
+    """Run the producer-fused quant ops in the given arithmetic mode (restored after)."""
+    import fp8_quantized_linear_rms_b200 as fq
+    prev = fq.fp8q_get_fused_quant_exact()
+    fq.fp8q_set_fused_quant_exact(exact)
+    try:
+        yield
+    finally:
+        fq.fp8q_set_fused_quant_exact(prev)

@@ -14,10 +14,24 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def test_library_exports_every_declared_function():
     names = fq.header_functions()
-    assert len(names) == 20
+    assert len(names) == 22
     for n in names:
         assert hasattr(fq.lib, n), n
         assert callable(getattr(fq, n)), f"binding lacks {n}"
+
+
+def test_fused_quant_mode_switch():
+    # host-side setting only: no GPU needed
+    assert fq.fp8q_get_fused_quant_exact() is False          # default: fast y, exact scales
+    try:
+        fq.fp8q_set_fused_quant_exact(True)
+        assert fq.fp8q_get_fused_quant_exact() is True
+        assert fq.lib.fp8q_set_fused_quant_exact(2) == fq.ERR_INVALID_ARG
+        assert fq.lib.fp8q_set_fused_quant_exact(-1) == fq.ERR_INVALID_ARG
+        assert fq.fp8q_get_fused_quant_exact() is True        # unchanged by a rejected value
+    finally:
+        fq.fp8q_set_fused_quant_exact(False)
+    assert fq.fp8q_get_fused_quant_exact() is False
 
 
 def test_status_strings_and_version():

@@ -14,9 +14,17 @@ import torch
 
 import fp8q_inputs as inp
 import oracle
-from helpers import codes_np, config_rows, quantized_weights, to_dev_codes
+from helpers import codes_np, config_rows, fused_quant_exact, quantized_weights, to_dev_codes
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _exact_standalone_quant():
+    # the fused epilogue computes y exactly; the standalone op it is compared
+    # with bit for bit runs in its exact mode
+    with fused_quant_exact(True):
+        yield
 
 if torch.cuda.is_available():
     import fp8_quantized_linear_rms_b200 as fq   # fails loudly if libfp8q.so is missing

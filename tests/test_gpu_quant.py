@@ -13,7 +13,7 @@ import torch
 
 import fp8q_inputs as inp
 import oracle
-from helpers import assert_fused_quant_close, codes_np, to_dev_bf16
+from helpers import assert_fused_quant_close, codes_np, fused_quant_exact, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -122,6 +122,34 @@ def test_silu_mul_extreme_gates():
         q, s = fq.fp8q_silu_mul_quant(to_dev_bf16(x), gs)
         torch.cuda.synchronize()
         assert_fused_quant_close(codes_np(q), s.cpu().numpy(), q_ref, s_ref, "silu tails")
+
+
+@pytest.mark.parametrize("I", [256, 12288])
+def test_silu_mul_tiny_gate_large_up(I):
+    # A gate so small that g / (1 + e^-g) is an fp32 subnormal, times an up
+    # value large enough to lift the product back into the normal range: each
+    # row's amax comes from such an element, so its bf16 value decides the
+    # scale.  Codes and scales must equal the definition bit for bit.
+    rng = np.random.default_rng(77)
+    g = rng.normal(0.0, 1e-3, size=(4, I))
+    u = rng.normal(0.0, 1e-3, size=(4, I))
+    for r, (gv, uv) in enumerate([(2.0 ** -133, 2.0 ** 120), (-(2.0 ** -128), 2.0 ** 115),
+                                  (2.0 ** -110, 2.0 ** 100), (3 * 2.0 ** -131, -(2.0 ** 118))]):
+        g[r, 5 + r] = gv
+        u[r, 5 + r] = uv
+    x = inp.to_bf16_bits(np.concatenate([g, u], axis=1))
+    for gs in (I, 128):
+        q_ref, s_ref = oracle.silu_mul_quant(x, gs)
+        with fused_quant_exact(True):
+            q, s = fq.fp8q_silu_mul_quant(to_dev_bf16(x), gs)
+            torch.cuda.synchronize()
+        np.testing.assert_array_equal(s.cpu().numpy(), s_ref)
+        np.testing.assert_array_equal(codes_np(q), q_ref)
+        # default (fast) mode: the deciding elements are exact, so are the scales
+        q, s = fq.fp8q_silu_mul_quant(to_dev_bf16(x), gs)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(s.cpu().numpy(), s_ref)
+        assert_fused_quant_close(codes_np(q), s.cpu().numpy(), q_ref, s_ref, "silu tiny gates, fast")
 
 
 @pytest.mark.parametrize("op", ["rmsnorm", "silu"])
