@@ -33,8 +33,9 @@ their own streams overlapping the neighbouring steps' kernels
 GEMM and quant launch against the measured peaks.  `e8m0_chain` times the
 blockwise stack again with packed UE8M0 scales and the block-scaled GEMM;
 `qk_norm_rope` times the attention-side fused op on the step's qkv output.
-The fused quant ops run in the library's default arithmetic (fast y with
-exact scales; fp8q_set_fused_quant_exact selects the bit-exact one).
+The quant ops run in the library's default arithmetic (per-token SiLU*mul
+with fast y and exact scales, the others bit-exact; fp8q_set_fused_quant_exact
+makes all of them bit-exact).
 `--impl reference` times the CPU oracle on a bounded sample of the workload.
 """
 from __future__ import annotations
@@ -118,8 +119,8 @@ def workload_config(M, n):
             "parallelism": f"replicas{n}" if n > 1 else "single-gpu",
             "l2": "flushed between timed steps (256 MiB write); the step's weights "
                   "(0.98 GB of e4m3) exceed L2 as well",
-            "fused_quant": "fast y, exact scales (the library default; codes within the fused "
-                           "tolerance)"}
+            "fused_quant": "library default: per-token SiLU*mul with fast y and exact scales "
+                           "(codes within the fused tolerance), the other quant ops bit-exact"}
 
 
 def load_peaks():

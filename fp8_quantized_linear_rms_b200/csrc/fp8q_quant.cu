@@ -124,21 +124,20 @@ struct SmemRow {
   }
 };
 
-// Candidate margin of the fast fused ops: a fast y lies within 2 bf16 steps of
-// its definition (RMSNorm: n within one step, then one more rounding of n w;
-// SiLU*mul: within one step), so the exact amax of a group is the exact value
-// of an element whose fast value is within 2 steps of the fast amax, and no
-// element more than 4 steps below it can reach that.
+// Candidate margin of the fast SiLU*mul: a fast y lies within one bf16 step
+// of its definition, so the exact amax of a group is the exact value of an
+// element whose fast value is within one step of the fast amax, and no element
+// more than 4 steps below it can reach that (a margin of two steps to spare).
 constexpr uint32_t kCandSteps = 4;
 
 // Quantize one row with a team of T threads (T a multiple of 32, CH chunks
 // of 8 elements per thread; chunk c of the row belongs to thread c mod T, so
 // every warp access is 512 contiguous bytes).  `release()` is called once the
 // row's input has been read into registers.
-// FAST (RMSNorm and SiLU*mul): y from the fast arithmetic of the quant math
-// header, then the elements within kCandSteps of their group's fast amax
-// recomputed exactly before the scales are taken, so scales are exact and
-// codes differ from the definition only where a fast y does.
+// FAST (SiLU*mul): y from the fast arithmetic of the quant math header, then
+// the elements within kCandSteps of their group's fast amax recomputed
+// exactly before the scales are taken, so scales are exact and codes differ
+// from the definition only where a fast y does.
 template <int OP, bool PER_TOKEN, int CH, bool FAST, typename Src, typename Release>
 __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, const Src& src,
                                             int tid, int T, int bar_id, double* red_d,
@@ -248,65 +247,6 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
       }
     }
     release();
-    bool exact_route = !FAST;
-    double r1 = 0.0;                // FAST: r from the fp32 sum of squares
-    if constexpr (FAST) {
-      // fp32 sum of squares in four packed accumulators (one per word of a
-      // chunk): each fp32 lane adds at most CH <= 8 squares, which are exact
-      // in fp32, so the relative error is <= 7 2^-24 < 2^-21.1; the eight
-      // lanes are added in fp64.  Rows whose sum leaves [2^-100, 2^120] (a
-      // square that overflows, or underflowed squares that could matter) take
-      // the exact route; the decision is the team's (ss is).
-      uint64_t s2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int i = 0; i < CH; ++i) {
-        uint64_t f = bf2_to_f2(xv[i].x);
-        s2[0] = fma2(f, f, s2[0]);
-        f = bf2_to_f2(xv[i].y);
-        s2[1] = fma2(f, f, s2[1]);
-        f = bf2_to_f2(xv[i].z);
-        s2[2] = fma2(f, f, s2[2]);
-        f = bf2_to_f2(xv[i].w);
-        s2[3] = fma2(f, f, s2[3]);
-      }
-      double part = 0.0;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float lo, hi;
-        up2(s2[k], lo, hi);
-        part += static_cast<double>(lo) + static_cast<double>(hi);
-      }
-      const double ssf = team_reduce(part, SumOp(), red_d, tid, T, bar_id);
-      exact_route = !(ssf >= 0x1p-100 && ssf <= 0x1p120);
-      if (!exact_route) {
-        r1 = rms_r1(__fma_rn(ssf, 1.0 / static_cast<double>(p.L), static_cast<double>(p.eps)));
-        const uint64_t rf2 = dup2(__double2float_rn(r1));
-#pragma unroll
-        for (int i = 0; i < CH; ++i) {
-          if (valid[i]) {
-            const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.w + off(i)));
-            y[i].x = bf2_mul(rms_n_pair_fast(xv[i].x, rf2), wv.x);
-            y[i].y = bf2_mul(rms_n_pair_fast(xv[i].y, rf2), wv.y);
-            y[i].z = bf2_mul(rms_n_pair_fast(xv[i].z, rf2), wv.z);
-            y[i].w = bf2_mul(rms_n_pair_fast(xv[i].w, rf2), wv.w);
-          } else {
-            y[i] = make_uint4(0, 0, 0, 0);
-          }
-        }
-      }
-    }
-    // FAST: the rare exact paths read the row's chunks again from global
-    // memory (x, or h as written back to the residual), so xv need not stay
-    // live past the fast y
-    auto reload = [&](int i) {
-      const uint16_t* src_row = OP == OP_ADD_RMS ? p.res + row * p.ldr : p.x + row * p.ldx;
-      return valid[i] ? ld_stream(src_row + off(i)) : make_uint4(0, 0, 0, 0);
-    };
-    if (exact_route) {
-    if constexpr (FAST) {
-#pragma unroll
-      for (int i = 0; i < CH; ++i) xv[i] = reload(i);
-    }
     // Sum of squares in fp64: squares of bf16 values are exact there (16
     // significant bits, exponents far inside the range).
     double a0 = 0.0, a1 = 0.0;
@@ -344,64 +284,6 @@ __device__ __forceinline__ void process_row(const QuantParams& p, int64_t row, c
         if ((fix >> i) & 1u)
           y[i] = rms_chunk_fix(xv[i], __ldg(reinterpret_cast<const uint4*>(p.w + off(i))), y[i], rlo2,
                                rhi2, ss, p.L, p.eps);
-    }
-    }  // exact route
-    if constexpr (FAST) {
-      if (!exact_route) {
-        // The elements that can decide an amax, exactly: first with the
-        // bracket r1 (1 -+ 2^-21) around the fast r (its relative error is
-        // below 2^-22.1: half the sum's), and where that leaves a rounding
-        // open, with the exact sum of squares (the whole team, rarely).
-        const uint32_t cand = candidates(y);
-        float wlo, whi;
-        rms_bracket_of(r1, 0x1p-21, wlo, whi);
-        const uint64_t wlo2 = dup2(wlo), whi2 = dup2(whi);
-        bool open = false;
-#pragma unroll
-        for (int i = 0; i < CH; ++i) {
-          if ((cand >> i) & 1u) {
-            const uint4 xc = reload(i);
-            const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.w + off(i)));
-            uint32_t d = 0;
-            y[i].x = bf2_mul(rms_n_pair(xc.x, wlo2, whi2, d), wv.x);
-            y[i].y = bf2_mul(rms_n_pair(xc.y, wlo2, whi2, d), wv.y);
-            y[i].z = bf2_mul(rms_n_pair(xc.z, wlo2, whi2, d), wv.z);
-            y[i].w = bf2_mul(rms_n_pair(xc.w, wlo2, whi2, d), wv.w);
-            open |= d != 0;
-          }
-        }
-        if (sm100::team_any(open, bar_id, T)) {
-          double a0 = 0.0, a1 = 0.0;
-#pragma unroll
-          for (int i = 0; i < CH; ++i) {
-            const uint4 xc = reload(i);
-            const uint32_t xw[4] = {xc.x, xc.y, xc.z, xc.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const double lo = __uint_as_float(xw[k] << 16), hi = __uint_as_float(xw[k] & 0xFFFF0000u);
-              a0 = __fma_rn(lo, lo, a0);
-              a1 = __fma_rn(hi, hi, a1);
-            }
-          }
-          const double ss = team_reduce(a0 + a1, SumOp(), red_d, tid, T, bar_id);
-          float r_lo, r_hi;
-          rms_bracket(__fma_rn(ss, 1.0 / static_cast<double>(p.L), static_cast<double>(p.eps)), r_lo, r_hi);
-          const uint64_t rlo2 = dup2(r_lo), rhi2 = dup2(r_hi);
-#pragma unroll
-          for (int i = 0; i < CH; ++i) {
-            if ((cand >> i) & 1u) {
-              const uint4 xc = reload(i);
-              const uint4 wv = __ldg(reinterpret_cast<const uint4*>(p.w + off(i)));
-              uint32_t d = 0;
-              y[i].x = bf2_mul(rms_n_pair(xc.x, rlo2, rhi2, d), wv.x);
-              y[i].y = bf2_mul(rms_n_pair(xc.y, rlo2, rhi2, d), wv.y);
-              y[i].z = bf2_mul(rms_n_pair(xc.z, rlo2, rhi2, d), wv.z);
-              y[i].w = bf2_mul(rms_n_pair(xc.w, rlo2, rhi2, d), wv.w);
-              if (d != 0) y[i] = rms_chunk_fix(xc, wv, y[i], rlo2, rhi2, ss, p.L, p.eps);
-            }
-          }
-        }
-      }
     }
   }
   if constexpr (FAST && OP == OP_SILU) {
@@ -789,7 +671,7 @@ fp8q_status launch_staged(const QuantParams& p, int T, int nbuf, int stride, cud
 constexpr int kGroupThreads = 256;
 constexpr int kGroupItems = 4;
 
-template <int OP, bool FAST>
+template <int OP>
 __global__ void __launch_bounds__(kGroupThreads) quant_groups_kernel(const QuantParams p) {
   constexpr int TEAMS = kGroupThreads / 16;
   const int t = threadIdx.x & 15;
@@ -823,7 +705,7 @@ __global__ void __launch_bounds__(kGroupThreads) quant_groups_kernel(const Quant
 #pragma unroll
     for (int u = 0; u < kGroupItems; ++u) {
       uint4 y;
-      auto exact_chunk = [&]() {
+      if constexpr (OP == OP_SILU) {
         uint32_t d = 0;
         bool bad = false;
         y.x = silu_pair(a[u].x, b[u].x, d, bad);
@@ -831,30 +713,12 @@ __global__ void __launch_bounds__(kGroupThreads) quant_groups_kernel(const Quant
         y.z = silu_pair(a[u].z, b[u].z, d, bad);
         y.w = silu_pair(a[u].w, b[u].w, d, bad);
         if (d != 0 || bad) y = silu_chunk_fix(a[u], b[u], y);   // rare: exact recomputation
-      };
-      if constexpr (OP == OP_SILU) {
-        if (FAST && chunk_min_gate(a[u]) >= -85.0f) {
-          y.x = silu_pair_fast(a[u].x, b[u].x);
-          y.y = silu_pair_fast(a[u].y, b[u].y);
-          y.z = silu_pair_fast(a[u].z, b[u].z);
-          y.w = silu_pair_fast(a[u].w, b[u].w);
-        } else {
-          exact_chunk();
-        }
       } else {
         y = a[u];
       }
       float am = absmax2_to_f32(chunk_absmax2(y, 0u));
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
-      if constexpr (FAST && OP == OP_SILU) {
-        // the chunks that can decide the group's amax, exactly; amax again
-        const float mine = absmax2_to_f32(chunk_absmax2(y, 0u));
-        if (mine >= bf16_steps_below(am, kCandSteps)) exact_chunk();
-        am = absmax2_to_f32(chunk_absmax2(y, 0u));
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
-      }
       const QScale qs = make_qscale(am, p.ue8m0, p.i8);
       if (ok[u]) {
         *reinterpret_cast<uint2*>(p.q + row[u] * p.ldq + col[u]) = codes_chunk(p, y, qs);
@@ -885,7 +749,7 @@ fp8q_status launch_quant_mode(const QuantParams& p, cudaStream_t stream) {
       int64_t blocks = (items + per_block - 1) / per_block;
       const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
       if (blocks > cap) blocks = cap;
-      return launch_kernel(quant_groups_kernel<OP, FAST>, dim3(static_cast<unsigned>(blocks)),
+      return launch_kernel(quant_groups_kernel<OP>, dim3(static_cast<unsigned>(blocks)),
                            dim3(kGroupThreads), 0, stream, 1, p);
     }
   }
@@ -914,13 +778,16 @@ fp8q_status launch_quant_mode(const QuantParams& p, cudaStream_t stream) {
   return per_token ? go(quant_rows_kernel<OP, true, 4, 512, 2, FAST>) : go(quant_rows_kernel<OP, false, 4, 512, 2, FAST>);
 }
 
-// The fused ops (RMSNorm, SiLU*mul) run their fast y unless the exact mode is
-// set (fp8q_set_fused_quant_exact); the plain quant is always exact.
+// SiLU*mul per token runs its fast y unless the exact mode is set
+// (fp8q_set_fused_quant_exact).  Everything else is exact in both modes: the
+// plain quant by definition; RMSNorm (row kernels, ring), residual add +
+// RMSNorm and the 1x128 SiLU*mul kernel measured no faster with the fast
+// arithmetic (their time goes to row latency and to the extra amax pass).
 std::atomic<int> g_fused_exact{0};
 
 template <int OP>
 fp8q_status launch_quant(const QuantParams& p, cudaStream_t stream) {
-  if constexpr (OP == OP_PLAIN) {
+  if constexpr (OP != OP_SILU) {
     return launch_quant_mode<OP, false>(p, stream);
   } else {
     return g_fused_exact.load(std::memory_order_relaxed) ? launch_quant_mode<OP, false>(p, stream)

@@ -364,16 +364,12 @@ __device__ __noinline__ uint4 silu_chunk_fix(const uint4 g, const uint4 u, uint4
 }
 
 // ---------------------------------------------------------------------------
-// Fast y (the fused ops' default mode).  y comes within one bf16 step of its
-// definition (differing only when the real value lies closer to a bf16
-// rounding midpoint than the fast value's error); the quant kernels recompute
-// exactly the elements that can decide a group's amax, so scales stay exact
-// and codes (from the exact IEEE quotient of y) differ only where y does.
-
-// bf16(x rf) of a pair, rf = fl32(r): one product, one rounding.
-__device__ __forceinline__ uint32_t rms_n_pair_fast(uint32_t xw, uint64_t rf2) {
-  return f2_to_bf2_rn(mul2(bf2_to_f2(xw), rf2));
-}
+// Fast y (SiLU*mul per token, the default mode).  y comes within one bf16
+// step of its definition (differing only when the real value lies closer to a
+// bf16 rounding midpoint than the fast value's error); the quant kernels
+// recompute exactly the elements that can decide a group's amax, so scales
+// stay exact and codes (from the exact IEEE quotient of y) differ only where
+// y does.
 
 // Fast bf16(silu(g) u) of a pair: (g u) / (1 + 2^(-g log2 e)) with ex2.approx
 // and rcp.approx.  For gates >= -85: the product g u is exact unless it

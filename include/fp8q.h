@@ -138,19 +138,21 @@ FP8Q_API fp8q_status fp8q_add_rmsnorm_quant(const void* x, void* residual, const
                                             void* stream);
 
 /*
- * fp8q_set_fused_quant_exact -- arithmetic of the producer-fused quant ops
- * (fp8q_rmsnorm_quant, fp8q_add_rmsnorm_quant, fp8q_silu_mul_quant and the
- * int8 forms of the first and last), whose tolerance the pages' workload
- * fixes at >= 99.9% of codes identical to the definition, the rest within one
- * step, scales within 1e-5 relative ("Helion in vLLM", "Per-kernel
- * performance": the fused ops are measured against the unfused chain).
- *   exact = 0 (default): y from fp32 arithmetic (fp32 sum of squares,
- *     ex2/rcp approximations), within two bf16 steps of its definition and
- *     equal to it except next to a bf16 rounding midpoint; the elements that
- *     can decide a group's amax are recomputed exactly, so every scale is
- *     bit-exact; codes are the exact e4m3 (or int8) of fl32(y / s).
+ * fp8q_set_fused_quant_exact -- arithmetic of the producer-fused quant ops,
+ * whose tolerance the pages' workload fixes at >= 99.9% of codes identical to
+ * the definition, the rest within one step, scales within 1e-5 relative
+ * ("Helion in vLLM", "Per-kernel performance": the fused ops are measured
+ * against the unfused chain).
+ *   exact = 0 (default): fp8q_silu_mul_quant and fp8q_silu_mul_quant_i8 with
+ *     per-token scales compute y with fp32 ex2/rcp approximations, within one
+ *     bf16 step of its definition and equal to it except next to a bf16
+ *     rounding midpoint; the elements that can decide the row's amax are
+ *     recomputed exactly, so every scale is bit-exact, and codes are the exact
+ *     e4m3 (or int8) codes of fl32(y / s).  All other fused ops (RMSNorm,
+ *     residual add + RMSNorm, 1x128 SiLU*mul) are bit-exact in this mode too:
+ *     a fast arithmetic measured no faster for them.
  *   exact = 1: every y is the correctly rounded value of its definition, so
- *     codes and scales are bit-exact (about twice the arithmetic).
+ *     codes and scales of every fused op are bit-exact.
  * Process-wide; applies to calls made after it returns (captured CUDA graphs
  * keep the kernels they captured).  Other values: FP8Q_ERR_INVALID_ARG.
  * fp8q_get_fused_quant_exact returns the current setting.
