@@ -1213,6 +1213,124 @@ __global__ void __launch_bounds__(Cfg2<BN, BW>::THREADS, 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
 }
 
+// ------------------------------------------------------------------ decode (M <= 8)
+// At M <= 8 tokens a linear layer is bound by reading its weights once from
+// HBM (N K bytes; 52 MB for the Qwen3-32B qkv projection) and does only 2 M
+// flops per weight byte, so this kernel streams the weights with 16-byte
+// loads straight into the registers of the warp-level MMA
+// (mma.sync.m16n8k32, e4m3 x e4m3 -> f32: the weight rows in its 16-row slot,
+// the tokens in its 8 columns, absent tokens as zeros).  There is no TMEM
+// allocation, no tensor-map setup and no split-K round trip through global
+// memory: a CTA owns 16 weight rows, its kDecodeWarps warps split K, and their
+// partial sums meet once in shared memory.
+// K order inside a 64-deep chunk: lane (g, t) = (lane / 4, lane % 4) loads the
+// 16 contiguous bytes [16 t, 16 t + 16) of weight rows g and g + 8 and of token
+// g; bytes 0-7 feed the chunk's first MMA and 8-15 its second.  The MMA's own
+// k order inside an instruction differs, but every product a[m][k] b[n][k] of
+// the chunk is formed exactly once, and a chunk never straddles a 128-deep
+// block, so the blockwise scales apply to the right sums.
+// Scales as in the tcgen05 kernels: blockwise, each K block's fp32 partial
+// times sa[m, kb] sb[n / 128, kb] into the fp32 total; per token, the total
+// times sa[m] sb[n] at the end.
+constexpr int kDecodeWarps = 8;
+constexpr int kDecodeRows = 16;
+constexpr int kDecodeMaxM = 8;
+
+__device__ __forceinline__ void mma_e4m3_m16n8k32(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
+                                                  uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 ld_weight(const uint8_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+template <bool BW>
+__global__ void __launch_bounds__(32 * kDecodeWarps) decode_kernel(const uint8_t* __restrict__ a,
+                                                                   const uint8_t* __restrict__ b,
+                                                                   const GemmArgs p) {
+  __shared__ float red[kDecodeWarps][kDecodeRows][kDecodeMaxM];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int n0 = static_cast<int>(blockIdx.x) * kDecodeRows;
+  const int kblocks = p.K / BK;
+  const int kb0 = (kblocks * warp) / kDecodeWarps, kb1 = (kblocks * (warp + 1)) / kDecodeWarps;
+  const uint8_t* w0 = b + static_cast<int64_t>(n0 + g) * p.K + 16 * t;
+  const uint8_t* w1 = w0 + 8LL * p.K;
+  const bool tok = g < p.M;
+  const uint8_t* ar = a + static_cast<int64_t>(tok ? g : 0) * p.K + 16 * t;
+  griddep_wait();                       // activations and scales may come from the previous kernel
+  griddep_launch_dependents();
+  // one K block = two 64-deep chunks
+  auto load = [&](int kb, uint4* wa, uint4* wb, uint4* av) {
+    const int64_t k0 = static_cast<int64_t>(kb) * BK;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      wa[c] = ld_weight(w0 + k0 + 64 * c);
+      wb[c] = ld_weight(w1 + k0 + 64 * c);
+      av[c] = tok ? __ldg(reinterpret_cast<const uint4*>(ar + k0 + 64 * c)) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  auto compute = [&](int kb, const uint4* wa, const uint4* wb, const uint4* av) {
+    float cc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float* d = BW ? cc : acc;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      mma_e4m3_m16n8k32(d, wa[c].x, wb[c].x, wa[c].y, wb[c].y, av[c].x, av[c].y);
+      mma_e4m3_m16n8k32(d, wa[c].z, wb[c].z, wa[c].w, wb[c].w, av[c].z, av[c].w);
+    }
+    if constexpr (BW) {
+      // C fragment: cc[0], cc[1] = rows g, tokens 2t, 2t+1; cc[2], cc[3] = row g + 8
+      const float sbk = __ldg(p.sb + (n0 / 128) * p.sb_snb + kb * p.sb_skb);
+      const float s0 = 2 * t < p.M ? __ldg(p.sa + (2 * t) * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
+      const float s1 = 2 * t + 1 < p.M ? __ldg(p.sa + (2 * t + 1) * p.sa_sm + kb * p.sa_skb) * sbk : 0.0f;
+      acc[0] = fmaf(cc[0], s0, acc[0]);
+      acc[1] = fmaf(cc[1], s1, acc[1]);
+      acc[2] = fmaf(cc[2], s0, acc[2]);
+      acc[3] = fmaf(cc[3], s1, acc[3]);
+    }
+  };
+  // a ring of three K blocks in registers: block kb + 3's loads are issued as
+  // soon as block kb's MMAs have read their operands
+  uint4 a0[2], b0[2], v0[2], a1[2], b1[2], v1[2], a2[2], b2[2], v2[2];
+  if (kb0 < kb1) load(kb0, a0, b0, v0);
+  if (kb0 + 1 < kb1) load(kb0 + 1, a1, b1, v1);
+  if (kb0 + 2 < kb1) load(kb0 + 2, a2, b2, v2);
+  for (int kb = kb0; kb < kb1; kb += 3) {
+    compute(kb, a0, b0, v0);
+    if (kb + 3 < kb1) load(kb + 3, a0, b0, v0);
+    if (kb + 1 < kb1) compute(kb + 1, a1, b1, v1);
+    if (kb + 4 < kb1) load(kb + 4, a1, b1, v1);
+    if (kb + 2 < kb1) compute(kb + 2, a2, b2, v2);
+    if (kb + 5 < kb1) load(kb + 5, a2, b2, v2);
+  }
+  red[warp][g][2 * t] = acc[0];
+  red[warp][g][2 * t + 1] = acc[1];
+  red[warp][g + 8][2 * t] = acc[2];
+  red[warp][g + 8][2 * t + 1] = acc[3];
+  __syncthreads();
+  // the warps' partials in warp order; one thread per (row, token)
+  if (threadIdx.x < kDecodeRows * kDecodeMaxM) {
+    const int r = threadIdx.x / kDecodeMaxM, m = threadIdx.x % kDecodeMaxM;
+    if (m < p.M) {
+      float v = red[0][r][m];
+#pragma unroll
+      for (int w = 1; w < kDecodeWarps; ++w) v += red[w][r][m];
+      if constexpr (!BW) v *= __ldg(p.sa + m * p.sa_sm) * __ldg(p.sb + (n0 + r) * p.sb_sn);
+      p.y[static_cast<int64_t>(m) * p.ldy + n0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    }
+  }
+}
+
 // ------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -1371,6 +1489,8 @@ fp8q_gemm_variant g_force{0, 1, 128, 0};
 // block scales (block-scaled MMA).
 bool variant_supported(const fp8q_gemm_variant& v, int blockwise) {
   if (v.cta_pair != 0 && v.cta_pair != 1) return false;
+  // warp-MMA weight streaming for M <= 8 (fp32 scales, per token or blockwise)
+  if (v.block_n == kDecodeMaxM) return blockwise <= 1 && v.swap_ab == 1 && v.split_k == 1 && !v.cta_pair;
   if (blockwise == 3) blockwise = 0;   // int8: the per-token scheme's variants
   if (blockwise == 2) {
     // single CTAs only; 224-column tiles leave TMEM room for the scale factors
@@ -1428,6 +1548,15 @@ bool tuned_variant(int64_t M, int64_t N, int64_t K, int blockwise, fp8q_gemm_var
 fp8q_gemm_variant heuristic_variant(int64_t M, int64_t N, int64_t K, int blockwise) {
   fp8q_gemm_variant v;
   v.cta_pair = 0;
+  // M <= 8: the warp-MMA weight streaming kernel, measured fastest on every
+  // table shape with K <= 12288 (the longer K of a 25600-deep layer leaves its
+  // warps too few loads in flight; there Swap-AB tiles stay faster)
+  if (blockwise <= 1 && M <= kDecodeMaxM && K % BK == 0 && N % kDecodeRows == 0 && K <= 16384) {
+    v.swap_ab = 1;
+    v.split_k = 1;
+    v.block_n = kDecodeMaxM;
+    return v;
+  }
   if (M <= 128) {
     // Swap-AB: the weight rows fill the 128-row MMA slot, the tokens its N.
     v.swap_ab = 1;
@@ -1550,6 +1679,14 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int blockwise, const fp8q_gemm_v
   return pl;
 }
 
+template <bool BW>
+fp8q_status launch_decode(const void* a_q, const void* b_q, const GemmArgs& p, cudaStream_t stream) {
+  if (p.M > kDecodeMaxM || p.K % BK != 0 || p.N % kDecodeRows != 0) return FP8Q_ERR_UNSUPPORTED;
+  return launch_kernel(decode_kernel<BW>, dim3(static_cast<unsigned>(p.N / kDecodeRows)),
+                       dim3(32 * kDecodeWarps), 0, stream, 1, static_cast<const uint8_t*>(a_q),
+                       static_cast<const uint8_t*>(b_q), p);
+}
+
 template <bool BW, bool MX = false, bool I8 = false>
 fp8q_status run_gemm(const void* a_q, const void* b_q, GemmArgs& p, const Plan& pl, void* ws,
                      cudaStream_t stream) {
@@ -1567,6 +1704,10 @@ fp8q_status run_gemm(const void* a_q, const void* b_q, GemmArgs& p, const Plan& 
   p.ws = pl.max_contrib > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.counter_bytes) : nullptr;
   p.status = device_status_ptr();
   const int bn = pl.v.block_n;
+  if (bn == kDecodeMaxM) {
+    if constexpr (MX || I8) return FP8Q_ERR_UNSUPPORTED;
+    else return launch_decode<BW>(a_q, b_q, p, stream);
+  }
   if constexpr (MX) {
     if (pl.v.cta_pair) return FP8Q_ERR_UNSUPPORTED;
     if (pl.v.swap_ab) {

@@ -25,6 +25,7 @@ import argparse
 import datetime
 import json
 import os
+import re
 import statistics
 
 import torch
@@ -43,7 +44,8 @@ SHAPES = [
     ("qwen3-32b gate_up", 5120, 51200), ("qwen3-32b down", 25600, 5120),
     ("square 2048", 2048, 2048),
 ]
-M_BUCKETS = [1, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192]
+M_BUCKETS = [1, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192]
+DECODE_MAX_M = 8
 TIE = 1.02
 
 
@@ -76,6 +78,8 @@ def candidates(M: int, N: int, K: int, sms: int, blockwise: bool) -> list[tuple[
     """(swap_ab, split_k, block_n, cta_pair) variants worth timing for this shape."""
     kb = K // 128
     out = []
+    if M <= DECODE_MAX_M and K % 128 == 0 and N % 16 == 0:
+        out.append((1, 1, 8, 0))            # warp-MMA weight streaming
     if M <= 128:
         bn = next(b for b in (16, 32, 64, 128) if b >= M)
         for b in sorted({bn, min(128, 2 * bn)}):
@@ -164,6 +168,27 @@ def tune(reps: int = 5, shapes=SHAPES, buckets=M_BUCKETS, log=print):
     return rows
 
 
+_ROW = re.compile(r"^\{(\d+), (\d+), (\d+), (\d+), (\d+), (\d+), (\d+), (\d+)\},\s*// (.*?): ([0-9.]+) us$")
+
+
+def merge_rows(rows, path: str):
+    """The table at `path` with the measured rows replacing (or joining) those of
+    the same (scheme, m_max, N, K); returns row dicts in shape, scheme, M order."""
+    have = {}
+    with open(path) as f:
+        for line in f:
+            m = _ROW.match(line.strip())
+            if m:
+                v = [int(x) for x in m.groups()[:8]]
+                have[(v[0], v[1], v[2], v[3])] = {"shape": m.group(9), "blockwise": v[0], "m_max": v[1],
+                                                  "N": v[2], "K": v[3], "variant": v[4:8],
+                                                  "us": float(m.group(10))}
+    for r in rows:
+        have[(r["blockwise"], r["m_max"], r["N"], r["K"])] = r
+    order = {name: i for i, (name, _, _) in enumerate(SHAPES)}
+    return sorted(have.values(), key=lambda r: (order.get(r["shape"], 99), r["m_max"], r["blockwise"]))
+
+
 def write_table(rows, path: str, device: str | None = None) -> None:
     dev = device or torch.cuda.get_device_name()
     with open(path, "w") as f:
@@ -182,6 +207,9 @@ def main():
     ap.add_argument("--out", default=os.path.join(HERE, "csrc", "fp8q_variant_table.inc"))
     ap.add_argument("--json", default=None, help="also write every timing as JSON lines")
     ap.add_argument("--reps", type=int, default=5, help="trials per variant")
+    ap.add_argument("--buckets", default=None,
+                    help="comma-separated M buckets to measure (default: all); the measured rows "
+                         "replace those of the same buckets in the existing table, the others stay")
     args = ap.parse_args()
     jf = open(args.json, "w") if args.json else None
 
@@ -191,7 +219,11 @@ def main():
             jf.write(line + "\n")
             jf.flush()
 
-    rows = tune(args.reps, log=log)
+    if args.buckets:
+        rows = tune(args.reps, buckets=[int(b) for b in args.buckets.split(",")], log=log)
+        rows = merge_rows(rows, args.out)
+    else:
+        rows = tune(args.reps, log=log)
     write_table(rows, args.out)
     if jf:
         jf.close()

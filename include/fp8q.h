@@ -421,9 +421,13 @@ FP8Q_API fp8q_status fp8q_select_gemm_variant(int64_t M, int64_t N, int64_t K, i
 /* Force a variant for every following GEMM call in this process (testing and
  * tuning only; not thread-safe).  NULL restores automatic selection.  Returns
  * FP8Q_ERR_INVALID_ARG if the variant is malformed (block_n not one of
- * 16, 32, 64, 128, 224, 256; split_k < 0 or > 64; cta_pair not 0 or 1, or
+ * 8, 16, 32, 64, 128, 224, 256; split_k < 0 or > 64; cta_pair not 0 or 1, or
  * set with another combination than the one above).  A GEMM call whose
- * scheme cannot run the forced variant returns FP8Q_ERR_UNSUPPORTED. */
+ * scheme cannot run the forced variant returns FP8Q_ERR_UNSUPPORTED.
+ * {swap_ab 1, split_k 1, block_n 8, cta_pair 0} is the decode variant: the
+ * weights streamed through the warp-level MMA (mma.sync m16n8k32 e4m3) for
+ * M <= 8 tokens, K a multiple of 128, per-token/per-channel or blockwise fp32
+ * scales; no workspace. */
 FP8Q_API fp8q_status fp8q_force_gemm_variant(const fp8q_gemm_variant* v);
 
 /* ------------------------------------------------------------------------ */

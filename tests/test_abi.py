@@ -156,11 +156,16 @@ def test_variant_table_lookup():
 
 
 def test_variant_selection_host_logic():
-    # shapes outside the table: Swap-AB with tokens padded to 16/32/64/128 for
-    # small M, no swap for large M
+    # shapes outside the table: the warp-MMA decode variant for M <= 8 (K up to
+    # 16384), Swap-AB with tokens padded to 16/32/64/128 for other small M, no
+    # swap for large M
     N, K = 3072, 2560
-    assert fq.fp8q_select_gemm_variant(1, N, K, True)["swap_ab"] == 1
-    assert fq.fp8q_select_gemm_variant(1, N, K, True)["block_n"] == 16
+    for M in (1, 5, 8):
+        assert fq.fp8q_select_gemm_variant(M, N, K, True) == \
+            {"swap_ab": 1, "split_k": 1, "block_n": 8, "cta_pair": 0}
+        assert fq.fp8q_select_gemm_variant(M, N, K, False)["block_n"] == 8
+    assert fq.fp8q_select_gemm_variant(1, N, 32768, True)["block_n"] == 16
+    assert fq.fp8q_select_gemm_variant(9, N, K, True)["block_n"] == 16
     assert fq.fp8q_select_gemm_variant(33, N, K, True)["block_n"] == 64
     assert fq.fp8q_select_gemm_variant(100, N, K, False)["block_n"] == 128
     v = fq.fp8q_select_gemm_variant(8192, N, K, True)

@@ -31,10 +31,12 @@ def test_every_candidate_is_accepted_by_the_library():
 
 
 def test_candidate_sets_follow_the_shape():
-    # decode: Swap-AB with the token count padded to 16, split-K / stream-K
-    # because 48 weight tiles do not fill the SMs
+    # decode: the warp-MMA weight-streaming variant, and Swap-AB with the token
+    # count padded to 16, split-K / stream-K because 48 weight tiles do not
+    # fill the SMs
     c = tune.candidates(1, 6144, 4096, SMS, True)
-    assert all(v[0] == 1 for v in c) and {v[2] for v in c} == {16, 32}
+    assert (1, 1, 8, 0) in c and (1, 1, 8, 0) not in tune.candidates(9, 6144, 4096, SMS, True)
+    assert all(v[0] == 1 for v in c) and {v[2] for v in c} == {8, 16, 32}
     assert {v[1] for v in c} >= {1, 0, 2, 3}
     assert all(v[3] == 0 for v in c)
     # large M: no swap, whole-K tiles only once they fill the SMs, pairs for
