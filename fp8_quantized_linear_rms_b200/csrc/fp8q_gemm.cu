@@ -117,13 +117,15 @@ struct Cfg {
   static_assert(!(BW && MX) && !(I8 && (BW || MX)), "one scale scheme");
   static constexpr int B_BYTES = BN * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;           // TMA bytes per stage
-  // Scale factors (MX): per pipeline stage a TMEM slot of 4 columns for the
-  // 128 MMA rows and 4 per 128 MMA columns, written by SF_WARPS warps (one
-  // per TMEM lane quadrant) with tcgen05.st.
+  // Scale factors (MX): per pipeline stage a shared-memory slot of 512 bytes
+  // for the 128 MMA rows and 512 per 128 MMA columns, written by the SF warp,
+  // and a TMEM slot of 4 + 4 per 128 columns, filled from it by the MMA
+  // thread with tcgen05.cp.
   static constexpr int SFB_CHUNKS = (BN + 127) / 128;
   static constexpr int SF_COLS = 4 * (1 + SFB_CHUNKS);
-  static constexpr int SF_WARPS = MX ? 4 : 0;
-  static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
+  static constexpr int SF_BYTES = MX ? 512 * (1 + SFB_CHUNKS) : 0;
+  static constexpr int SF_WARPS = MX ? 1 : 0;
+  static constexpr int STAGES_RAW = kSmemBudget / (STAGE_BYTES + SF_BYTES);
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int EPI_WARPS = (BW && BN >= 128) ? 8 : 4;
   static constexpr int COL_GROUPS = EPI_WARPS / 4;        // column slices per TMEM lane quadrant
@@ -146,7 +148,7 @@ struct Cfg {
   static constexpr int EPI_BASE = REGSPLIT ? 0 : 2;             // first epilogue warp
   static constexpr int THREADS = REGSPLIT ? 384 : 64 + 32 * (EPI_WARPS + SF_WARPS);
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * NBUF + 1) + 16;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * (STAGE_BYTES + SF_BYTES) + BAR_BYTES;
   static_assert(STAGES >= 2, "pipeline too shallow");
   static_assert(TMEM_NEED <= 512, "accumulators exceed TMEM");
   static_assert(CPT % CHUNK == 0 && (CHUNK == 8 || CHUNK == 16 || CHUNK == 32), "chunking");
@@ -262,7 +264,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * C::B_BYTES);
+  uint8_t* sSF = sB + S * C::B_BYTES;            // MX: per-stage scale-factor slots
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSF + S * C::SF_BYTES);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + NB;
@@ -274,7 +277,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
-      mbar_init(&full[i], 1 + C::SF_WARPS);     // TMA bytes (+ the SF warps' stores)
+      mbar_init(&full[i], 1 + C::SF_WARPS);     // TMA bytes (+ the SF warp's slot)
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < NB; ++i) {
@@ -371,9 +374,14 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
           const uint64_t adesc = smem_desc_kmajor_sw128(sA + st * A_BYTES);
           const uint64_t bdesc = smem_desc_kmajor_sw128(sB + st * C::B_BYTES);
           if constexpr (MX) {
-            // the four block-scaled MMAs of the stage, with the scale
-            // factors the SF warps stored in the stage's TMEM slot
+            // the stage's scale factors from its shared-memory slot into its
+            // TMEM slot, then the four block-scaled MMAs of the stage (a
+            // thread's tcgen05 operations run in issue order)
             const uint32_t sf = tmem_base + C::SF_COL0 + st * C::SF_COLS;
+            const uint8_t* ssf = sSF + st * C::SF_BYTES;
+            tmem_cp_sf_chunk(sf, ssf);
+#pragma unroll
+            for (int h = 0; h < C::SFB_CHUNKS; ++h) tmem_cp_sf_chunk(sf + 4 + 4 * h, ssf + 512 * (1 + h));
 #pragma unroll
             for (int k = 0; k < BK / UMMA_K; ++k) {
               const uint32_t acc = (kb > kb0 || k > 0);
@@ -409,13 +417,17 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
   };
   auto role_sf = [&]() {
     // ------------------------------------------------------------ scale factors (MX)
-    // Four warps, one per TMEM lane quadrant.  For every stage each writes
-    // the E8M0 scale factors into its quadrant of the stage's TMEM slot --
-    // lane l, column c of the SFA chunk: MMA row 32 c + l; of SFB chunk h:
-    // MMA column 128 h + 32 c + l; each byte repeated over the stage's four
-    // 32-deep K slices -- waits for its stores and arrives on the stage's
-    // full barrier.  A slot is rewritten only after the empty barrier of its
-    // stage, so the MMAs that read it have completed.  Rows or columns
+    // One warp (on a sub-partition other than the MMA and producer warps').
+    // For every stage it writes the E8M0 scale factors into the stage's
+    // shared-memory slot -- row l of the SFA chunk: MMA rows l, l+32, l+64,
+    // l+96; of SFB chunk h: MMA columns 128 h + l + 32 j; each byte repeated
+    // over the stage's four 32-deep K slices -- and arrives on the stage's
+    // full barrier; the MMA thread copies the slot into TMEM (tcgen05.cp)
+    // right before the stage's MMAs.  (Factors stored into TMEM directly by
+    // four warps, one per lane quadrant, were slower: the warp sharing a
+    // sub-partition with the MMA thread fell ~3 stages behind.)  A slot is
+    // rewritten only after the empty barrier of its stage, so the copies and
+    // MMAs that read it have completed.  Rows or columns
     // outside the problem take the scale 1 (byte 127): their operands are
     // zero-filled by TMA.  The scale bytes of a stage are loaded SFD stages
     // ahead (a register ring) so their global latency stays off the path:
@@ -427,7 +439,6 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
     constexpr int SFD = 4;
     constexpr int NRAW = SWAP ? 1 + 4 * C::SFB_CHUNKS : 7;
     constexpr uint32_t kOneByte = 127u;
-    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int nb_rows = p.N >> 7;                    // weight block rows
     uint32_t raw[SFD][NRAW];
     SegIter sai(p);
@@ -519,14 +530,15 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
         int w_ok = 1;
         if (lane == 0) w_ok = mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status);
         if (!__shfl_sync(0xFFFFFFFFu, w_ok, 0)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sfa = tmem_base + lane_addr + C::SF_COL0 + st * C::SF_COLS;
-        tmem_st_32x32b_x4(sfa, wa[0], wa[1], wa[2], wa[3]);
+        // row `lane` of each 512-byte chunk: the factors of MMA rows (or
+        // columns) lane, lane + 32, lane + 64, lane + 96
+        uint32_t* sf = reinterpret_cast<uint32_t*>(sSF + st * C::SF_BYTES);
+        *reinterpret_cast<uint4*>(sf + lane * 4) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
 #pragma unroll
         for (int h = 0; h < C::SFB_CHUNKS; ++h)
-          tmem_st_32x32b_x4(sfa + 4 + 4 * h, wb[h][0], wb[h][1], wb[h][2], wb[h][3]);
-        tmem_st_wait();
-        tc_fence_before();
+          *reinterpret_cast<uint4*>(sf + 128 * (1 + h) + lane * 4) =
+              make_uint4(wb[h][0], wb[h][1], wb[h][2], wb[h][3]);
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[st]);
       }
@@ -1545,13 +1557,15 @@ bool tuned_variant(int64_t M, int64_t N, int64_t K, int blockwise, fp8q_gemm_var
 }
 
 // Shapes outside the table: rules drawn from the same measurements.
-fp8q_gemm_variant heuristic_variant(int64_t M, int64_t N, int64_t K, int blockwise) {
+fp8q_gemm_variant heuristic_variant(int64_t M, int64_t N, int64_t K, int blockwise,
+                                    bool allow_decode = true) {
   fp8q_gemm_variant v;
   v.cta_pair = 0;
   // M <= 8: the warp-MMA weight streaming kernel, measured fastest on every
   // table shape with K <= 12288 (the longer K of a 25600-deep layer leaves its
   // warps too few loads in flight; there Swap-AB tiles stay faster)
-  if (blockwise <= 1 && M <= kDecodeMaxM && K % BK == 0 && N % kDecodeRows == 0 && K <= 16384) {
+  if (allow_decode && blockwise <= 1 && M <= kDecodeMaxM && K % BK == 0 && N % kDecodeRows == 0 &&
+      K <= 16384) {
     v.swap_ab = 1;
     v.split_k = 1;
     v.block_n = kDecodeMaxM;
@@ -1608,12 +1622,15 @@ fp8q_gemm_variant pick_variant(int64_t M, int64_t N, int64_t K, int blockwise,
     if (forced) *forced = g_forced;
     if (g_forced) return g_force;
   }
-  if (blockwise == 3) return auto_variant(M, N, K, 0);   // int8: same kernel structure
-  if (blockwise == 2) {
-    // The block-scaled MMA keeps the whole K loop in TMEM like the per-token
-    // kernel, so it follows the per-token scheme's measured choice, on
-    // single CTAs with 224-column tiles where that takes 256-column tiles.
+  if (blockwise >= 2) {
+    // int8 (3) and the block-scaled MMA (2) keep the whole K loop in TMEM like
+    // the per-token kernel, so they follow the per-token scheme's measured
+    // choice -- except its warp-MMA decode kernel (fp8 with fp32 scales only),
+    // for which they take the tcgen05 rule's Swap-AB tiles.
     fp8q_gemm_variant v = auto_variant(M, N, K, 0);
+    if (v.block_n == kDecodeMaxM) v = heuristic_variant(M, N, K, 0, false);
+    if (blockwise == 3) return v;
+    // E8M0: single CTAs, with 224-column tiles where that takes 256-column tiles
     if (v.cta_pair) v = fp8q_gemm_variant{0, 1, 224, 0};
     if (!v.swap_ab && v.block_n == 256) v.block_n = 224;
     return v;

@@ -418,6 +418,26 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Make generic-proxy writes to shared memory visible to the async proxy
+// (tcgen05.cp, TMA) before they are signalled.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// One 512-byte scale-factor chunk -- 32 rows of 16 bytes in shared memory,
+// row l holding the factors of MMA rows l, l+32, l+64, l+96 (4 bytes each) --
+// into TMEM columns [taddr, taddr + 4) of all four lane quadrants
+// (tcgen05.cp 32x128b.warpx4).  Source descriptor: K-major, no swizzle, the
+// four 8-row core matrices 128 bytes apart (stride byte offset), version 1.
+// A thread's tcgen05 operations run in issue order, so MMAs issued after the
+// copy by the same thread read the copied factors.
+__device__ __forceinline__ void tmem_cp_sf_chunk(uint32_t taddr, const void* src) {
+  const uint64_t desc = (static_cast<uint64_t>(smem_u32(src) & 0x3FFFF) >> 4) |
+                        (static_cast<uint64_t>(128 >> 4) << 32) | (1ull << 46);
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+               : "memory");
+}
+
 // Instruction descriptor, kind::mxf8f6f4 with block scaling: A and B e4m3
 // (bits 7-9, 10-12 = 0), K-major, N >> 3 at bits 17-22, scale format E8M0
 // (bit 23), M >> 4 at bits 24-28, scale factor ids of B (bits 4-5) and A

@@ -155,6 +155,17 @@ def test_variant_table_lookup():
             {"swap_ab": r[4], "split_k": r[5], "block_n": r[6], "cta_pair": r[7]}
 
 
+def test_int8_and_e8m0_never_take_the_decode_variant():
+    # the warp-MMA decode kernel serves fp8 with fp32 scales only; where the
+    # per-token table picks it, the int8 and E8M0 schemes take Swap-AB tiles
+    for M in (1, 2, 8):
+        for N, K in ((10240, 5120), (6144, 4096), (3072, 2560)):
+            assert fq.fp8q_select_gemm_variant(M, N, K, False)["block_n"] == 8
+            for scheme in (2, 3):
+                v = fq.fp8q_select_gemm_variant(M, N, K, scheme)
+                assert v["block_n"] in (16, 32, 64, 128) and v["swap_ab"] == 1, (M, N, K, scheme, v)
+
+
 def test_variant_selection_host_logic():
     # shapes outside the table: the warp-MMA decode variant for M <= 8 (K up to
     # 16384), Swap-AB with tokens padded to 16/32/64/128 for other small M, no
@@ -202,7 +213,7 @@ def test_e8m0_variant_selection_host_logic():
     for M, N, K in [(8192, 51200, 5120), (2048, 24576, 4096), (4096, 6144, 4096)]:
         v = fq.fp8q_select_gemm_variant(M, N, K, 2)
         assert v["cta_pair"] == 0 and v["swap_ab"] == 0 and v["block_n"] in (128, 224), v
-    for M in (1, 16, 32, 64):
+    for M in (16, 32, 64):
         v = fq.fp8q_select_gemm_variant(M, 10240, 5120, 2)
         pt = fq.fp8q_select_gemm_variant(M, 10240, 5120, False)
         assert v == pt, (M, v, pt)
