@@ -59,6 +59,7 @@ LAYERS = (("qkv", H, QKV), ("o", ATT, H), ("gate_up", H, 2 * I), ("down", I, H))
 DEFAULT_M = 8192
 METRIC = "FP8 quant+scaled_mm TFLOP/s (Qwen3-32B prefill linear stack, per-token + blockwise)"
 EPS = 1e-6
+NOMINAL_FP8_TFLOPS = 4500.0      # dense e4m3 tensor peak on the data sheet, for context beside `frac`
 
 
 def parse():
@@ -527,7 +528,8 @@ def run_native(args, rank, world, local_rank):
     if dkind == "gemm":
         roof = {"bound": "tensor", "kernel": dname, "achieved": round(dunits / davg / 1e12, 1),
                 "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(dunits / davg / 1e12 / peak, 4),
-                "peak_source": peak_src}
+                "peak_source": peak_src,
+                "frac_of_nominal_fp8": round(dunits / davg / 1e12 / NOMINAL_FP8_TFLOPS, 4)}
     else:
         roof = {"bound": "hbm", "kernel": dname, "achieved": round(dunits / davg / 1e9, 1),
                 "peak": round(hbm, 1), "unit": "GB/s", "frac": round(dunits / davg / 1e9 / hbm, 4),

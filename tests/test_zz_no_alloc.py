@@ -24,7 +24,7 @@ if torch.cuda.is_available():
     import fp8_quantized_linear_rms_b200 as fq   # fails loudly if libfp8q.so is missing
 
 
-@pytest.mark.parametrize("M,N,K", [(16, 5120, 25600), (1, 10240, 5120), (64, 4096, 12288)])
+@pytest.mark.parametrize("M,N,K", [(16, 5120, 25600), (8, 5120, 8192), (1, 5120, 25600), (64, 4096, 12288)])
 def test_noalloc_matches_workspace_entry_point(M, N, K):
     fq.fp8q_force_gemm_variant()
     v = fq.fp8q_select_gemm_variant(M, N, K, True)
