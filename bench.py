@@ -234,8 +234,10 @@ class ClockSampler:
             os.remove(self.path)
         if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        srt = sorted(self.samples)
+        return {"sm_mhz": statistics.median(srt), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": srt[0], "sm_mhz_p10": srt[len(srt) // 10],
+                "reasons": sorted(self.reasons), "samples": len(srt)}
 
 
 # ------------------------------------------------------------------ native arm

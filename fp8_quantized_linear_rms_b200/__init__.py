@@ -359,7 +359,10 @@ def fp8q_scaled_mm_blockwise_silu_quant(a_q: torch.Tensor, b_q: torch.Tensor, a_
                                         scale_layout: str = "row_major", stream=None):
     """gate_up blockwise GEMM with the SiLU*mul 1x128 quant fused into its epilogue.
     b_q [2I, K] and b_scale [2I/128, K/128] in the interleaved layout of
-    interleave_gate_up.  Returns (q e4m3 [M, I], scales [M, I/128] or [I/128, M])."""
+    interleave_gate_up.  Returns (q e4m3 [M, I], scales [M, I/128] or [I/128, M]).
+    Exact mode: bit-identical to fp8q_scaled_mm_blockwise followed by
+    fp8q_silu_mul_quant(h, 128); fast mode (default): the same scales, codes
+    within the fused-quant tolerance (fp8q_set_fused_quant_exact)."""
     for t, n in ((a_q, "a_q"), (b_q, "b_q")):
         _need(t, torch.float8_e4m3fn, n)
         if not t.is_contiguous():

@@ -106,6 +106,9 @@ struct GemmArgs {
   float* sq_s;
   int64_t sq_s_sm, sq_s_sg;
   int sq_ue8m0;
+  // 1: every SiLU*mul value exact; 0 (fast): an open pair is kept within one
+  // bf16 step of its value unless its chunk can decide the group amax
+  int sq_exact;
 };
 
 // MX: E8M0 block scales applied by the tensor core (kind::mxf8f6f4.block_scale);
@@ -253,10 +256,11 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
   using C = Cfg<BN, SWAP, BW, MX, I8>;
   static_assert(!SQ || (BW && !SWAP && BN == 256 && C::EPI_WARPS == 8 && 64 % C::CHUNK == 0),
                 "the fused SiLU*mul quant epilogue runs on 128x256 blockwise tiles");
-  // SQ: per-slice partial group amax, double-buffered by tile parity, and the
-  // mbarrier (one arrival per epilogue warp and tile) that orders the exchange
+  // SQ: per-slice partial group amax, double-buffered by tile parity, and one
+  // mbarrier per TMEM lane quadrant (one arrival from each of its two warps,
+  // which hold the two column slices of the same rows, per tile)
   __shared__ float sq_red[SQ ? 2 : 1][2][SQ ? BM : 1];
-  __shared__ uint64_t sq_bar;
+  __shared__ uint64_t sq_bar[SQ ? 4 : 1];
   constexpr int S = C::STAGES;
   constexpr int NB = C::NBUF;
   extern __shared__ uint8_t smem_raw[];
@@ -285,7 +289,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
       mbar_init(&tempty[i], C::EPI_WARPS);
     }
     mbar_init(drain, 1);
-    if (SQ) mbar_init(&sq_bar, C::EPI_WARPS);
+    if (SQ)
+      for (int i = 0; i < 4; ++i) mbar_init(&sq_bar[i], 2);   // the two warps of a TMEM lane quadrant
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -827,8 +832,18 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
         if constexpr (SQ) {
           // gate values in acc[0, 32), up values in acc[32, 64) (pairs);
           // h = bf16 of each, as the GEMM emits y; y = bf16(silu(h_gate) h_up)
-          uint4 yv[8];
-          uint32_t m2 = 0;
+          // Each pair's value is the bf16 rounding of the low end of its
+          // bracket.  A pair whose bracket straddles a rounding midpoint
+          // ("open") is within one bf16 step of its exact value; in the exact
+          // mode, and for tiny values or gates below -85 always, its chunk is
+          // recomputed exactly right away.  In the fast mode an open chunk is
+          // recomputed only if it can decide the group amax (within
+          // kCandSteps of this slice's amax: the slice's exact amax is then
+          // exact, and the partner slice's likewise), so scales stay exact
+          // and codes differ from the exact ones only where an open y does.
+          // (Open pairs are rare, ~1e-3 of the values, but an exact
+          // recomputation in a warp stalls the whole tile's epilogue.)
+          uint4 gv[8], uv[8];                          // h = bf16 of the sums, 8 chunks
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint32_t gw[4], uw[4];
@@ -840,6 +855,15 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
               gw[k] = pack_bf16x2(a0, a1);
               uw[k] = pack_bf16x2(b0, b1);
             }
+            gv[c] = make_uint4(gw[0], gw[1], gw[2], gw[3]);
+            uv[c] = make_uint4(uw[0], uw[1], uw[2], uw[3]);
+          }
+          uint4 yv[8];
+          uint32_t m2 = 0, open = 0;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t gw[4] = {gv[c].x, gv[c].y, gv[c].z, gv[c].w};
+            const uint32_t uw[4] = {uv[c].x, uv[c].y, uv[c].z, uv[c].w};
             uint32_t d = 0;
             bool bad = false;
             uint4 y;
@@ -847,22 +871,34 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
             y.y = silu_pair(gw[1], uw[1], d, bad);
             y.z = silu_pair(gw[2], uw[2], d, bad);
             y.w = silu_pair(gw[3], uw[3], d, bad);
-            if (d != 0 || bad)
-              y = silu_chunk_fix(make_uint4(gw[0], gw[1], gw[2], gw[3]), make_uint4(uw[0], uw[1], uw[2], uw[3]), y);
+            if (bad || (d != 0 && p.sq_exact))
+              y = silu_chunk_fix(gv[c], uv[c], y);
+            else
+              open |= static_cast<uint32_t>(d != 0) << c;
             yv[c] = y;
             m2 = chunk_absmax2(y, m2);
           }
+          if (open) {
+            const float thr = bf16_steps_below(absmax2_to_f32(m2), kCandSteps);
+            m2 = 0;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              if (((open >> c) & 1u) && absmax2_to_f32(chunk_absmax2(yv[c], 0u)) >= thr)
+                yv[c] = silu_chunk_fix(gv[c], uv[c], yv[c]);
+              m2 = chunk_absmax2(yv[c], m2);
+            }
+          }
           // group amax over the two column slices of the row: write this
-          // slice's partial, one arrival per warp, bounded wait for all 8
-          // warps of the tile, read the partner's.  The slot of tile t is
-          // written again at tile t + 2, after every warp has arrived for
-          // tile t + 1 and so has read it.
+          // slice's partial, one arrival per warp, bounded wait for the
+          // partner warp (same lane quadrant), read its partial.  The slot of
+          // tile t is written again at tile t + 2, after both warps have arrived for
+          // tile t + 1, so the partner has read it.
           float am = absmax2_to_f32(m2);
           const int par = sq_t & 1;
           sq_red[par][cg][row] = am;
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sq_bar);
-          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sq_bar, static_cast<uint32_t>(par), abort_flag, p.status))) {
+          if (lane == 0) mbar_arrive(&sq_bar[quad]);
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sq_bar[quad], static_cast<uint32_t>(par), abort_flag, p.status))) {
             ok = false;
             break;
           }
@@ -1987,6 +2023,7 @@ extern "C" fp8q_status fp8q_scaled_mm_blockwise_silu_quant(
   p.sq_s_sm = s_stride_m;
   p.sq_s_sg = s_stride_g;
   p.sq_ue8m0 = ue8m0;
+  p.sq_exact = fp8q_get_fused_quant_exact();
   p.tiles_a = pl.tiles_a;
   p.tiles_b = pl.tiles_b;
   p.kblocks = pl.kblocks;

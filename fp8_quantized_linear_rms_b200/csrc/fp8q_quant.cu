@@ -124,12 +124,6 @@ struct SmemRow {
   }
 };
 
-// Candidate margin of the fast SiLU*mul: a fast y lies within one bf16 step
-// of its definition, so the exact amax of a group is the exact value of an
-// element whose fast value is within one step of the fast amax, and no element
-// more than 4 steps below it can reach that (a margin of two steps to spare).
-constexpr uint32_t kCandSteps = 4;
-
 // Quantize one row with a team of T threads (T a multiple of 32, CH chunks
 // of 8 elements per thread; chunk c of the row belongs to thread c mod T, so
 // every warp access is 512 contiguous bytes).  `release()` is called once the

@@ -400,6 +400,12 @@ __device__ __forceinline__ float chunk_min_gate(const uint4& g) {
   return fminf(__low2float(m), __high2float(m));
 }
 
+// Candidate margin of the fast SiLU*mul: a fast y lies within one bf16 step
+// of its definition, so the exact amax of a group is the exact value of an
+// element whose fast value is within one step of the fast amax, and no element
+// more than 4 steps below it can reach that (a margin of two steps to spare).
+constexpr uint32_t kCandSteps = 4;
+
 // The bf16 magnitude `steps` below a (a bf16 value as fp32, >= 0; 0 stays 0):
 // consecutive bf16 magnitudes are consecutive integers.
 __device__ __forceinline__ float bf16_steps_below(float a, uint32_t steps) {

@@ -148,9 +148,14 @@ FP8Q_API fp8q_status fp8q_add_rmsnorm_quant(const void* x, void* residual, const
  *     bf16 step of its definition and equal to it except next to a bf16
  *     rounding midpoint; the elements that can decide the row's amax are
  *     recomputed exactly, so every scale is bit-exact, and codes are the exact
- *     e4m3 (or int8) codes of fl32(y / s).  All other fused ops (RMSNorm,
- *     residual add + RMSNorm, 1x128 SiLU*mul) are bit-exact in this mode too:
- *     a fast arithmetic measured no faster for them.
+ *     e4m3 (or int8) codes of fl32(y / s).  In the gate_up GEMM with the
+ *     fused SiLU*mul quant (fp8q_scaled_mm_blockwise_silu_quant) a y whose
+ *     rounding the fp32 bracket leaves open (about 1e-3 of the values) keeps
+ *     the lower bracket end, within one bf16 step, unless it can decide its
+ *     group's amax: scales stay bit-exact, codes differ only where such a y
+ *     does.  All other fused ops (RMSNorm, residual add + RMSNorm, the
+ *     standalone 1x128 SiLU*mul) are bit-exact in this mode too: a fast
+ *     arithmetic measured no faster for them.
  *   exact = 1: every y is the correctly rounded value of its definition, so
  *     codes and scales of every fused op are bit-exact.
  * Process-wide; applies to calls made after it returns (captured CUDA graphs
@@ -262,10 +267,13 @@ FP8Q_API fp8q_status fp8q_scaled_mm_blockwise(const void* a_q, const void* b_q, 
  * SiLU*mul quant fused into its epilogue: one of the fusions "on either side
  * of the path" that continue the pages' cut of the call count ("Helion in
  * vLLM", "Kernels integrated into vLLM": fused ops replace chains of calls).
- * Equal to, and bit-identical with,
+ * In the exact mode (fp8q_set_fused_quant_exact(1)) equal to, and
+ * bit-identical with,
  *   h = fp8q_scaled_mm_blockwise(a, W)          (bf16 [M, 2I] = [gate | up])
  *   q, scales = fp8q_silu_mul_quant(h, group_size = 128, ue8m0)
- * run with the same 128x256 whole-K GEMM variant, without ever writing h.
+ * run with the same 128x256 whole-K GEMM variant, without ever writing h; in
+ * the fast mode (the default) the scales are the same and the codes meet the
+ * fused-quant tolerance (see fp8q_set_fused_quant_exact).
  *
  *   b_q, b_scale  the gate_up weight [2I, K] and its [2I/128, K/128] block
  *            scales with the rows interleaved in 128-row blocks:
