@@ -61,6 +61,27 @@ METRIC = "FP8 quant+scaled_mm TFLOP/s (Qwen3-32B prefill linear stack, per-token
 EPS = 1e-6
 NOMINAL_FP8_TFLOPS = 4500.0      # dense e4m3 tensor peak on the data sheet, for context beside `frac`
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the step's dominant kernel, from one ncu capture of the full-size launch
+# (profiles/gemm_blockwise_silu_quant_qwen3_32b_gate_up.md gives the
+# command).  It holds for the GEMM sources it was taken on: the line reports
+# it only while their SHA-256 digest is unchanged, else null.
+GEMM_SOURCES = ("fp8q_gemm.cu", "fp8q_sm100.cuh", "fp8q_quant_math.cuh", "fp8q_common.cuh")
+TRAFFIC_CAPTURES = {
+    ("scaled_mm_blockwise_silu_quant", 8192): {
+        "read": 374152960, "write": 211215616,
+        "sources_sha256": "e7381c61eb1092ec4801bb3a263a277bc48d9b41eeb608216772f34cddc65e5e"},
+}
+
+
+def gemm_sources_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "fp8_quantized_linear_rms_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -83,6 +104,15 @@ def parse():
 def gemm_flops(M):
     """GEMM FLOPs of one step: both schemes x the four layers."""
     return 2 * sum(2 * M * N * K for _, K, N in LAYERS)
+
+
+def fused_gate_up_bytes(M):
+    """Algorithmic HBM bytes of the fused gate_up + SiLU*mul 1x128 quant launch:
+    e4m3 activations and weights and their fp32 block scales read once, e4m3
+    codes [M, I] and fp32 group scales written once."""
+    K, N2 = H, 2 * I
+    return (M * K + N2 * K + 4 * M * (K // 128) + 4 * (N2 // 128) * (K // 128)
+            + M * I + 4 * M * (I // 128))
 
 
 def quant_bytes(op, M, L, g):
@@ -537,9 +567,16 @@ def run_native(args, rank, world, local_rank):
                 "peak": round(hbm, 1), "unit": "GB/s", "frac": round(dunits / davg / 1e9 / hbm, 4),
                 "peak_source": hbm_src}
     roof["share_of_step"] = round(share[dom] / (sum(share)), 4)
-    roof["traffic"] = None
-    roof["traffic_note"] = ("DRAM read+write bytes per launch come from an ncu capture of the same "
-                            "kernel build, kept with the profiles; not measured in this run")
+    cap = TRAFFIC_CAPTURES.get((dname.split(" ")[0], M))
+    if cap and gemm_sources_digest() == cap["sources_sha256"]:
+        roof["traffic"] = cap["read"] + cap["write"]
+        roof["traffic_note"] = (f"ncu dram__bytes_read.sum {cap['read']} + dram__bytes_write.sum "
+                                f"{cap['write']} of one full-size launch of this kernel build (not "
+                                f"measured in this run); algorithmic bytes {fused_gate_up_bytes(M)}")
+    else:
+        roof["traffic"] = None
+        roof["traffic_note"] = ("no ncu capture of this kernel build at this size; DRAM bytes of the "
+                                "captured builds are in the profiles")
 
     line = {
         "metric": METRIC,
@@ -912,12 +949,45 @@ def run_sweep(args):
             for layer in ("qkv", "o", "gate_up", "down"):
                 K, N = sh[layer]
                 gemm_case(f"qwen3-32b {layer}", M, N, K, True)
+    def fused_gate_up_case(tag, M, K, N2):
+        """The gate_up GEMM with the SiLU*mul 1x128 quant in its epilogue, on the
+        bench step's kind of operands (heavy-tailed activations normalized and
+        quantized in 1x128 groups, N(0, 0.02) weights in 128x128 blocks), beside
+        the plain blockwise GEMM of the same operands (bf16 [gate | up] out)."""
+        x = bf16_rand((M, K), 5)
+        w = torch.ones(K, device=dev, dtype=torch.bfloat16)
+        a, sa = fq.fp8q_rmsnorm_quant(x, w, 1e-6, 128, scale_layout="group_major")
+        g = torch.Generator(device=dev).manual_seed(6)
+        wb = (torch.randn(N2, K, generator=g, device=dev) * 0.02).view(N2 // 128, 128, K // 128, 128)
+        sb = wb.abs().amax(dim=(1, 3)).clamp_min(1e-10) / 448.0
+        b = (wb / sb[:, None, :, None]).clamp(-448, 448).to(torch.float8_e4m3fn).view(N2, K)
+        b = fq.interleave_gate_up(b.view(torch.uint8)).view(torch.float8_e4m3fn)
+        sb = fq.interleave_gate_up(sb.contiguous(), block=1)
+        del wb, x
+        q = torch.empty((M, N2 // 2), dtype=torch.float8_e4m3fn, device=dev)
+        s = torch.empty((N2 // 256, M), dtype=torch.float32, device=dev)
+        y = torch.empty((M, N2), dtype=torch.bfloat16, device=dev)
+        flops = 2.0 * M * N2 * K
+        t_sq = timeit(lambda: fq.fp8q_scaled_mm_blockwise_silu_quant(a, b, sa, sb, a_scale_layout="group_major",
+                                                                      q=q, scales=s, scale_layout="group_major"))
+        t_bw = timeit(lambda: fq.fp8q_scaled_mm_blockwise(a, b, sa, sb, a_scale_layout="group_major", y=y))
+        emit({"op": "scaled_mm_blockwise_silu_quant", "shape": tag, "M": M, "N": N2, "K": K,
+              "fused_quant": "exact" if fq.fp8q_get_fused_quant_exact() else "fast",
+              "us": round(t_sq * 1e6, 2), "TFLOP/s": round(flops / t_sq / 1e12, 1),
+              "frac_fp8_peak": round(flops / t_sq / 1e12 / fp8_peak, 3),
+              "plain_blockwise_us": round(t_bw * 1e6, 2), "fused_over_plain": round(t_sq / t_bw, 3)})
+
     if which in ("prefill32b", "all"):
         sh = inp.linear_shapes(inp.QWEN3_32B)
         for bw in (False, True, "e8m0", "i8"):
             for layer in ("qkv", "o", "gate_up", "down"):
                 K, N = sh[layer]
                 gemm_case(f"qwen3-32b {layer}", 8192, N, K, bw)
+        K, N2 = sh["gate_up"]
+        fused_gate_up_case("qwen3-32b gate_up", 8192, K, N2)
+        fq.fp8q_set_fused_quant_exact(True)
+        fused_gate_up_case("qwen3-32b gate_up", 8192, K, N2)
+        fq.fp8q_set_fused_quant_exact(False)
     if which in ("e8m0", "all"):
         sh8, sh32 = inp.linear_shapes(inp.QWEN3_8B), inp.linear_shapes(inp.QWEN3_32B)
         for M in sweep_ms((1, 16, 64, 256, 1024, 4096)):
