@@ -2,7 +2,7 @@
 """Benchmark of the FP8 W8A8 linear path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--m M] [--impl reference]
-                    [--no-e8m0] [--sweep quant|gemm8b|decode32b|prefill32b|all|oracle]
+                    [--no-e8m0] [--sweep quant|gemm8b|decode32b|prefill32b|library|all|oracle]
 
 Workload: the linear stack of one Qwen3-32B-shaped decoder block in prefill
 (hidden 5120, intermediate 25600, 64 query / 8 kv heads of 128) on a batch of
@@ -93,7 +93,7 @@ def parse():
     ap.add_argument("--no-e8m0", action="store_true", help="skip the E8M0 (UE8M0) chain")
     ap.add_argument("--no-rope", action="store_true", help="skip timing fused_qk_norm_rope")
     ap.add_argument("--sweep", default=None,
-                    help="per-op timing instead of the step: quant, gemm8b, decode32b, prefill32b, "
+                    help="per-op timing instead of the step: quant, gemm8b, decode32b, prefill32b, library, "
                          "e8m0, all (GPU), or oracle (the CPU oracle, all host cores and one core)")
     ap.add_argument("--reps", type=int, default=50)
     ap.add_argument("--sweep-m", default=None,
@@ -976,6 +976,38 @@ def run_sweep(args):
               "us": round(t_sq * 1e6, 2), "TFLOP/s": round(flops / t_sq / 1e12, 1),
               "frac_fp8_peak": round(flops / t_sq / 1e12 / fp8_peak, 3),
               "plain_blockwise_us": round(t_bw * 1e6, 2), "fused_over_plain": round(t_sq / t_bw, 3)})
+
+    def library_case(tag, M, N, K, scales):
+        """torch._scaled_mm (the library's FP8 GEMM) on the same shape, as the
+        measured ceiling beside this library's scaled_mm: row-wise scales
+        (per token x per channel) or one scale per tensor."""
+        a = torch.randint(0, 126, (M, K), dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
+        b = torch.randint(0, 126, (N, K), dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
+        if scales == "rowwise":
+            sa = torch.rand((M, 1), device=dev) * 1e-3 + 1e-4
+            sb = torch.rand((1, N), device=dev) * 1e-3 + 1e-4
+        else:
+            sa = torch.tensor(1e-3, device=dev)
+            sb = torch.tensor(1e-3, device=dev)
+        fn = lambda: torch._scaled_mm(a, b.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
+        d = {"op": "torch._scaled_mm", "scales": scales, "shape": tag, "M": M, "N": N, "K": K}
+        try:
+            t = timeit(fn)
+        except Exception as e:                      # a scaling the installed library lacks
+            d["unavailable"] = f"{type(e).__name__}: {str(e)[:160]}"
+            emit(d)
+            return
+        flops = 2.0 * M * N * K
+        d.update({"us": round(t * 1e6, 2), "TFLOP/s": round(flops / t / 1e12, 1),
+                  "frac_fp8_peak": round(flops / t / 1e12 / fp8_peak, 3)})
+        emit(d)
+
+    if which in ("library", "all"):
+        sh = inp.linear_shapes(inp.QWEN3_32B)
+        for scales in ("rowwise", "tensor"):
+            for layer in ("qkv", "o", "gate_up", "down"):
+                K, N = sh[layer]
+                library_case(f"qwen3-32b {layer}", 8192, N, K, scales)
 
     if which in ("prefill32b", "all"):
         sh = inp.linear_shapes(inp.QWEN3_32B)
