@@ -978,18 +978,27 @@ def run_sweep(args):
               "plain_blockwise_us": round(t_bw * 1e6, 2), "fused_over_plain": round(t_sq / t_bw, 3)})
 
     def library_case(tag, M, N, K, scales):
-        """torch._scaled_mm (the library's FP8 GEMM) on the same shape, as the
-        measured ceiling beside this library's scaled_mm: row-wise scales
-        (per token x per channel) or one scale per tensor."""
+        """torch's FP8 GEMM (torch._scaled_mm / F.scaled_mm) on the same shape, as
+        the measured library figure beside this library's: row-wise scales (per
+        token x per channel), one scale per tensor, or 1x128 x 128x128 blocks."""
         a = torch.randint(0, 126, (M, K), dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
         b = torch.randint(0, 126, (N, K), dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
-        if scales == "rowwise":
+        if scales == "blockwise":
+            # 1x128 activation groups, 128x128 weight blocks, in the layouts the
+            # library takes: [M, K/128] and [K/128, N/128], both M-/K-block-major
+            import torch.nn.functional as F
+            sa = (torch.rand((K // 128, M), device=dev) * 1e-3 + 1e-4).t()
+            sb = (torch.rand((N // 128, K // 128), device=dev) * 1e-3 + 1e-4).t()
+            fn = lambda: F.scaled_mm(a, b.t(), sa, F.ScalingType.BlockWise1x128, sb,
+                                     F.ScalingType.BlockWise128x128, output_dtype=torch.bfloat16)
+        elif scales == "rowwise":
             sa = torch.rand((M, 1), device=dev) * 1e-3 + 1e-4
             sb = torch.rand((1, N), device=dev) * 1e-3 + 1e-4
+            fn = lambda: torch._scaled_mm(a, b.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
         else:
             sa = torch.tensor(1e-3, device=dev)
             sb = torch.tensor(1e-3, device=dev)
-        fn = lambda: torch._scaled_mm(a, b.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
+            fn = lambda: torch._scaled_mm(a, b.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
         d = {"op": "torch._scaled_mm", "scales": scales, "shape": tag, "M": M, "N": N, "K": K}
         try:
             t = timeit(fn)
@@ -1004,7 +1013,7 @@ def run_sweep(args):
 
     if which in ("library", "all"):
         sh = inp.linear_shapes(inp.QWEN3_32B)
-        for scales in ("rowwise", "tensor"):
+        for scales in ("rowwise", "tensor", "blockwise"):
             for layer in ("qkv", "o", "gate_up", "down"):
                 K, N = sh[layer]
                 library_case(f"qwen3-32b {layer}", 8192, N, K, scales)
