@@ -63,9 +63,11 @@ NOMINAL_FP8_TFLOPS = 4500.0      # dense e4m3 tensor peak on the data sheet, for
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the step's dominant kernel, from one ncu capture of the full-size launch
-# (profiles/gemm_blockwise_silu_quant_qwen3_32b_gate_up.md gives the
-# command).  It holds for the GEMM sources it was taken on: the line reports
-# it only while their SHA-256 digest is unchanged, else null.
+# (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k regex:gemm_
+# -s 6 -c 1` on `bench.py --steps 1 --warmup 3 --no-e8m0 --no-rope`, the
+# seventh GEMM launch being the fused gate_up).  It holds for the GEMM sources
+# it was taken on: the line reports it only while their SHA-256 digest is
+# unchanged, else null.
 GEMM_SOURCES = ("fp8q_gemm.cu", "fp8q_sm100.cuh", "fp8q_quant_math.cuh", "fp8q_common.cuh")
 TRAFFIC_CAPTURES = {
     ("scaled_mm_blockwise_silu_quant", 8192): {
