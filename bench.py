@@ -33,9 +33,10 @@ their own streams overlapping the neighbouring steps' kernels
 GEMM and quant launch against the measured peaks.  `e8m0_chain` times the
 blockwise stack again with packed UE8M0 scales and the block-scaled GEMM;
 `qk_norm_rope` times the attention-side fused op on the step's qkv output.
-The quant ops run in the library's default arithmetic (per-token SiLU*mul
-with fast y and exact scales, the others bit-exact; fp8q_set_fused_quant_exact
-makes all of them bit-exact).
+The quant ops run in the library's default arithmetic: the per-token SiLU*mul
+quant and the SiLU*mul quant fused into the gate_up GEMM keep exact scales
+with codes within the fused tolerance, the others are bit-exact;
+fp8q_set_fused_quant_exact makes all of them bit-exact.
 `--impl reference` times the CPU oracle on a bounded sample of the workload.
 """
 from __future__ import annotations
@@ -152,8 +153,9 @@ def workload_config(M, n):
             "parallelism": f"replicas{n}" if n > 1 else "single-gpu",
             "l2": "flushed between timed steps (256 MiB write); the step's weights "
                   "(0.98 GB of e4m3) exceed L2 as well",
-            "fused_quant": "library default: per-token SiLU*mul with fast y and exact scales "
-                           "(codes within the fused tolerance), the other quant ops bit-exact"}
+            "fused_quant": "library default (fast mode): the per-token SiLU*mul quant and the "
+                           "SiLU*mul quant fused into the gate_up GEMM keep exact scales, codes "
+                           "within the fused tolerance; the other quant ops bit-exact"}
 
 
 def load_peaks():
