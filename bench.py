@@ -66,23 +66,29 @@ NOMINAL_FP8_TFLOPS = 4500.0      # dense e4m3 tensor peak on the data sheet, for
 # the step's dominant kernel, from one ncu capture of the full-size launch
 # (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k regex:gemm_
 # -s 6 -c 1` on `bench.py --steps 1 --warmup 3 --no-e8m0 --no-rope`, the
-# seventh GEMM launch being the fused gate_up).  It holds for the GEMM sources
-# it was taken on: the line reports it only while their SHA-256 digest is
-# unchanged, else null.
+# seventh GEMM launch being the fused gate_up).  It holds for the GEMM code
+# it was taken on: the line reports it only while the SHA-256 digest of that
+# code (comments and blank space dropped) is unchanged, else null.
 GEMM_SOURCES = ("fp8q_gemm.cu", "fp8q_sm100.cuh", "fp8q_quant_math.cuh", "fp8q_common.cuh")
 TRAFFIC_CAPTURES = {
     ("scaled_mm_blockwise_silu_quant", 8192): {
         "read": 374152960, "write": 211215616,
-        "sources_sha256": "e7381c61eb1092ec4801bb3a263a277bc48d9b41eeb608216772f34cddc65e5e"},
+        "sources_sha256": "b1260ac965384b5946926603b737a6d07914143869a423c8cfd65d10016c7530"},
 }
 
 
 def gemm_sources_digest():
+    """SHA-256 of the GEMM sources' code: comments and blank space dropped, so
+    that an edit of a comment keeps a capture valid and any code edit does not."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in GEMM_SOURCES:
-        with open(os.path.join(ROOT, "fp8_quantized_linear_rms_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "fp8_quantized_linear_rms_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)    # block comments
+        src = re.sub(r"//[^\n]*", " ", src)                  # line comments
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()
 
 

@@ -245,7 +245,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // holds gate outputs [128 tb, 128 tb + 128) in columns 0-127 and the matching
 // up outputs in columns 128-255.  Each epilogue thread owns 64 gate and the
 // matching 64 up columns of its row; after the K loop it rounds both to bf16
-// as the GEMM emits them, applies the exact SiLU*mul of the quant kernels,
+// as the GEMM emits them, applies the SiLU*mul of the quant kernels (exact,
+// or in the fast mode exact wherever a value can decide the group amax),
 // takes the 1x128 group amax with its partner thread (the other column
 // slice, same row) through shared memory and writes e4m3 codes and the
 // group's scale.  The 2I-wide bf16 intermediate is never written.
