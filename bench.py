@@ -73,7 +73,7 @@ GEMM_SOURCES = ("fp8q_gemm.cu", "fp8q_sm100.cuh", "fp8q_quant_math.cuh", "fp8q_c
 TRAFFIC_CAPTURES = {
     ("scaled_mm_blockwise_silu_quant", 8192): {
         "read": 374152960, "write": 211215616,
-        "sources_sha256": "b1260ac965384b5946926603b737a6d07914143869a423c8cfd65d10016c7530"},
+        "sources_sha256": "8cfca17b2a9d48b32d4f7278dc1d43b35810671a4314e026bcbe53cba4d81ac5"},
 }
 
 

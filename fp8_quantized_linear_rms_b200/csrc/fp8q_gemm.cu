@@ -139,7 +139,12 @@ struct Cfg {
   // 10 in all: 168 registers a thread), so it reads 8 columns at a time.
   static constexpr int CHUNK = BW ? (CPT >= 128 ? (kRegSplit && BN == 256 && !SWAP ? 32 : 8) : 16)
                                   : (CPT < 32 ? 16 : 32);
-  static constexpr int NBUF = (BW && BN < 256) ? 4 : 2;    // TMEM accumulator buffers
+  // TMEM accumulator buffers.  The E8M0 kernel's 256-column tile keeps one
+  // (two would leave no columns for the scale factors): its tile epilogue is
+  // not overlapped with the next tile's MMAs, and still measured 5-8% faster
+  // than 224-column tiles with two buffers, the block-scaled MMA's cost per
+  // instruction being spread over more columns.
+  static constexpr int NBUF = (MX && BN == 256) ? 1 : (BW && BN < 256) ? 4 : 2;
   static constexpr int SF_COL0 = NBUF * BN;                 // first scale-factor column (MX)
   static constexpr int TMEM_NEED = NBUF * BN + (MX ? STAGES * SF_COLS : 0);
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
@@ -361,8 +366,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
         uint32_t d = tmem_base;
         int buf = 0;
         if (!BW) {
-          buf = t & 1;
-          if (!mbar_wait(&tempty[buf], ((t >> 1) & 1) ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          buf = t % NB;
+          if (!mbar_wait(&tempty[buf], ((t / NB) & 1) ^ 1u, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           d = tmem_base + buf * BN;
         }
@@ -676,7 +681,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
         // every chunk (one load per 32 columns, issued before the wait), and the
         // products broadcast it with a shuffle.
         constexpr int NCH = C::CPT / C::CHUNK;
-        const int buf = t & 1;
+        const int buf = t % NB;
         float srow = 1.0f;
         float colsc[NCH];
         if constexpr (!MX) {
@@ -689,7 +694,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, BW, MX, I8>::THREADS, 1)
             else colsc[j] = (lane < C::CHUNK && b_idx < p.M) ? __ldg(p.sa + b_idx * p.sa_sm) : 0.0f;
           }
         }
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[buf], (t >> 1) & 1, abort_flag, p.status))) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[buf], (t / NB) & 1, abort_flag, p.status))) {
           ok = false;
           break;
         }
@@ -1542,10 +1547,10 @@ bool variant_supported(const fp8q_gemm_variant& v, int blockwise) {
   if (v.block_n == kDecodeMaxM) return blockwise <= 1 && v.swap_ab == 1 && v.split_k == 1 && !v.cta_pair;
   if (blockwise == 3) blockwise = 0;   // int8: the per-token scheme's variants
   if (blockwise == 2) {
-    // single CTAs only; 224-column tiles leave TMEM room for the scale factors
+    // single CTAs only; 224- and 256-column tiles (one accumulator buffer at 256)
     if (v.cta_pair || v.split_k < 0 || v.split_k > 64) return false;
     if (v.swap_ab) return v.block_n == 16 || v.block_n == 32 || v.block_n == 64 || v.block_n == 128;
-    return v.block_n == 128 || v.block_n == 224;
+    return v.block_n == 128 || v.block_n == 224 || v.block_n == 256;
   }
   // (pairs: blockwise with 128-column tiles -- four accumulator buffers --,
   // per token with 128 or 256)
@@ -1667,9 +1672,8 @@ fp8q_gemm_variant pick_variant(int64_t M, int64_t N, int64_t K, int blockwise,
     fp8q_gemm_variant v = auto_variant(M, N, K, 0);
     if (v.block_n == kDecodeMaxM) v = heuristic_variant(M, N, K, 0, false);
     if (blockwise == 3) return v;
-    // E8M0: single CTAs, with 224-column tiles where that takes 256-column tiles
-    if (v.cta_pair) v = fp8q_gemm_variant{0, 1, 224, 0};
-    if (!v.swap_ab && v.block_n == 256) v.block_n = 224;
+    // E8M0: single CTAs (a CTA-pair choice becomes 128x256 single-CTA tiles)
+    if (v.cta_pair) v = fp8q_gemm_variant{0, 1, 256, 0};
     return v;
   }
   return auto_variant(M, N, K, blockwise);
@@ -1779,6 +1783,7 @@ fp8q_status run_gemm(const void* a_q, const void* b_q, GemmArgs& p, const Plan& 
     p.rows_b = p.N;
     if (bn == 128) return launch_gemm<128, false, false, true>(a_q, b_q, p, stream);
     if (bn == 224) return launch_gemm<224, false, false, true>(a_q, b_q, p, stream);
+    if (bn == 256) return launch_gemm<256, false, false, true>(a_q, b_q, p, stream);
     return FP8Q_ERR_UNSUPPORTED;
   }
   if (pl.v.cta_pair) {

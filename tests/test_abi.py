@@ -208,11 +208,13 @@ def test_variant_selection_host_logic():
 
 
 def test_e8m0_variant_selection_host_logic():
-    # The E8M0 GEMM follows the per-token scheme's choice, single CTAs only,
-    # 224-column tiles where that scheme takes 256-column ones.
+    # The E8M0 GEMM follows the per-token scheme's choice, single CTAs only
+    # (128x256 tiles where that scheme takes CTA pairs).
     for M, N, K in [(8192, 51200, 5120), (2048, 24576, 4096), (4096, 6144, 4096)]:
         v = fq.fp8q_select_gemm_variant(M, N, K, 2)
-        assert v["cta_pair"] == 0 and v["swap_ab"] == 0 and v["block_n"] in (128, 224), v
+        pt = fq.fp8q_select_gemm_variant(M, N, K, False)
+        assert v["cta_pair"] == 0 and v["swap_ab"] == 0 and v["block_n"] in (128, 256), v
+        assert v["block_n"] == (256 if pt["cta_pair"] else pt["block_n"]), (v, pt)
     for M in (16, 32, 64):
         v = fq.fp8q_select_gemm_variant(M, 10240, 5120, 2)
         pt = fq.fp8q_select_gemm_variant(M, 10240, 5120, False)

@@ -5,7 +5,7 @@ bit: codes and E8M0 scale bytes (the fused ops within their tolerance, which
 for bytes means identical).  The block-scaled GEMM (tcgen05 kind::mxf8f6f4
 with hardware block scaling) must meet the GEMM tolerance against the fp64
 reference on the decoded scales, for every variant it runs (Swap-AB tiles,
-128- and 224-column tiles, split-K, stream-K) on shapes with ragged M and N
+128-, 224- and 256-column tiles, split-K, stream-K) on shapes with ragged M and N
 tails, and on the config shapes through the automatic variant choice.
 """
 import numpy as np
@@ -59,7 +59,7 @@ def test_e8m0_gemm_one_tile():
     gemm_tolerance_check(y, y_ref, ad, "e8m0 one tile")
 
 
-E8_VARIANTS = [(0, 128), (0, 224), (1, 16), (1, 32), (1, 64), (1, 128)]
+E8_VARIANTS = [(0, 128), (0, 224), (0, 256), (1, 16), (1, 32), (1, 64), (1, 128)]
 
 
 @pytest.mark.parametrize("split", [0, 1, 3])
