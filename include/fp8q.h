@@ -311,8 +311,9 @@ FP8Q_API fp8q_status fp8q_scaled_mm_blockwise_silu_quant(
  *   A byte of 255 (E8M0 NaN) makes the affected outputs NaN.  N and K
  *   multiples of 128; other arguments as in fp8q_scaled_mm_blockwise, with
  *   fp8q_workspace_bytes(M, N, K, 2).  Variants: Swap-AB tiles (block_n
- *   16..128), or 128-row tiles of block_n 128 or 224 (224 leaves TMEM room
- *   for the scale factors next to two accumulator buffers); no CTA pairs.
+ *   16..128), or 128-row tiles of block_n 128, 224 (two accumulator buffers
+ *   next to the scale factors in TMEM) or 256 (one buffer; the automatic
+ *   choice for wide tiles); no CTA pairs.
  */
 FP8Q_API fp8q_status fp8q_scaled_mm_blockwise_e8m0(const void* a_q, const void* b_q,
                                                    const uint8_t* a_sf, int64_t as_stride_m,
@@ -409,7 +410,8 @@ FP8Q_API size_t fp8q_workspace_bytes(int64_t M, int64_t N, int64_t K, int blockw
  * cta_pair = 1 runs each 256-row tile on a cluster of two CTAs (two SMs)
  * sharing one tcgen05 .cta_group::2 MMA, each SM staging half of the B tile
  * (only with swap_ab = 0 and split_k = 1; block_n 128, or 256 for the
- * per-token scheme).  block_n 224 is the E8M0 GEMM's wide tile (no swap). */
+ * per-token scheme).  block_n 224 (and 256 with one accumulator buffer) are
+ * the E8M0 GEMM's wide tiles (no swap). */
 typedef struct {
     int swap_ab;
     int split_k;
