@@ -12,7 +12,9 @@ Rebuild the library afterwards (``python fp8_quantized_linear_rms_b200/build.py`
 Timing: CUDA events around a run of back-to-back calls, each on its own copy
 of the weight matrix, with enough copies (384 MiB in all, 2 to 64 of them) that every
 call reads its weights from HBM as a model's successive layers do; the time
-per call is the median over trials of the run's mean.
+per call is the median over trials of the run's mean.  Each trial times every
+candidate once, in an order rotated from trial to trial, so that the GPU's
+clock under its power cap drifts over all candidates alike.
 
 Where variants come within 2% of the fastest, the simplest wins, in this
 order: whole-K tiles, split-K, stream-K (they need no / a fixed / a larger
@@ -120,6 +122,20 @@ def _time_run(fns, trials: int) -> float:
     return statistics.median(per)
 
 
+def _round_robin(runs, reps: int, time_one) -> dict:
+    """Median over `reps` trials of time_one(v, fns) for every (v, fns) in runs.
+    Trial r goes round the candidates starting at candidate r mod len(runs), so
+    that every candidate is timed at every point of the GPU's warming under its
+    power cap (timing one candidate's trials after another's let the later one
+    run at a lower clock)."""
+    per = {v: [] for v, _ in runs}
+    for r in range(reps):
+        k = r % len(runs)
+        for v, fns in runs[k:] + runs[:k]:
+            per[v].append(time_one(v, fns))
+    return {v: statistics.median(ts) for v, ts in per.items()}
+
+
 def tune(reps: int = 5, shapes=SHAPES, buckets=M_BUCKETS, log=print):
     dev = torch.device("cuda", torch.cuda.current_device())
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -139,21 +155,32 @@ def tune(reps: int = 5, shapes=SHAPES, buckets=M_BUCKETS, log=print):
             sa_grp = torch.rand((K // 128, M), device=dev, generator=g) * 1e-3
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             for bw in (0, 1):
-                times = {}
+                # Each candidate's calls, with the workspace its variant needs.
+                runs = []
                 for v in candidates(M, N, K, sms, bool(bw)):
                     fq.fp8q_force_gemm_variant(*v)
                     try:
                         ws = fq.make_workspace(M, N, K, bool(bw), dev)
-                        if bw:
-                            fns = [lambda b=b: fq.fp8q_scaled_mm_blockwise(
-                                a, b, sa_grp, sb_bl, a_scale_layout="group_major", y=y,
-                                workspace=ws) for b in bs]
-                        else:
-                            fns = [lambda b=b: fq.fp8q_scaled_mm(a, b, sa_tok, sb_ch, y=y,
-                                                                 workspace=ws) for b in bs]
-                        times[v] = _time_run(fns, reps)
                     finally:
                         fq.fp8q_force_gemm_variant()
+                    if bw:
+                        fns = [lambda b=b, ws=ws: fq.fp8q_scaled_mm_blockwise(
+                            a, b, sa_grp, sb_bl, a_scale_layout="group_major", y=y,
+                            workspace=ws) for b in bs]
+                    else:
+                        fns = [lambda b=b, ws=ws: fq.fp8q_scaled_mm(a, b, sa_tok, sb_ch, y=y,
+                                                                    workspace=ws) for b in bs]
+                    runs.append((v, fns))
+
+                def time_one(v, fns):
+                    fq.fp8q_force_gemm_variant(*v)
+                    try:
+                        return _time_run(fns, 1)
+                    finally:
+                        fq.fp8q_force_gemm_variant()
+
+                times = _round_robin(runs, reps, time_one)
+                del runs
                 best_t = min(times.values())
                 best = min((v for v, t in times.items() if t <= best_t * TIE),
                            key=lambda v: (_complexity(v), times[v]))

@@ -74,3 +74,17 @@ def test_written_table_parses_back(tmp_path):
     tune.write_table(rows, path, device="NVIDIA B200")
     parsed = [tuple(int(x) for x in m.groups()) for m in map(ROW.match, open(path)) if m]
     assert parsed == [(r["blockwise"], r["m_max"], r["N"], r["K"], *r["variant"]) for r in rows]
+
+
+def test_trials_go_round_the_candidates():
+    # every trial times each candidate once, starting one candidate further
+    # along each time; the result is each candidate's median
+    runs = [("a", None), ("b", None), ("c", None)]
+    order, clock = [], iter(range(100))
+    def time_one(v, fns):
+        order.append(v)
+        return {"a": 10.0, "b": 20.0, "c": 30.0}[v] + next(clock) * 0.001
+    got = tune._round_robin(runs, 4, time_one)
+    assert order == ["a", "b", "c", "b", "c", "a", "c", "a", "b", "a", "b", "c"]
+    assert set(got) == {"a", "b", "c"}
+    assert 10 < got["a"] < 11 and 20 < got["b"] < 21 and 30 < got["c"] < 31
